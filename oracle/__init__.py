@@ -1,0 +1,166 @@
+"""ctypes binding of the C oracle (oracle/svo.c).
+
+TEST INFRASTRUCTURE ONLY.  The oracle is a plain double-precision CPU
+restatement of the speculative-decoding verification rule.  Only the tests,
+the smoke check and the benchmark's CPU-baseline leg may import this package;
+the product library never does, and it shares no code with it.
+
+Arrays are numpy: fp32 logits as ``float32``, bf16 logits as their raw
+``uint16`` bit patterns.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+SVO_F32, SVO_BF16 = 0, 1
+SVO_STOCHASTIC, SVO_GREEDY, SVO_SAGUARO = 0, 1, 2
+
+FLAG_ACCEPT_NEAR_TIE = 1 << 0
+FLAG_RACE_NEAR_TIE = 1 << 1
+FLAG_RESIDUAL_EMPTY = 1 << 2
+FLAG_BAD_TOKEN = 1 << 8
+FLAG_BAD_ROW_D = 1 << 9
+FLAG_NONFINITE = 1 << 10
+FLAG_BAD_PARAM = 1 << 11
+FLAG_NEAR_TIE = FLAG_ACCEPT_NEAR_TIE | FLAG_RACE_NEAR_TIE
+FLAG_ERRORS = FLAG_BAD_TOKEN | FLAG_BAD_ROW_D | FLAG_NONFINITE | FLAG_BAD_PARAM
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [
+        ("temperature_per_req", ctypes.c_void_p),
+        ("mode_per_req", ctypes.c_void_p),
+        ("saguaro_k", ctypes.c_int),
+        ("saguaro_c", ctypes.c_double),
+        ("request_offset", ctypes.c_uint32),
+    ]
+
+
+_lib = None
+
+
+def _declare(L):
+    u32p = ctypes.POINTER(ctypes.c_uint32)
+    L.svo_philox4x32_10.argtypes = [u32p, u32p, u32p]
+    L.svo_philox4x32_10.restype = None
+    L.svo_accept_uniform.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32]
+    L.svo_accept_uniform.restype = ctypes.c_double
+    L.svo_race_exponential.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32]
+    L.svo_race_exponential.restype = ctypes.c_double
+    L.svo_row_lse.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_double]
+    L.svo_row_lse.restype = ctypes.c_double
+    L.svo_row_argmax.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int]
+    L.svo_row_argmax.restype = ctypes.c_int
+    L.svo_verify.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_float, ctypes.c_int, ctypes.c_uint64, ctypes.POINTER(_Params),
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int,
+    ]
+    L.svo_verify.restype = ctypes.c_int
+    L.svo_has_openmp.argtypes = []
+    L.svo_has_openmp.restype = ctypes.c_int
+    return L
+
+
+def lib():
+    """The oracle library (built from oracle/svo.c on first use)."""
+    global _lib
+    if _lib is None:
+        _lib = _declare(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+def load_variant(path):
+    """Load another build of the same source (the tests use this to check that
+    their pins reject deliberately broken copies of the oracle)."""
+    return _declare(ctypes.CDLL(path))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(a):
+    if a.dtype == np.float32:
+        return SVO_F32
+    if a.dtype == np.uint16:
+        return SVO_BF16
+    raise TypeError(f"logits must be float32 or uint16 (bf16 bits), got {a.dtype}")
+
+
+def philox4x32_10(ctr, key, L=None):
+    c = (ctypes.c_uint32 * 4)(*[int(v) & 0xFFFFFFFF for v in ctr])
+    k = (ctypes.c_uint32 * 2)(*[int(v) & 0xFFFFFFFF for v in key])
+    o = (ctypes.c_uint32 * 4)()
+    (L or lib()).svo_philox4x32_10(c, k, o)
+    return [int(v) for v in o]
+
+
+def accept_uniform(seed, g, d, L=None):
+    return (L or lib()).svo_accept_uniform(int(seed), int(g), int(d))
+
+
+def race_exponential(seed, g, x, L=None):
+    return (L or lib()).svo_race_exponential(int(seed), int(g), int(x))
+
+
+def row_lse(row, T, L=None):
+    row = np.ascontiguousarray(row)
+    return (L or lib()).svo_row_lse(_ptr(row), row.shape[-1], _dtype_code(row), float(T))
+
+
+def row_argmax(row, L=None):
+    row = np.ascontiguousarray(row)
+    return (L or lib()).svo_row_argmax(_ptr(row), row.shape[-1], _dtype_code(row))
+
+
+def has_openmp():
+    return bool(lib().svo_has_openmp())
+
+
+def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SVO_STOCHASTIC,
+           seed=0, temperature_per_req=None, mode_per_req=None, saguaro_k=5,
+           saguaro_c=0.5, request_offset=0, nthreads=1, L=None):
+    """Run the oracle on host arrays.
+
+    target [B, D_max+1, V], draft [B, D_max, V] (or None when all greedy),
+    tokens [B, D_max] int32, row_D [B] int32 or None.
+    Returns dict(tokens [B, D_max+1] int32, accept_len [B] int32,
+    flags [B] uint32, row_lse [B, 2*D_max+1] float64).
+    """
+    target = np.ascontiguousarray(target)
+    B, Dp1, V = target.shape
+    D_max = Dp1 - 1
+    dt = _dtype_code(target)
+    if draft is not None:
+        draft = np.ascontiguousarray(draft)
+        assert draft.dtype == target.dtype and draft.shape == (B, D_max, V)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, D_max)
+    if row_D is not None:
+        row_D = np.ascontiguousarray(row_D, dtype=np.int32).reshape(B)
+    tpr = None if temperature_per_req is None else np.ascontiguousarray(
+        temperature_per_req, dtype=np.float32).reshape(B)
+    mpr = None if mode_per_req is None else np.ascontiguousarray(
+        mode_per_req, dtype=np.int8).reshape(B)
+    p = _Params(
+        temperature_per_req=None if tpr is None else tpr.ctypes.data,
+        mode_per_req=None if mpr is None else mpr.ctypes.data,
+        saguaro_k=int(saguaro_k), saguaro_c=float(saguaro_c),
+        request_offset=int(request_offset),
+    )
+    out_tokens = np.empty((B, D_max + 1), dtype=np.int32)
+    out_al = np.empty((B,), dtype=np.int32)
+    out_flags = np.empty((B,), dtype=np.uint32)
+    out_lse = np.empty((B, 2 * D_max + 1), dtype=np.float64)
+    rc = (L or lib()).svo_verify(
+        _ptr(target), _ptr(draft), _ptr(tokens), _ptr(row_D), B, D_max, V, dt,
+        float(temperature), int(mode), int(seed) & (2**64 - 1), ctypes.byref(p),
+        _ptr(out_tokens), _ptr(out_al), _ptr(out_flags), _ptr(out_lse), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (rc={rc})")
+    return dict(tokens=out_tokens, accept_len=out_al, flags=out_flags, row_lse=out_lse)

@@ -1,0 +1,100 @@
+/*
+ * svo.h -- the ORACLE for speculative-decoding verification.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is a plain, slow, single-threaded (optionally
+ * OpenMP-over-requests) CPU restatement of the verification rule in double
+ * precision.  Only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg may load it.  It shares no code, header, table or constant
+ * generator with the CUDA library, and it never calls it.
+ *
+ * Sources (cited by page title and section):
+ *   [Sonar]  "Accélérer Sonar par la Spéculation" (Perplexity), sections
+ *            "Décodage spéculatif", "Cible-Brouillon".
+ *   [SSD]    "Speculative Speculative Decoding – асинхронизируй это." (x0ct.com),
+ *            the numbered speculative-decoding rule (items 1-3 and the closing
+ *            remark that the output is distributed like p) and the numbered
+ *            saguaro recipe (items 1-3).
+ *   [NV5]    "NVIDIA: öt irányelv gyorsíthatja az LLM-ek spekulatív
+ *            dekódolását", section "Mit csinál a spekulatív dekódolás?"
+ *            (accept in order until the first mismatch; AL in [1, 1+D]).
+ *   Philox4x32-10: Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+ *            Easy as 1, 2, 3", SC'11 (the published round function, multipliers
+ *            and Weyl key schedule).
+ *
+ * Readings taken where the pages are silent or garbled are listed in the
+ * project's design notes and repeated at the function that applies them.
+ */
+#ifndef SVO_H
+#define SVO_H
+#include <stdint.h>
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { SVO_F32 = 0, SVO_BF16 = 1 };
+enum { SVO_STOCHASTIC = 0, SVO_GREEDY = 1, SVO_SAGUARO = 2 };
+
+/* per-request flag bits written to out_flags[b] */
+enum {
+  SVO_FLAG_ACCEPT_NEAR_TIE = 1u << 0, /* some tested position had |u - a| < 1e-5 */
+  SVO_FLAG_RACE_NEAR_TIE = 1u << 1,   /* top-2 race keys closer than 1e-6 (log space) */
+  SVO_FLAG_RESIDUAL_EMPTY = 1u << 2,  /* {p > q} was empty; sampled from p instead */
+  SVO_FLAG_BAD_TOKEN = 1u << 8,       /* a tested draft token outside [0, V) */
+  SVO_FLAG_BAD_ROW_D = 1u << 9,       /* row_D[b] outside [0, D_max] */
+  SVO_FLAG_NONFINITE = 1u << 10       /* NaN or +inf in a needed row, or a row all -inf */
+};
+
+/* Published Philox4x32-10 bijection: counter ctr[4], key key[2] -> out[4]. */
+void svo_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+
+/* Accept uniform u for (seed, global request g, position d): word 0 of
+ * Philox(key = seed, counter = (d, g, 0, 0)), top 24 bits, times 2^-24. */
+double svo_accept_uniform(uint64_t seed, uint32_t g, uint32_t d);
+
+/* Race exponential E for (seed, global request g, token x):
+ * word (x mod 4) of Philox(key = seed, counter = (x / 4, g, 1, 0)) = o,
+ * W = (o + 1/2) 2^-32, E = -ln(1 - W). */
+double svo_race_exponential(uint64_t seed, uint32_t g, uint32_t x);
+
+/* Log-sum-exp of one row at temperature T: ln sum_x exp(z_x / T), double.
+ * Returns -inf for a row whose every entry is -inf. */
+double svo_row_lse(const void* row, int V, int dtype, double T);
+
+/* Lowest index of the largest raw logit. */
+int svo_row_argmax(const void* row, int V, int dtype);
+
+typedef struct {
+  const float* temperature_per_req; /* [B] or NULL */
+  const int8_t* mode_per_req;       /* [B] or NULL: per-request mode overrides */
+  int saguaro_k;                    /* <= 0 -> 5 */
+  double saguaro_c;                 /* <= 0 -> 0.5 */
+  uint32_t request_offset;          /* global index of request 0 (sharding) */
+} svo_params;
+
+/*
+ * The whole verification step for B requests.
+ *   target  [B, D_max+1, V] dtype;  draft [B, D_max, V] dtype (may be NULL only
+ *   if every request is greedy);  tokens [B, D_max];  row_D [B] or NULL (= D_max).
+ * Outputs (all caller-owned, host):
+ *   out_tokens [B, D_max+1], out_accept_len [B], out_flags [B] (may be NULL),
+ *   out_row_lse [B, 2*D_max+1] (may be NULL): slots 0..D_max are target rows,
+ *   slots D_max+1 .. 2*D_max draft rows; NaN where a row is not used.
+ * nthreads: 1 = plain single-threaded loop; > 1 = the same loop split over
+ * requests with OpenMP when the library was built with it.
+ * Returns 0, or -1 for invalid arguments.
+ */
+int svo_verify(const void* target, const void* draft, const int32_t* tokens,
+               const int32_t* row_D, int B, int D_max, int V, int dtype,
+               float temperature, int mode, uint64_t seed, const svo_params* params,
+               int32_t* out_tokens, int32_t* out_accept_len, uint32_t* out_flags,
+               double* out_row_lse, int nthreads);
+
+/* 1 when built with OpenMP, else 0. */
+int svo_has_openmp(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

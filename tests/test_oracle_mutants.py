@@ -1,0 +1,260 @@
+"""The pins must reject a broken oracle.
+
+Each case plants one plausible mistake (a dropped term, a wrong sign, a wrong
+index, a transposed operand) in a temporary copy of oracle/svo.c, builds it,
+and checks that at least one of the pin checks below fails on it.  The
+committed oracle itself is never modified.  The checks are smaller versions
+of the pins in test_oracle_lse.py, test_oracle_philox.py and
+test_oracle_rule.py."""
+import math
+import os
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+
+from svtest_util import bf16_bits, chi2_pvalue, sample_categorical, sample_rows, softmax, within_sigma
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "svo.c")
+
+MUTANTS = {
+    "lse_drops_temperature": ("s += exp(z / T - mT);", "s += exp(z - mT);"),
+    "lse_wrong_offset": ("return mT + log(s);", "return m + log(s);"),
+    "ratio_transposed": ("acc = fmin(1.0, exp(lp - lq));", "acc = fmin(1.0, exp(lq - lp));"),
+    "accept_compare_flipped": ("if (!(u < acc)) {", "if (!(u > acc)) {"),
+    "accept_scan_no_stop": ("        n = d;\n        break;\n      }\n    }\n\n    double gap",
+                            "        n = d;\n      }\n    }\n\n    double gap"),
+    "uniform_wrong_scale": ("return ldexp((double)(out[0] >> 8), -24);",
+                            "return ldexp((double)(out[0] >> 9), -24);"),
+    "residual_drops_q": ("lr = lp + log(-expm1(lq - lp));", "lr = lp;"),
+    "residual_wrong_support": ("if (!(lp > lq)) continue;", "if (!(lp < lq)) continue;"),
+    "race_noise_sign": ("double key = lr - log(svo_race_exponential",
+                        "double key = lr + log(svo_race_exponential"),
+    "race_noise_shared_lane": ("ldexp((double)out[x & 3u] + 0.5, -32)",
+                               "ldexp((double)out[0] + 0.5, -32)"),
+    "race_wrong_row": ("const void* trow_n = row_ptr(a->target, trow0 + n, V, dt);",
+                       "const void* trow_n = row_ptr(a->target, trow0 + Db, V, dt);"),
+    "philox_drops_key": ("uint32_t n0 = hi1 ^ c1 ^ k0;", "uint32_t n0 = hi1 ^ c1;"),
+    "philox_two_rounds": ("for (int round = 0; round < 10; ++round)",
+                          "for (int round = 0; round < 2; ++round)"),
+    "greedy_wrong_row": ("int am = svo_row_argmax(row_ptr(a->target, trow0 + d, V, dt), V, dt);",
+                         "int am = svo_row_argmax(row_ptr(a->target, trow0 + d + 1, V, dt), V, dt);"),
+    "argmax_last_tie": ("    if (z > bz) {\n      bz = z;\n      best = x;",
+                        "    if (z >= bz) {\n      bz = z;\n      best = x;"),
+    "saguaro_no_renormalise": ("return lq + (in_k ? q->ln_c : 0.0) - q->ln_Z;",
+                               "return lq + (in_k ? q->ln_c : 0.0);"),
+    "saguaro_topk_last_tie": ("if (best < 0 || z > bz) {", "if (best < 0 || z >= bz) {"),
+}
+
+
+def tile(a, B):
+    return np.ascontiguousarray(np.broadcast_to(a, (B,) + a.shape))
+
+
+# ------------------------------------------------------------ pin checks
+
+
+def check_lse(svo, L):
+    for V, T in ((7, 0.7), (1024, 1.0), (300, 2.5)):
+        if abs(svo.row_lse(np.full(V, 1.375, np.float32), T, L=L) - (1.375 / T + math.log(V))) > 1e-9:
+            return False
+    vals = np.array([-2.5] * 3 + [4.0] * 5, np.float32)
+    expect = -2.5 / 0.7 + math.log(3 + 5 * math.exp(6.5 / 0.7))
+    return abs(svo.row_lse(vals, 0.7, L=L) - expect) < 1e-9
+
+
+def check_argmax(svo, L):
+    rng = np.random.default_rng(11)
+    for _ in range(30):
+        z = np.round(rng.standard_normal(200) * 2).astype(np.float32)
+        if svo.row_argmax(z, L=L) != int(np.argmax(z)):
+            return False
+    return True
+
+
+def check_avalanche(svo, L):
+    rng = np.random.default_rng(1)
+    d = []
+    for _ in range(100):
+        ctr = [int(v) for v in rng.integers(0, 2**32, 4, dtype=np.uint64)]
+        key = [int(v) for v in rng.integers(0, 2**32, 2, dtype=np.uint64)]
+        for w in range(6):
+            c2, k2 = list(ctr), list(key)
+            if w < 4:
+                c2[w] ^= 1 << int(rng.integers(0, 32))
+            else:
+                k2[w - 4] ^= 1 << int(rng.integers(0, 32))
+            a = svo.philox4x32_10(ctr, key, L=L)
+            b = svo.philox4x32_10(c2, k2, L=L)
+            d.append(sum(bin(x ^ y).count("1") for x, y in zip(a, b)))
+    d = np.array(d, float)
+    return abs(d.mean() - 64) < 4 * 5.66 / math.sqrt(len(d)) and d.min() > 30
+
+
+def check_uniform(svo, L):
+    from scipy import stats
+    u = np.array([svo.accept_uniform(9, g, dd, L=L) for g in range(1500) for dd in range(4)])
+    return stats.kstest(u, "uniform").pvalue > 1e-4
+
+
+def check_p_eq_q(svo, L):
+    rng = np.random.default_rng(1)
+    z = (rng.standard_normal((100, 4, 50)) * 3).astype(np.float32)
+    tok = rng.integers(0, 50, (100, 3)).astype(np.int32)
+    out = svo.verify(z, np.ascontiguousarray(z[:, :3]), tok, seed=3, L=L)
+    return bool(np.all(out["accept_len"] == 4))
+
+
+def check_al_law(svo, L):
+    rng = np.random.default_rng(4)
+    V, D, N = 8, 3, 60_000
+    zt = (rng.standard_normal((D + 1, V)) * 1.5).astype(np.float32)
+    zq = (zt[:D] + rng.standard_normal((D, V))).astype(np.float32)
+    p, q = softmax(zt, 0.7), softmax(zq, 0.7)
+    tok = np.array([int(np.argmax(q[d] / p[d])) if d % 2 == 0 else int(np.argmax(p[d]))
+                    for d in range(D)], np.int32)
+    a = np.minimum(1.0, p[np.arange(D), tok] / q[np.arange(D), tok])
+    law = np.array([np.prod(a[:k]) * (1 - a[k]) for k in range(D)] + [np.prod(a)])
+    out = svo.verify(tile(zt, N), tile(zq, N), tile(tok, N), temperature=0.7, seed=17, nthreads=8, L=L)
+    counts = np.bincount(out["accept_len"] - 1, minlength=D + 1)
+    return within_sigma(counts, law, 4.0)[0]
+
+
+def check_residual_law(svo, L):
+    rng = np.random.default_rng(5)
+    V, N = 8, 60_000
+    zt = (rng.standard_normal((2, V)) * 1.5).astype(np.float32)
+    zq = (zt[:1] + rng.standard_normal((1, V)) * 1.5).astype(np.float32)
+    p, q = softmax(zt)[0], softmax(zq)[0]
+    x0 = int(np.argmax(q / p))
+    r = np.maximum(0.0, p - q)
+    r /= r.sum()
+    out = svo.verify(tile(zt, N), tile(zq, N), np.full((N, 1), x0, np.int32), seed=23, nthreads=8, L=L)
+    rej = out["accept_len"] == 1
+    if not rej.any():
+        return False
+    emitted = out["tokens"][rej, 0]
+    if np.any(emitted < 0) or np.any(p[emitted] <= q[emitted]):
+        return False
+    return within_sigma(np.bincount(emitted, minlength=V), r, 4.0)[0]
+
+
+def check_bonus_law(svo, L):
+    rng = np.random.default_rng(6)
+    V, N = 8, 60_000
+    zt = (rng.standard_normal((3, V)) * 1.5).astype(np.float32)
+    p = softmax(zt, 0.5)[2]
+    out = svo.verify(tile(zt, N), tile(zt[:2], N), np.zeros((N, 2), np.int32), temperature=0.5,
+                     seed=29, nthreads=8, L=L)
+    if not np.all(out["accept_len"] == 3):
+        return False
+    return within_sigma(np.bincount(out["tokens"][:, 2], minlength=V), p, 4.0)[0]
+
+
+def check_marginal(svo, L, mode):
+    rng = np.random.default_rng(100 + mode)
+    V, D, N = 8, 2, 200_000
+    zt = (rng.standard_normal((D + 1, V)) * 1.5).astype(np.float32)
+    zq = (zt[:D] + rng.standard_normal((D, V)) * 1.2).astype(np.float32)
+    p, q = softmax(zt), softmax(zq)
+    qd = q.copy()
+    if mode == 2:
+        for d in range(D):
+            top = np.lexsort((np.arange(V), -zq[d].astype(np.float64)))[:5]
+            qd[d, top] *= 0.5
+            qd[d] /= qd[d].sum()
+    tok = np.stack([sample_categorical(rng, qd[d], N) for d in range(D)], axis=1)
+    out = svo.verify(tile(zt, N), tile(zq, N), tok, mode=mode, seed=31, nthreads=8, L=L)
+    AL, toks = out["accept_len"], out["tokens"]
+    for slot, sel in ((0, np.ones_like(AL, bool)), (1, AL >= 2), (2, AL == 3)):
+        if not within_sigma(np.bincount(toks[sel, slot], minlength=V), p[slot], 4.0)[0]:
+            return False
+    return True
+
+
+def check_saguaro_ties(svo, L):
+    # tied draft logits: K = tokens 0..4, q'(0..4) = 1/7, q'(5) = 2/7
+    zq1 = np.zeros((1, 1, 6), np.float32)
+    zt1 = np.zeros((1, 2, 6), np.float32)
+    zt1[0, 0, :] = math.log(1 / 7) + 1e-6
+    zt1[0, 0, 5] = math.log(2 / 7)
+    for s in range(40):
+        for x in (0, 5):
+            out = svo.verify(zt1, zq1, np.array([[x]], np.int32), mode=2, seed=s, L=L)
+            if x == 0 and out["accept_len"][0] != 2:
+                return False
+    return True
+
+
+def check_greedy(svo, L):
+    rng = np.random.default_rng(9)
+    V, D = 40, 4
+    Tt = (rng.standard_normal((V, V)) * 1.5).astype(np.float32)
+    Qt = (Tt + rng.standard_normal((V, V)) * 0.8).astype(np.float32)
+    ref, last = [], 0
+    for _ in range(30):
+        last = int(np.argmax(Tt[last]))
+        ref.append(last)
+    seq, last = [], 0
+    while len(seq) < 30:
+        prev, tok = [last], []
+        for _ in range(D):
+            tok.append(int(np.argmax(Qt[prev[-1]])))
+            prev.append(tok[-1])
+        out = svo.verify(Tt[np.array(prev)][None], None, np.array([tok], np.int32), mode=1, L=L)
+        k = int(out["accept_len"][0])
+        if k < 1:
+            return False
+        seq.extend(int(t) for t in out["tokens"][0, :k])
+        last = seq[-1]
+    if seq[:30] != ref:
+        return False
+    # a draft that proposes the target's own argmax chain is accepted in full
+    prev = [0] + ref[:D]
+    out = svo.verify(Tt[np.array(prev)][None], None, np.array([ref[:D]], np.int32), mode=1, L=L)
+    return int(out["accept_len"][0]) == D + 1 and list(out["tokens"][0]) == ref[:D + 1]
+
+
+CHECKS = [check_lse, check_argmax, check_avalanche, check_uniform, check_p_eq_q, check_al_law,
+          check_residual_law, check_bonus_law, lambda s, L: check_marginal(s, L, 0),
+          lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy]
+
+
+def _build_variant(tmp, text):
+    import oracle.build as ob
+    src = os.path.join(tmp, "svo.c")
+    with open(src, "w") as f:
+        f.write(text)
+    hdr = os.path.join(ROOT, "oracle", "svo.h")
+    os.symlink(hdr, os.path.join(tmp, "svo.h"))
+    lib = os.path.join(tmp, "libsvo_variant.so")
+    subprocess.run(["gcc", *ob.CFLAGS, src, "-o", lib, "-lm"], check=True,
+                   stderr=subprocess.DEVNULL)
+    return lib
+
+
+def test_unmodified_oracle_passes_every_check(svo):
+    L = svo.lib()
+    for chk in CHECKS:
+        assert chk(svo, L), chk
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(svo, name):
+    old, new = MUTANTS[name]
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
+    with tempfile.TemporaryDirectory() as tmp:
+        L = svo.load_variant(_build_variant(tmp, text.replace(old, new)))
+        failed = []
+        for chk in CHECKS:
+            try:
+                ok = chk(svo, L)
+            except Exception:  # a crash or a rejected call also counts as caught
+                ok = False
+            if not ok:
+                failed.append(chk)
+                break
+        assert failed, f"no pin caught the planted mistake {name}"
