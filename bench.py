@@ -1,0 +1,416 @@
+"""Benchmark of the speculative-decoding verification step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload b256] [--variant auto|split|fused]
+
+One step = one call of the library (row statistics, accept scan, race) over one
+batch of synthetic logits already resident in HBM.  Workload (default): B=256
+requests, D=7 drafts, V=128256, bf16 logits, target N(0, 3^2), draft = target +
+N(0, 0.75^2), draft tokens sampled from q, T=1, stochastic mode.  Its inputs
+(985 MB) exceed the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (launched by torchrun): requests shard with no exchange, so every
+rank verifies its own batch of the same shape (weak scaling, no data-path
+collective); the step time is the max over ranks.
+
+Prints one JSON line on rank 0.  `--impl reference` times the CPU oracle (the
+plain double-precision restatement of the rule) on the host cores instead.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verified rows/s (B×(D+1)) and achieved HBM GB/s vs B200 peak, 1 GPU"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(w):
+    m = w.meta
+    return (f"{w.name}: B={w.B}, D={w.D_max}, V={w.V}, "
+            f"{'bf16' if w.dtype == 1 else 'fp32'} logits, target N(0,{m['target_sd']}^2), "
+            f"draft = target + N(0,{m['draft_sd']}^2), draft tokens sampled from q, T={w.temperature}, "
+            f"{['stochastic', 'greedy', 'saguaro'][w.mode]}")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.active = False
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if self.active:
+                self.samples.append([s.strip() for s in line.split(",")])
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in self.samples:
+            try:
+                sm.append(float(s[1]))
+                mx.append(float(s[2]))
+            except Exception:
+                continue
+            for name, v in zip(names, s[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_record(kernel_name, sources):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for s in sources:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    sha = h.hexdigest()[:16]
+    rec = {}
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and parts[0] == kernel_name:
+                rec[parts[1]] = (float(parts[2]), int(parts[3]))  # sha -> (bytes per launch, units)
+    return rec.get(sha)
+
+
+def cpu_baseline(w, target_seconds=10.0):
+    """The oracle, as it stands, on the host cores over the same host copy of the
+    inputs; the whole batch is repeated until about `target_seconds` pass."""
+    import oracle
+    h = w.host_arrays()
+    cores = os.cpu_count() or 1
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.verify(h["target"], h["draft"], h["tokens"], h["row_D"], temperature=w.temperature,
+                      mode=w.mode, seed=w.seed, temperature_per_req=h["temperature_per_req"],
+                      mode_per_req=h["mode_per_req"], saguaro_k=w.saguaro_k,
+                      saguaro_c=w.saguaro_c, nthreads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= target_seconds or reps >= 50:
+            break
+    rows = reps * w.verified_rows()
+    return {"value": rows / el, "unit": "rows/s", "cores": cores, "kind": "oracle",
+            "sample": f"the whole {w.name} batch ({w.B} requests, {w.verified_rows()} verified rows) "
+                      f"x {reps} repetitions, {el:.1f} s, OpenMP over requests"}
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores, timed per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch  # noqa: F401  (workload generation)
+    from speculative_decoding_verification_lse_b200 import workloads
+    w = workloads.make(args.workload, "cpu")
+    import oracle
+    h = w.host_arrays()
+    cores = os.cpu_count() or 1
+
+    def run(sl):
+        oracle.verify(h["target"][sl], h["draft"][sl], h["tokens"][sl],
+                      None if h["row_D"] is None else h["row_D"][sl], temperature=w.temperature,
+                      mode=w.mode, seed=w.seed,
+                      temperature_per_req=None if h["temperature_per_req"] is None
+                      else h["temperature_per_req"][sl],
+                      mode_per_req=None if h["mode_per_req"] is None else h["mode_per_req"][sl],
+                      saguaro_k=w.saguaro_k, saguaro_c=w.saguaro_c, nthreads=cores,
+                      request_offset=sl.start)
+
+    # a bounded sample per step: one request per core, repeated so that all
+    # warm-up and timed steps together take about `ref_seconds`
+    t0 = time.perf_counter()
+    run(slice(0, 1))
+    t_req = time.perf_counter() - t0
+    per_step = args.ref_seconds / max(1, args.steps + args.warmup)
+    waves = max(1, int(per_step / max(t_req, 1e-6)))
+    nreq = max(1, min(w.B, cores * waves))
+    sl = slice(0, nreq)
+    rows = sum(d + 1 for d in w.row_D_list()[:nreq])
+
+    def step():
+        run(sl)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = rows * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "B": w.B, "D": w.D_max, "V": w.V},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {nreq} of {w.B} requests ({rows} verified rows) per step"},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import speculative_decoding_verification_lse_b200 as sv
+    from speculative_decoding_verification_lse_b200 import workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    sv.load()
+    variant = {"auto": sv.SV_VARIANT_AUTO, "split": sv.SV_VARIANT_SPLIT,
+               "fused": sv.SV_VARIANT_FUSED}[args.variant]
+
+    # every rank verifies its own batch (its own seed and request range)
+    w = workloads.make(args.workload, dev, seed=workloads.CONFIGS[args.workload]["seed"] + 97 * rank)
+    offset = rank * w.B
+    stream = torch.cuda.current_stream(dev)
+    out = dict(tokens=torch.empty((w.B, w.D_max + 1), dtype=torch.int32, device=dev),
+               accept_len=torch.empty((w.B,), dtype=torch.int32, device=dev),
+               flags=torch.empty((w.B,), dtype=torch.int32, device=dev))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def step(i, ev=None):
+        sv.verify_workload(w, seed=1000 + i, request_offset=offset, variant=variant,
+                           stream=stream, out=out, timing_events=ev)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    status = sv.sv_get_device_status(stream)
+    if status & sv.SV_FLAG_ERRORS:
+        raise RuntimeError(f"device status {status:#x} during warm-up")
+
+    # dominant-kernel timing events, one pair per step
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.active = True
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, kev[i])
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    clocks.active = False
+    barrier()
+    clocks.stop()
+    ms = t_start.elapsed_time(t_stop)
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_per_step = ms / args.steps
+    rows_total = w.verified_rows() * args.steps * world
+    value = rows_total / (ms / 1e3)
+
+    # end to end through the same call with host buffers: pinned H2D of the
+    # step's inputs, the call, D2H of the step's outputs, all in the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        h_t = torch.empty(w.target.shape, dtype=w.target.dtype, pin_memory=True)
+        h_q = torch.empty(w.draft.shape, dtype=w.draft.dtype, pin_memory=True)
+        h_x = torch.empty(w.tokens.shape, dtype=w.tokens.dtype, pin_memory=True)
+        h_t.copy_(w.target)
+        h_q.copy_(w.draft)
+        h_x.copy_(w.tokens)
+        o_t = torch.empty(out["tokens"].shape, dtype=torch.int32, pin_memory=True)
+        o_a = torch.empty(out["accept_len"].shape, dtype=torch.int32, pin_memory=True)
+        d_t, d_q, d_x = torch.empty_like(w.target), torch.empty_like(w.draft), torch.empty_like(w.tokens)
+
+        def e2e_step(i):
+            d_t.copy_(h_t, non_blocking=True)
+            d_q.copy_(h_q, non_blocking=True)
+            d_x.copy_(h_x, non_blocking=True)
+            sv.verify(d_t, d_q, d_x, None, temperature=w.temperature, mode=w.mode, seed=5000 + i,
+                      request_offset=offset, variant=variant, stream=stream, out=out)
+            o_t.copy_(out["tokens"], non_blocking=True)
+            o_a.copy_(out["accept_len"], non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.e2e_steps):
+            e2e_step(1 + i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([ems], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        h2d = h_t.numel() * h_t.element_size() + h_q.numel() * h_q.element_size() + h_x.numel() * 4
+        d2h = o_t.numel() * 4 + o_a.numel() * 4
+        e2e = {"value": w.verified_rows() * args.e2e_steps * world / (ems / 1e3), "unit": "rows/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / args.e2e_steps}
+
+    status = sv.sv_get_device_status(stream)
+    if status & sv.SV_FLAG_ERRORS:
+        raise RuntimeError(f"device status {status:#x} after the timed region")
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        step_bytes = w.algorithmic_bytes()
+        used_variant = args.variant if args.variant != "auto" else "split"
+        if used_variant == "fused":
+            kname, kbytes, ksrc = "fused_verify", step_bytes, ["speculative_decoding_verification_lse_b200/csrc/fused_verify.cu"]
+        else:
+            # the statistics pass reads every needed logit row once
+            rows_read = 0
+            for d, m in zip(w.row_D_list(), w.modes()):
+                rows_read += (d + 1) + (0 if m == 1 else d)
+            kname, kbytes = "row_stats", rows_read * w.V * (2 if w.dtype == 1 else 4)
+            ksrc = ["speculative_decoding_verification_lse_b200/csrc/row_stats.cu",
+                    "speculative_decoding_verification_lse_b200/csrc/sv_common.cuh"]
+        achieved = kbytes / (k_ms / 1e3) / 1e9
+        tr = traffic_record(kname, ksrc)
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "rows/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == 1 else "f32",
+            "data": "synthetic",
+            "config": {
+                "workload": workload_desc(w),
+                "B": w.B, "D": w.D_max, "V": w.V,
+                "variant": used_variant,
+                "l2": f"inputs {step_bytes / 1e6:.0f} MB > 126 MB L2: no flush between steps",
+                "parallelism": f"replicas x{world} (request-sharded, no collective)",
+            },
+            "hbm": {
+                "algorithmic_bytes_per_step": step_bytes,
+                "achieved_gbs": step_bytes / (ms_per_step / 1e3) / 1e9,
+                "frac_of_spec_8000": step_bytes / (ms_per_step / 1e3) / 1e9 / SPEC_HBM_GBS,
+                f"frac_of_{peak_kind}_{peak:.0f}": step_bytes / (ms_per_step / 1e3) / 1e9 / peak,
+            },
+            "roofline": {
+                "bound": "hbm",
+                "kernel": kname,
+                "achieved": achieved,
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": achieved / peak,
+                "traffic": None if tr is None else tr[0],
+                "algorithmic_bytes_per_launch": kbytes,
+                "launch_ms": k_ms,
+            },
+            "clocks": clocks.summary(),
+            "gpu_launches": (1 if used_variant == "fused" else 3) * args.steps,
+            "e2e": e2e,
+        }
+        if args.cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="b256")
+    ap.add_argument("--variant", choices=["auto", "split", "fused"], default="auto")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

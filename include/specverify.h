@@ -1,0 +1,196 @@
+/*
+ * specverify.h -- libspecverify: the speculative-decoding verification step on
+ * NVIDIA B200 (sm_100a), as a C ABI.
+ *
+ * What the step computes (sources cited by page title and section):
+ *   [Sonar] "Accélérer Sonar par la Spéculation" (Perplexity):
+ *           section "Décodage spéculatif" -- the target scores every drafted
+ *           prefix in one pass (row d of the target logits is its distribution
+ *           for draft token d) and gives one extra token (n drafts -> up to n+1
+ *           tokens); section "Cible-Brouillon" -- the sampler finds the accepted
+ *           length by comparing the full draft and target distributions, and the
+ *           target's next logits are sampled for the extra token.
+ *   [SSD]   "Speculative Speculative Decoding – асинхронизируй это." (x0ct.com):
+ *           the numbered rule -- accept when q(x) <= p(x); otherwise accept with
+ *           probability p(x)/q(x) (the page's "reject with probability p/q" is
+ *           read as the acceptance probability, the only reading under which the
+ *           output is distributed like p, as the page's closing remark states);
+ *           on rejection draw from norm(max(0, p - q)).  The saguaro recipe:
+ *           take the draft's five most likely tokens and lower their
+ *           probabilities (read: multiply by c, renormalise) for drafting and
+ *           for the residual.
+ *   [NV5]   "NVIDIA: öt irányelv gyorsíthatja az LLM-ek spekulatív dekódolását",
+ *           section "Mit csinál a spekulatív dekódolás?" -- accept the drafts in
+ *           order until the first mismatch; the accepted length AL lies in
+ *           [1, 1 + D]; greedy verification reproduces ordinary decoding.
+ *
+ * The rule, per request b with D_b drafts x_0..x_{D_b-1} and temperature T:
+ *   p_d = softmax(target[b, d, :] / T),  q_d = softmax(draft[b, d, :] / T)
+ *   (saguaro: q'_d(x) = q_d(x) c^[x in K_d] / Z_d, K_d the k largest draft
+ *    logits, Z_d = 1 - (1 - c) sum_{x in K_d} q_d(x); q' replaces q below)
+ *   a_d = min(1, p_d(x_d) / q_d(x_d));  u_d = Philox uniform (below)
+ *   n = first d with u_d >= a_d, else D_b;  AL = n + 1
+ *   token n = residual race on (p_n, q_n) if n < D_b, else bonus race on p_{D_b}
+ *   race: argmax over candidates x of r(x) / E_x, E_x unit exponentials
+ *     residual: r = p - q over {p > q};  bonus: r = p over {p > 0}
+ *     (if {p > q} is empty through rounding, the bonus race runs on p_n)
+ *   greedy: accept while x_d == argmax target[b, d, :]; token n = that argmax
+ *
+ * Random numbers (a convention of this library; the pages fix none):
+ *   Philox4x32-10 (Salmon et al., SC'11) with key (seed mod 2^32, seed >> 32).
+ *   u_d: word 0 at counter (d, g, 0, 0), top 24 bits times 2^-24.
+ *   E_x: word (x mod 4) at counter (x / 4, g, 1, 0) = o, W = (o + 1/2) 2^-32,
+ *        E_x = -ln(1 - W).
+ *   g = request_offset + b is the request's global index, so a batch split
+ *   across devices gives the same results as one call.  The caller changes
+ *   `seed` between decoding steps.
+ *
+ * Ties: argmax, top-k and the race keep the lowest token index.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers on the current CUDA device,
+ *     row-major and contiguous; the caller owns every buffer.
+ *   - Calls are asynchronous on the stream (sv_params.stream, default: the
+ *     legacy default stream) and never synchronise.
+ *   - Host-detectable argument errors return a negative code, launch nothing
+ *     and leave the outputs untouched; sv_last_error() describes the error.
+ *   - Errors found on the device (a draft token outside [0, V), row_D[b]
+ *     outside [0, D_max], NaN or +inf in a row the rule reads, a row that is
+ *     all -inf, a per-request temperature <= 0 or mode out of range) set bits
+ *     in the library's device status word and in that request's flags, and
+ *     that request's outputs are all -1.  No kernel traps or asserts.
+ *   - A logit of -inf masks its token (p = 0).
+ *   - Rows beyond a request's D_b (and draft rows of greedy requests) are
+ *     never read; they may hold anything, NaN included.
+ */
+#ifndef SPECVERIFY_H
+#define SPECVERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SV_API __attribute__((visibility("default")))
+#else
+#define SV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* dtype of the logits */
+enum { SV_F32 = 0, SV_BF16 = 1 };
+
+/* verification mode */
+enum { SV_STOCHASTIC = 0, SV_GREEDY = 1, SV_SAGUARO = 2 };
+
+/* return codes */
+enum { SV_OK = 0, SV_ERR_INVALID_ARG = -1, SV_ERR_UNSUPPORTED = -2, SV_ERR_CUDA = -3 };
+
+/* sv_params.variant */
+enum { SV_VARIANT_AUTO = 0, SV_VARIANT_SPLIT = 1, SV_VARIANT_FUSED = 2 };
+
+/* per-request flag bits (sv_params.out_flags) */
+enum {
+  SV_FLAG_ACCEPT_NEAR_TIE = 1u << 0, /* a tested position had |u - a| < 1e-5 */
+  SV_FLAG_RACE_NEAR_TIE = 1u << 1,   /* top-2 race keys ln r - ln E within 1e-6 */
+  SV_FLAG_RESIDUAL_EMPTY = 1u << 2,  /* {p > q} empty: the token came from p */
+  SV_FLAG_BAD_TOKEN = 1u << 8,
+  SV_FLAG_BAD_ROW_D = 1u << 9,
+  SV_FLAG_NONFINITE = 1u << 10,
+  SV_FLAG_BAD_PARAM = 1u << 11
+};
+
+/* device status word bits (sv_get_device_status): the union of the error
+ * flags of every request since the word was last cleared */
+enum {
+  SV_STATUS_BAD_TOKEN = SV_FLAG_BAD_TOKEN,
+  SV_STATUS_BAD_ROW_D = SV_FLAG_BAD_ROW_D,
+  SV_STATUS_NONFINITE = SV_FLAG_NONFINITE,
+  SV_STATUS_BAD_PARAM = SV_FLAG_BAD_PARAM,
+  SV_STATUS_RESIDUAL_EMPTY = SV_FLAG_RESIDUAL_EMPTY
+};
+
+/* Limits checked on the host. */
+#define SV_MAX_DRAFT 32  /* D_max <= 32 */
+#define SV_MAX_SAGUARO_K 8
+
+/*
+ * Optional parameters.  Zero-initialise, then set what you need.
+ */
+typedef struct sv_params {
+  void* stream;                      /* cudaStream_t; NULL = legacy default stream */
+  const float* temperature_per_req;  /* [B] device; NULL: every request uses `temperature` */
+  const int8_t* mode_per_req;        /* [B] device; NULL: every request uses `mode` */
+  int saguaro_k;                     /* size of K; <= 0 means 5; at most SV_MAX_SAGUARO_K */
+  float saguaro_c;                   /* down-weighting factor in (0, 1]; <= 0 means 0.5 */
+  int variant;                       /* SV_VARIANT_*; AUTO picks per shape */
+  uint32_t request_offset;           /* global index of request 0 (sharded batches) */
+  float* out_row_lse;                /* [B, 2*D_max+1] device, optional: natural-log LSE of
+                                        target rows (slots 0..D_max) and draft rows (slots
+                                        D_max+1..2*D_max) at temperature T; NaN where the row
+                                        is not used (greedy requests, rows beyond D_b) */
+  uint32_t* out_flags;               /* [B] device, optional: SV_FLAG_* per request */
+  void* workspace;                   /* optional caller scratch (device, 256-byte aligned);
+                                        NULL: a per-device cache grown on demand with
+                                        cudaMalloc and freed by sv_shutdown */
+  size_t workspace_bytes;            /* size of `workspace`; >= sv_workspace_bytes(...) */
+  void* timing_events;               /* optional cudaEvent_t[2]: recorded on the stream
+                                        immediately before and after the row-statistics
+                                        kernel (split) or the fused kernel (fused) */
+} sv_params;
+
+/*
+ * sv_verify: the whole verification step for B requests.
+ *   target_logits  [B, D_max+1, V] of dtype; row d scores draft token d, row D_b is
+ *                  the bonus row                       ([Sonar] "Décodage spéculatif")
+ *   draft_logits   [B, D_max, V] of dtype; may be NULL only if every request is greedy
+ *   draft_tokens   [B, D_max] int32; entries at d >= D_b are ignored
+ *   row_D          [B] int32, D_b in [0, D_max]; NULL means D_max for every request
+ *   B >= 0, 0 <= D_max <= SV_MAX_DRAFT, V >= 1, dtype SV_F32 or SV_BF16
+ *   temperature    > 0 and finite unless every request is greedy
+ *   mode           SV_STOCHASTIC, SV_GREEDY or SV_SAGUARO
+ *   seed           Philox key for this step
+ *   out_tokens     [B, D_max+1] int32: the accepted drafts x_0..x_{n-1}, then the
+ *                  sampled token at slot n, then -1
+ *   out_accept_len [B] int32: AL = n + 1 in [1, 1 + D_b]   ([NV5] "Mit csinál...")
+ * Returns SV_OK or a negative code.
+ */
+SV_API int sv_verify(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
+              const int32_t* row_D, int B, int D_max, int V, int dtype, float temperature,
+              int mode, uint64_t seed, int32_t* out_tokens, int32_t* out_accept_len);
+
+/* Greedy verification ([NV5]: same output as ordinary argmax decoding).  Draft
+ * logits are never read; T is not used.  Same layout as sv_verify. */
+SV_API int sv_verify_greedy(const void* target_logits, const int32_t* draft_tokens,
+                     const int32_t* row_D, int B, int D_max, int V, int dtype,
+                     int32_t* out_tokens, int32_t* out_accept_len);
+
+/* sv_verify with optional parameters (p may be NULL). */
+SV_API int sv_verify_ex(const void* target_logits, const void* draft_logits,
+                 const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max, int V,
+                 int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
+                 int32_t* out_accept_len, const sv_params* p);
+
+/* Bytes of scratch one call with these sizes needs (for sv_params.workspace). */
+SV_API size_t sv_workspace_bytes(int B, int D_max, int V, int dtype);
+
+/* Synchronises `stream` (cudaStream_t, NULL = legacy default), copies the device
+ * status word of the current device into *status_bits and clears it.
+ * Returns SV_OK or SV_ERR_CUDA. */
+SV_API int sv_get_device_status(void* stream, uint32_t* status_bits);
+
+/* Message for the last error returned on this host thread ("" if none). */
+SV_API const char* sv_last_error(void);
+
+/* Frees the cached per-device workspaces.  Call with no call in flight. */
+SV_API void sv_shutdown(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+SV_API int sv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPECVERIFY_H */

@@ -1,0 +1,233 @@
+"""Python binding of libspecverify (the C ABI in include/specverify.h).
+
+Argument marshalling only: tensors are turned into device pointers and sizes,
+and every step of the verification runs in the library's CUDA kernels.  There
+is no CPU path: without the built library or a CUDA device the calls raise.
+
+    import speculative_decoding_verification_lse_b200 as sv
+    out = sv.verify(target, draft, tokens, temperature=1.0, seed=0)   # torch CUDA tensors
+    out["tokens"], out["accept_len"], out["flags"]
+"""
+import ctypes
+import os
+
+SV_F32, SV_BF16 = 0, 1
+SV_STOCHASTIC, SV_GREEDY, SV_SAGUARO = 0, 1, 2
+SV_OK, SV_ERR_INVALID_ARG, SV_ERR_UNSUPPORTED, SV_ERR_CUDA = 0, -1, -2, -3
+SV_VARIANT_AUTO, SV_VARIANT_SPLIT, SV_VARIANT_FUSED = 0, 1, 2
+
+SV_FLAG_ACCEPT_NEAR_TIE = 1 << 0
+SV_FLAG_RACE_NEAR_TIE = 1 << 1
+SV_FLAG_RESIDUAL_EMPTY = 1 << 2
+SV_FLAG_BAD_TOKEN = 1 << 8
+SV_FLAG_BAD_ROW_D = 1 << 9
+SV_FLAG_NONFINITE = 1 << 10
+SV_FLAG_BAD_PARAM = 1 << 11
+SV_FLAG_NEAR_TIE = SV_FLAG_ACCEPT_NEAR_TIE | SV_FLAG_RACE_NEAR_TIE
+SV_FLAG_ERRORS = SV_FLAG_BAD_TOKEN | SV_FLAG_BAD_ROW_D | SV_FLAG_NONFINITE | SV_FLAG_BAD_PARAM
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspecverify.so")
+
+
+class SvParams(ctypes.Structure):
+    """Mirror of sv_params."""
+    _fields_ = [
+        ("stream", ctypes.c_void_p),
+        ("temperature_per_req", ctypes.c_void_p),
+        ("mode_per_req", ctypes.c_void_p),
+        ("saguaro_k", ctypes.c_int),
+        ("saguaro_c", ctypes.c_float),
+        ("variant", ctypes.c_int),
+        ("request_offset", ctypes.c_uint32),
+        ("out_row_lse", ctypes.c_void_p),
+        ("out_flags", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("timing_events", ctypes.c_void_p),
+    ]
+
+
+class SvError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"libspecverify error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+_VERIFY_ARGS = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_float, ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]
+
+
+def load(build_if_needed=True):
+    """Load libspecverify.so (compiling it first if it is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if build_if_needed:
+        from . import build as _build
+        _build.build()
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run __graft_entry__.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    L.sv_verify.argtypes = _VERIFY_ARGS
+    L.sv_verify.restype = ctypes.c_int
+    L.sv_verify_ex.argtypes = _VERIFY_ARGS + [ctypes.POINTER(SvParams)]
+    L.sv_verify_ex.restype = ctypes.c_int
+    L.sv_verify_greedy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_void_p, ctypes.c_void_p]
+    L.sv_verify_greedy.restype = ctypes.c_int
+    L.sv_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    L.sv_workspace_bytes.restype = ctypes.c_size_t
+    L.sv_get_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
+    L.sv_get_device_status.restype = ctypes.c_int
+    L.sv_last_error.argtypes = []
+    L.sv_last_error.restype = ctypes.c_char_p
+    L.sv_shutdown.argtypes = []
+    L.sv_shutdown.restype = None
+    L.sv_version.argtypes = []
+    L.sv_version.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _p(x):
+    """A device pointer from a tensor, an int or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _check(rc):
+    if rc != SV_OK:
+        raise SvError(rc, load().sv_last_error().decode())
+    return rc
+
+
+# ---- the C ABI, same names (pointers may be tensors or ints)
+
+def sv_verify(target_logits, draft_logits, draft_tokens, row_D, B, D_max, V, dtype,
+              temperature, mode, seed, out_tokens, out_accept_len):
+    return load().sv_verify(_p(target_logits), _p(draft_logits), _p(draft_tokens), _p(row_D),
+                            B, D_max, V, dtype, temperature, mode, seed & (2**64 - 1),
+                            _p(out_tokens), _p(out_accept_len))
+
+
+def sv_verify_greedy(target_logits, draft_tokens, row_D, B, D_max, V, dtype, out_tokens,
+                     out_accept_len):
+    return load().sv_verify_greedy(_p(target_logits), _p(draft_tokens), _p(row_D), B, D_max, V,
+                                   dtype, _p(out_tokens), _p(out_accept_len))
+
+
+def sv_verify_ex(target_logits, draft_logits, draft_tokens, row_D, B, D_max, V, dtype,
+                 temperature, mode, seed, out_tokens, out_accept_len, params=None):
+    return load().sv_verify_ex(_p(target_logits), _p(draft_logits), _p(draft_tokens), _p(row_D),
+                               B, D_max, V, dtype, temperature, mode, seed & (2**64 - 1),
+                               _p(out_tokens), _p(out_accept_len),
+                               ctypes.byref(params) if params is not None else None)
+
+
+def sv_workspace_bytes(B, D_max, V, dtype):
+    return load().sv_workspace_bytes(B, D_max, V, dtype)
+
+
+def sv_get_device_status(stream=None):
+    bits = ctypes.c_uint32(0)
+    _check(load().sv_get_device_status(_stream_ptr(stream), ctypes.byref(bits)))
+    return bits.value
+
+
+def sv_last_error():
+    return load().sv_last_error().decode()
+
+
+def sv_shutdown():
+    load().sv_shutdown()
+
+
+def sv_version():
+    return load().sv_version()
+
+
+# ---- convenience wrapper over torch tensors
+
+def _stream_ptr(stream):
+    if stream is None:
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return SV_F32
+    if t.dtype == torch.bfloat16:
+        return SV_BF16
+    raise TypeError(f"logits must be float32 or bfloat16 CUDA tensors, got {t.dtype}")
+
+
+def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHASTIC, seed=0,
+           temperature_per_req=None, mode_per_req=None, saguaro_k=5, saguaro_c=0.5,
+           request_offset=0, variant=SV_VARIANT_AUTO, stream=None, row_lse=False,
+           out=None, workspace=None, timing_events=None):
+    """Verify a batch held in CUDA tensors; returns dict(tokens, accept_len, flags
+    [, row_lse]) as CUDA tensors, enqueued on `stream` (not synchronised)."""
+    import torch
+    if not target.is_cuda:
+        raise ValueError("target logits must be a CUDA tensor (there is no CPU path)")
+    dt = _dtype_code(target)
+    if not target.is_contiguous():
+        raise ValueError("target logits must be contiguous")
+    B, Dp1, V = target.shape
+    D = Dp1 - 1
+    if draft is not None:
+        if draft.dtype != target.dtype or tuple(draft.shape) != (B, D, V) or not draft.is_contiguous():
+            raise ValueError("draft logits must be contiguous [B, D_max, V] of the target's dtype")
+    if tokens.dtype != torch.int32 or tuple(tokens.shape) != (B, D) or not tokens.is_contiguous():
+        raise ValueError("draft tokens must be contiguous int32 [B, D_max]")
+    for name, t, dtp in (("row_D", row_D, torch.int32),
+                         ("temperature_per_req", temperature_per_req, torch.float32),
+                         ("mode_per_req", mode_per_req, torch.int8)):
+        if t is not None and (t.dtype != dtp or t.numel() != B or not t.is_cuda):
+            raise ValueError(f"{name} must be a CUDA {dtp} tensor of {B} elements")
+    dev = target.device
+    if out is None:
+        out = dict(tokens=torch.empty((B, D + 1), dtype=torch.int32, device=dev),
+                   accept_len=torch.empty((B,), dtype=torch.int32, device=dev),
+                   flags=torch.empty((B,), dtype=torch.int32, device=dev))
+        if row_lse:
+            out["row_lse"] = torch.empty((B, 2 * D + 1), dtype=torch.float32, device=dev)
+    prm = SvParams()
+    prm.stream = _stream_ptr(stream)
+    prm.temperature_per_req = _p(temperature_per_req)
+    prm.mode_per_req = _p(mode_per_req)
+    prm.saguaro_k = int(saguaro_k)
+    prm.saguaro_c = float(saguaro_c)
+    prm.variant = int(variant)
+    prm.request_offset = int(request_offset)
+    prm.out_row_lse = _p(out.get("row_lse"))
+    prm.out_flags = _p(out.get("flags"))
+    if workspace is not None:
+        prm.workspace = _p(workspace)
+        prm.workspace_bytes = workspace.numel() * workspace.element_size()
+    if timing_events is not None:
+        arr = (ctypes.c_void_p * 2)(timing_events[0].cuda_event, timing_events[1].cuda_event)
+        prm.timing_events = ctypes.cast(arr, ctypes.c_void_p)
+    with torch.cuda.device(dev):
+        _check(sv_verify_ex(target, draft, tokens, row_D, B, D, V, dt, float(temperature),
+                            int(mode), int(seed), out["tokens"], out["accept_len"], prm))
+    return out
+
+
+def verify_workload(w, **kw):
+    """verify() on a workloads.Workload."""
+    return verify(w.target, w.draft, w.tokens, w.row_D, temperature=w.temperature, mode=w.mode,
+                  seed=kw.pop("seed", w.seed), temperature_per_req=w.temperature_per_req,
+                  mode_per_req=w.mode_per_req, saguaro_k=w.saguaro_k, saguaro_c=w.saguaro_c, **kw)

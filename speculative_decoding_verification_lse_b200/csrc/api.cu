@@ -1,0 +1,268 @@
+// api.cu -- the C ABI of libspecverify (declared in include/specverify.h):
+// argument checks, the per-device workspace cache, the device status word and
+// the launch sequence.  Every step of the computation runs in the kernels.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "specverify.h"
+#include "sv_common.cuh"
+
+namespace sv {
+
+// The device status word: one per device, in the library's own device memory.
+__device__ unsigned int g_status_word;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct DeviceCache {
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  unsigned int* status = nullptr;  // device address of g_status_word
+};
+
+std::mutex g_mu;
+std::vector<DeviceCache> g_dev;
+
+DeviceCache* device_cache(int dev) {
+  if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
+  return &g_dev[dev];
+}
+
+// Device address of the status word on the current device (looked up once).
+int status_word(int dev, unsigned int** out) {
+  DeviceCache* c = device_cache(dev);
+  if (!c->status) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+    c->status = (unsigned int*)p;
+  }
+  *out = c->status;
+  return SV_OK;
+}
+
+// The cached workspace of the current device, grown to at least `bytes`.
+int cached_workspace(int dev, size_t bytes, void** out) {
+  DeviceCache* c = device_cache(dev);
+  if (c->ws_bytes < bytes) {
+    if (c->ws) {
+      // the old buffer may still be in use by work queued earlier on any stream
+      cudaError_t e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+      cudaFree(c->ws);
+      c->ws = nullptr;
+      c->ws_bytes = 0;
+    }
+    size_t want = bytes < (1u << 20) ? (1u << 20) : bytes;
+    cudaError_t e = cudaMalloc(&c->ws, want);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
+    c->ws_bytes = want;
+  }
+  *out = c->ws;
+  return SV_OK;
+}
+
+}  // namespace
+}  // namespace sv
+
+using namespace sv;
+
+extern "C" {
+
+int sv_version(void) { return 10000; }
+
+const char* sv_last_error(void) { return g_last_error.c_str(); }
+
+size_t sv_workspace_bytes(int B, int D_max, int V, int dtype) {
+  if (B < 0 || D_max < 0 || V < 1 || (dtype != SV_F32 && dtype != SV_BF16)) return 0;
+  return ws_layout(B, D_max, V, dtype).total;
+}
+
+int sv_verify_ex(const void* target_logits, const void* draft_logits,
+                 const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max, int V,
+                 int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
+                 int32_t* out_accept_len, const sv_params* p) {
+  sv_params prm;
+  memset(&prm, 0, sizeof prm);
+  if (p) prm = *p;
+  g_last_error.clear();
+
+  if (B < 0) return fail(SV_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  if (D_max < 0 || D_max > SV_MAX_DRAFT)
+    return fail(SV_ERR_INVALID_ARG, "D_max must be in [0, %d] (got %d)", SV_MAX_DRAFT, D_max);
+  if (V < 1) return fail(SV_ERR_INVALID_ARG, "V must be >= 1 (got %d)", V);
+  if (dtype != SV_F32 && dtype != SV_BF16)
+    return fail(SV_ERR_INVALID_ARG, "dtype must be SV_F32 or SV_BF16 (got %d)", dtype);
+  if (mode != SV_STOCHASTIC && mode != SV_GREEDY && mode != SV_SAGUARO)
+    return fail(SV_ERR_INVALID_ARG, "mode must be SV_STOCHASTIC, SV_GREEDY or SV_SAGUARO (got %d)",
+                mode);
+  if (!prm.temperature_per_req && mode != SV_GREEDY && !(temperature > 0.0f && std::isfinite(temperature)))
+    return fail(SV_ERR_INVALID_ARG, "temperature must be > 0 and finite (got %g)", (double)temperature);
+  int k = prm.saguaro_k <= 0 ? 5 : prm.saguaro_k;
+  if (k > SV_MAX_SAGUARO_K)
+    return fail(SV_ERR_INVALID_ARG, "saguaro_k must be <= %d (got %d)", SV_MAX_SAGUARO_K, k);
+  if (k > V) k = V;
+  const float c = prm.saguaro_c <= 0.0f ? 0.5f : prm.saguaro_c;
+  if (!(c > 0.0f && c <= 1.0f))
+    return fail(SV_ERR_INVALID_ARG, "saguaro_c must be in (0, 1] (got %g)", (double)c);
+  if (prm.variant < SV_VARIANT_AUTO || prm.variant > SV_VARIANT_FUSED)
+    return fail(SV_ERR_INVALID_ARG, "unknown variant %d", prm.variant);
+  if (B == 0) return SV_OK;
+  if (!target_logits || !out_tokens || !out_accept_len)
+    return fail(SV_ERR_INVALID_ARG, "target_logits, out_tokens and out_accept_len must be non-NULL");
+  if (D_max > 0 && !draft_tokens) return fail(SV_ERR_INVALID_ARG, "draft_tokens is NULL");
+  if (!draft_logits && D_max > 0 && !prm.mode_per_req && mode != SV_GREEDY)
+    return fail(SV_ERR_INVALID_ARG, "draft_logits is NULL but the mode reads it");
+  const size_t es = dtype == SV_F32 ? 4 : 2;
+  if (((uintptr_t)target_logits % es) || (draft_logits && ((uintptr_t)draft_logits % es)))
+    return fail(SV_ERR_INVALID_ARG, "logit pointers must be aligned to the element size");
+
+  int nvec, nch;
+  row_geometry(V, dtype, &nvec, &nch);
+  if ((mode == SV_SAGUARO || prm.mode_per_req) && nch > 64)
+    return fail(SV_ERR_UNSUPPORTED, "saguaro supports V up to %d for this dtype",
+                64 * kChunkVecs * vec_elems(dtype));
+  const long long slots = 2LL * D_max + 1;
+  if ((long long)B * slots * nch > 0x7FFFFFFFLL)
+    return fail(SV_ERR_UNSUPPORTED, "B * (2*D_max+1) * chunks exceeds the grid limit");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+
+  const WsLayout L = ws_layout(B, D_max, V, dtype);
+  void* ws = prm.workspace;
+  unsigned int* status = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int rc = status_word(dev, &status);
+    if (rc) return rc;
+    if (ws) {
+      if (prm.workspace_bytes < L.total)
+        return fail(SV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes",
+                    prm.workspace_bytes, L.total);
+      if ((uintptr_t)ws % 256)
+        return fail(SV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    } else {
+      rc = cached_workspace(dev, L.total, &ws);
+      if (rc) return rc;
+    }
+  }
+
+  VerifyArgs a;
+  memset(&a, 0, sizeof a);
+  a.target = target_logits;
+  a.draft = draft_logits;
+  a.tokens = draft_tokens;
+  a.row_D = row_D;
+  a.temp_per_req = prm.temperature_per_req;
+  a.mode_per_req = prm.mode_per_req;
+  a.out_tokens = out_tokens;
+  a.out_al = out_accept_len;
+  a.out_row_lse = prm.out_row_lse;
+  a.out_flags = prm.out_flags;
+  a.status = status;
+  a.cstat = (ChunkStat*)((char*)ws + L.cstat);
+  a.rdesc = (RaceDesc*)((char*)ws + L.rdesc);
+  a.rpart = (RacePart*)((char*)ws + L.rpart);
+  a.rcount = (unsigned int*)((char*)ws + L.rcount);
+  a.seed = seed;
+  a.B = B;
+  a.D_max = D_max;
+  a.V = V;
+  a.dtype = dtype;
+  a.nvec = nvec;
+  a.nch = nch;
+  a.slots = (int)slots;
+  a.mode = mode;
+  a.temperature = temperature;
+  a.saguaro_k = k;
+  a.saguaro_c = c;
+  a.request_offset = prm.request_offset;
+
+  cudaStream_t s = (cudaStream_t)prm.stream;
+  cudaEvent_t* ev = (cudaEvent_t*)prm.timing_events;
+  if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = launch_row_stats(a, s)) != cudaSuccess) return cuda_fail(e, "row statistics launch");
+  if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = launch_accept_scan(a, s)) != cudaSuccess) return cuda_fail(e, "accept scan launch");
+  if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");
+  return SV_OK;
+}
+
+int sv_verify(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
+              const int32_t* row_D, int B, int D_max, int V, int dtype, float temperature,
+              int mode, uint64_t seed, int32_t* out_tokens, int32_t* out_accept_len) {
+  return sv_verify_ex(target_logits, draft_logits, draft_tokens, row_D, B, D_max, V, dtype,
+                      temperature, mode, seed, out_tokens, out_accept_len, nullptr);
+}
+
+int sv_verify_greedy(const void* target_logits, const int32_t* draft_tokens,
+                     const int32_t* row_D, int B, int D_max, int V, int dtype,
+                     int32_t* out_tokens, int32_t* out_accept_len) {
+  return sv_verify_ex(target_logits, nullptr, draft_tokens, row_D, B, D_max, V, dtype, 1.0f,
+                      SV_GREEDY, 0, out_tokens, out_accept_len, nullptr);
+}
+
+int sv_get_device_status(void* stream, uint32_t* status_bits) {
+  g_last_error.clear();
+  if (!status_bits) return fail(SV_ERR_INVALID_ARG, "status_bits is NULL");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  unsigned int* status = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int rc = status_word(dev, &status);
+    if (rc) return rc;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned int host = 0;
+  if ((e = cudaMemcpyAsync(&host, status, sizeof host, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemcpyAsync(status)");
+  if ((e = cudaMemsetAsync(status, 0, sizeof host, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync(status)");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  *status_bits = host;
+  return SV_OK;
+}
+
+void sv_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (size_t d = 0; d < g_dev.size(); ++d) {
+    if (g_dev[d].ws) {
+      cudaSetDevice((int)d);
+      cudaFree(g_dev[d].ws);
+    }
+    g_dev[d].ws = nullptr;
+    g_dev[d].ws_bytes = 0;
+  }
+  cudaSetDevice(cur);
+}
+
+}  // extern "C"

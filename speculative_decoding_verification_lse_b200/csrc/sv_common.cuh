@@ -1,0 +1,258 @@
+// sv_common.cuh -- layouts and device helpers shared by the libspecverify kernels.
+//
+// Row decomposition (fixed by V and dtype only, so that identical rows always
+// reduce in the same order and give bit-identical statistics):
+//   a row of V logits is read as 16-byte vectors of VEC elements (8 bf16 or 4 fp32);
+//   a chunk is kChunkVecs = kThreads * kVecsPerThread consecutive vectors;
+//   thread t of the CTA handling chunk c owns vectors c*kChunkVecs + t + j*kThreads,
+//   j = 0..kVecsPerThread-1, so each warp reads 512 contiguous bytes per j.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sv {
+
+constexpr int kThreads = 256;        // threads per statistics / race CTA
+constexpr int kVecsPerThread = 8;    // 16-byte vectors per thread per chunk
+constexpr int kChunkVecs = kThreads * kVecsPerThread;  // 2048 vectors = 32 KiB per chunk
+constexpr int kMaxDraft = 32;
+constexpr int kMaxTopK = 8;
+constexpr int kScanWarps = 4;        // requests per accept-scan CTA
+
+enum : int { kF32 = 0, kBF16 = 1 };
+enum : int { kStochastic = 0, kGreedy = 1, kSaguaro = 2 };
+enum : int { kRaceNone = 0, kRaceBonus = 1, kRaceResidual = 2 };
+
+enum : uint32_t {
+  kFlagAcceptNearTie = 1u << 0,
+  kFlagRaceNearTie = 1u << 1,
+  kFlagResidualEmpty = 1u << 2,
+  kFlagBadToken = 1u << 8,
+  kFlagBadRowD = 1u << 9,
+  kFlagNonfinite = 1u << 10,
+  kFlagBadParam = 1u << 11,
+  kFlagErrors = kFlagBadToken | kFlagBadRowD | kFlagNonfinite | kFlagBadParam
+};
+
+// Partial statistics of one chunk of one row.
+//   m   : largest logit in the chunk (raw, as float); -inf if every entry is -inf
+//   mk  : fl(m * k2), k2 = fl(log2(e) / T): the offset the chunk's exponents used
+//   S   : sum over the chunk of 2^(fl(z*k2 - mk))   (so S * 2^mk = sum 2^(z*k2))
+//   argmax: lowest index of m inside the chunk (INT_MAX if none)
+//   bad : nonzero if a NaN or +inf was seen
+//   top : the chunk's largest logits (value desc, index asc), saguaro draft rows only
+struct __align__(16) ChunkStat {
+  float m;
+  float mk;
+  float S;
+  int argmax;
+  uint32_t bad;
+  int ntop;
+  float topv[kMaxTopK];
+  int topi[kMaxTopK];
+  int pad[2];
+};
+
+// What the race of one request needs; written by the accept scan.
+struct __align__(16) RaceDesc {
+  int kind;          // kRaceNone / kRaceBonus / kRaceResidual
+  int n;             // the position sampled (target row n; draft row n for residual)
+  uint32_t g;        // global request index (Philox counter word 1)
+  uint32_t flags;    // flags gathered so far (accept near-tie)
+  double T;          // temperature (double of the float given)
+  double lse_t;      // natural-log LSE of target row n
+  double lse_q;      // natural-log LSE of draft row n (residual)
+  double ln_c;       // saguaro: ln c
+  double ln_Z;       // saguaro: ln Z of draft row n
+  float k2;          // fl(log2(e) / T)
+  float l2_t;        // fl(lse_t * log2(e))
+  int ntop;          // saguaro: size of K (0 otherwise)
+  int top[kMaxTopK]; // saguaro: K of draft row n
+};
+
+// One race chunk's result: the best and second-best exact keys and the winner.
+struct __align__(16) RacePart {
+  double best;
+  double second;
+  int idx;           // -1 if the chunk had no candidate
+  int pad;
+};
+
+// Everything a kernel needs, passed by value.
+struct VerifyArgs {
+  const void* target;
+  const void* draft;
+  const int32_t* tokens;
+  const int32_t* row_D;
+  const float* temp_per_req;
+  const int8_t* mode_per_req;
+  int32_t* out_tokens;
+  int32_t* out_al;
+  float* out_row_lse;
+  uint32_t* out_flags;
+  unsigned int* status;    // the device status word
+  ChunkStat* cstat;        // [B, slots, nch]
+  RaceDesc* rdesc;         // [B]
+  RacePart* rpart;         // [B, nch]
+  unsigned int* rcount;    // [B]
+  uint64_t seed;
+  int B, D_max, V, dtype;
+  int nvec, nch, slots;
+  int mode;
+  float temperature;
+  int saguaro_k;
+  float saguaro_c;
+  uint32_t request_offset;
+};
+
+// Workspace layout (offsets in bytes from the workspace base, 256-aligned).
+struct WsLayout {
+  size_t cstat, rdesc, rpart, rcount, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline int vec_elems(int dtype) { return dtype == kF32 ? 4 : 8; }
+
+inline void row_geometry(int V, int dtype, int* nvec, int* nch) {
+  const int ve = vec_elems(dtype);
+  *nvec = (V + ve - 1) / ve;
+  *nch = (*nvec + kChunkVecs - 1) / kChunkVecs;
+}
+
+inline WsLayout ws_layout(int B, int D_max, int V, int dtype) {
+  int nvec, nch;
+  row_geometry(V, dtype, &nvec, &nch);
+  const size_t slots = 2 * (size_t)D_max + 1;
+  WsLayout L;
+  size_t off = 0;
+  L.cstat = off;
+  off = align_up(off + (size_t)B * slots * nch * sizeof(ChunkStat), 256);
+  L.rdesc = off;
+  off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
+  L.rpart = off;
+  off = align_up(off + (size_t)B * nch * sizeof(RacePart), 256);
+  L.rcount = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.total = off > 0 ? off : 256;
+  return L;
+}
+
+// ---------------------------------------------------------------- device helpers
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Streaming 16-byte load: read once, do not keep in L1.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// bf16 halves of a 32-bit word as floats (exact widening).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Float -> unsigned key whose unsigned order is the float order.
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Key for "largest value, then lowest index": compare as unsigned 64-bit, max wins.
+__device__ __forceinline__ unsigned long long value_index_key(float v, int idx) {
+  return ((unsigned long long)ordered_bits(v) << 32) | (0xFFFFFFFFu - (uint32_t)idx);
+}
+
+__device__ __forceinline__ float key_value(unsigned long long k) {
+  const uint32_t o = (uint32_t)(k >> 32);
+  const uint32_t b = (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
+  return __uint_as_float(b);
+}
+
+__device__ __forceinline__ int key_index(unsigned long long k) {
+  return (int)(0xFFFFFFFFu - (uint32_t)k);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ int warp_min_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
+
+// Request parameters as the kernels read them.
+struct ReqParams {
+  int Db;
+  int mode;
+  float T;
+  uint32_t err;  // kFlagBadRowD / kFlagBadParam found in the parameters
+};
+
+__device__ __forceinline__ ReqParams load_req(const VerifyArgs& a, int b) {
+  ReqParams r;
+  r.Db = a.row_D ? a.row_D[b] : a.D_max;
+  r.mode = a.mode_per_req ? (int)a.mode_per_req[b] : a.mode;
+  r.T = a.temp_per_req ? a.temp_per_req[b] : a.temperature;
+  r.err = 0;
+  if (r.Db < 0 || r.Db > a.D_max) r.err |= kFlagBadRowD;
+  if (r.mode != kStochastic && r.mode != kGreedy && r.mode != kSaguaro) r.err |= kFlagBadParam;
+  if (r.mode != kGreedy && !(r.T > 0.0f && r.T <= 3.0e38f)) r.err |= kFlagBadParam;
+  if (r.mode != kGreedy && a.draft == nullptr && r.Db > 0) r.err |= kFlagBadParam;
+  return r;
+}
+
+__device__ __forceinline__ const char* row_base(const VerifyArgs& a, int b, int slot) {
+  const size_t es = a.dtype == kF32 ? 4 : 2;
+  if (slot <= a.D_max)
+    return (const char*)a.target + ((size_t)b * (a.D_max + 1) + slot) * (size_t)a.V * es;
+  return (const char*)a.draft + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * (size_t)a.V * es;
+}
+
+__device__ __forceinline__ float load_logit(const VerifyArgs& a, const char* row, int x) {
+  if (a.dtype == kF32) return ((const float*)row)[x];
+  return __uint_as_float((uint32_t)((const uint16_t*)row)[x] << 16);
+}
+
+}  // namespace sv
+
+// Host-side launchers (one per kernel file), called from the C ABI.
+namespace sv {
+cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_accept_scan(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
+}  // namespace sv

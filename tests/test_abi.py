@@ -1,0 +1,130 @@
+"""The C ABI without a GPU: the library builds, loads, exports every entry point
+include/specverify.h declares, and rejects invalid arguments on the host before
+any CUDA call (no compute runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import speculative_decoding_verification_lse_b200 as sv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(sv_\w+)\s*\(", text, flags=re.M):
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return sv.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sv_verify", "sv_verify_greedy", "sv_verify_ex", "sv_workspace_bytes",
+                     "sv_get_device_status", "sv_last_error", "sv_shutdown", "sv_version"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(sv.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(raw, n)]
+    assert not missing, missing
+
+
+def test_only_the_abi_is_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", sv.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {n for n in exported if n.startswith("sv_")}
+    assert ours == set(declared_functions())
+
+
+def test_version_and_workspace_sizes(lib):
+    assert sv.sv_version() == 10000
+    a = sv.sv_workspace_bytes(256, 7, 128256, sv.SV_BF16)
+    b = sv.sv_workspace_bytes(1, 4, 1024, sv.SV_F32)
+    assert a > b > 0 and a % 256 == 0
+    assert sv.sv_workspace_bytes(-1, 4, 10, sv.SV_F32) == 0
+    assert sv.sv_workspace_bytes(1, 4, 10, 9) == 0
+
+
+@pytest.mark.parametrize("kw,needle", [
+    (dict(B=-1), "B must"),
+    (dict(D_max=33), "D_max"),
+    (dict(D_max=-1), "D_max"),
+    (dict(V=0), "V must"),
+    (dict(dtype=5), "dtype"),
+    (dict(mode=7), "mode"),
+    (dict(temperature=0.0), "temperature"),
+    (dict(temperature=float("nan")), "temperature"),
+    (dict(temperature=float("inf")), "temperature"),
+])
+def test_invalid_arguments_are_rejected_on_the_host(lib, kw, needle):
+    args = dict(B=2, D_max=3, V=100, dtype=sv.SV_BF16, temperature=1.0, mode=sv.SV_STOCHASTIC)
+    args.update(kw)
+    rc = sv.sv_verify(None, None, None, None, args["B"], args["D_max"], args["V"], args["dtype"],
+                      args["temperature"], args["mode"], 0, None, None)
+    assert rc == sv.SV_ERR_INVALID_ARG
+    assert needle in sv.sv_last_error()
+
+
+@pytest.mark.parametrize("field,value,needle", [
+    ("saguaro_k", 9, "saguaro_k"),
+    ("saguaro_c", 1.5, "saguaro_c"),
+    ("variant", 5, "variant"),
+])
+def test_invalid_params_are_rejected_on_the_host(lib, field, value, needle):
+    p = sv.SvParams()
+    setattr(p, field, value)
+    rc = sv.sv_verify_ex(None, None, None, None, 2, 3, 100, sv.SV_BF16, 1.0, sv.SV_SAGUARO, 0,
+                         None, None, p)
+    assert rc == sv.SV_ERR_INVALID_ARG and needle in sv.sv_last_error()
+
+
+def test_null_pointers_are_rejected_on_the_host(lib):
+    rc = sv.sv_verify(None, None, None, None, 2, 3, 100, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC, 0,
+                      None, None)
+    assert rc == sv.SV_ERR_INVALID_ARG and "non-NULL" in sv.sv_last_error()
+    # greedy needs no draft logits, stochastic does
+    fake = 1 << 20  # never dereferenced: the call is rejected first
+    rc = sv.sv_verify(fake, None, fake, None, 2, 3, 100, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC, 0,
+                      fake, fake)
+    assert rc == sv.SV_ERR_INVALID_ARG and "draft_logits" in sv.sv_last_error()
+    rc = sv.sv_verify(fake + 1, fake, fake, None, 2, 3, 100, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC,
+                      0, fake, fake)
+    assert rc == sv.SV_ERR_INVALID_ARG and "aligned" in sv.sv_last_error()
+
+
+def test_empty_batch_is_a_no_op(lib):
+    assert sv.sv_verify(None, None, None, None, 0, 3, 100, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC, 0,
+                        None, None) == sv.SV_OK
+
+
+def test_no_cpu_path_in_the_binding():
+    import torch
+    t = torch.zeros((1, 2, 8), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        sv.verify(t, t[:, :1], torch.zeros((1, 1), dtype=torch.int32))
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "speculative_decoding_verification_lse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "svo_" not in text and "svo.h" not in text, f
