@@ -253,6 +253,10 @@ def run_ours(args):
     # dominant-kernel timing events, one pair per step
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    for a_ev, b_ev in kev:  # torch creates the CUDA event on first record
+        a_ev.record(stream)
+        b_ev.record(stream)
+    torch.cuda.synchronize()
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()

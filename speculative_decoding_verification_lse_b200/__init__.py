@@ -218,6 +218,9 @@ def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHA
         prm.workspace = _p(workspace)
         prm.workspace_bytes = workspace.numel() * workspace.element_size()
     if timing_events is not None:
+        # torch creates an event's CUDA handle on its first record()
+        if not timing_events[0].cuda_event or not timing_events[1].cuda_event:
+            raise ValueError("timing events must have been recorded once before use")
         arr = (ctypes.c_void_p * 2)(timing_events[0].cuda_event, timing_events[1].cuda_event)
         prm.timing_events = ctypes.cast(arr, ctypes.c_void_p)
     with torch.cuda.device(dev):

@@ -41,6 +41,9 @@ struct DeviceCache {
   void* ws = nullptr;
   size_t ws_bytes = 0;
   unsigned int* status = nullptr;  // device address of g_status_word
+  int sms = 0;                     // multiprocessor count
+  int fused_per_sm[2] = {0, 0};    // resident fused CTAs per SM, by dtype
+  int stats_per_sm[2] = {0, 0};    // resident statistics CTAs per SM, by dtype
 };
 
 std::mutex g_mu;
@@ -61,6 +64,22 @@ int status_word(int dev, unsigned int** out) {
     c->status = (unsigned int*)p;
   }
   *out = c->status;
+  return SV_OK;
+}
+
+// Resident grids of the persistent kernels on the current device.
+int persistent_grid(int dev, int dtype, bool fused, int* grid) {
+  DeviceCache* c = device_cache(dev);
+  if (!c->sms) {
+    cudaError_t e = cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
+  int* per_sm = fused ? &c->fused_per_sm[dtype] : &c->stats_per_sm[dtype];
+  if (!*per_sm) {
+    *per_sm = fused ? fused_blocks_per_sm(dtype) : row_stats_blocks_per_sm(dtype);
+    if (*per_sm < 1) return fail(SV_ERR_CUDA, "kernel cannot be resident on this device");
+  }
+  *grid = c->sms * *per_sm;
   return SV_OK;
 }
 
@@ -98,7 +117,7 @@ const char* sv_last_error(void) { return g_last_error.c_str(); }
 
 size_t sv_workspace_bytes(int B, int D_max, int V, int dtype) {
   if (B < 0 || D_max < 0 || V < 1 || (dtype != SV_F32 && dtype != SV_BF16)) return 0;
-  return ws_layout(B, D_max, V, dtype).total;
+  return ws_layout(B, D_max, V, dtype, true).total;
 }
 
 int sv_verify_ex(const void* target_logits, const void* draft_logits,
@@ -140,26 +159,30 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   if (((uintptr_t)target_logits % es) || (draft_logits && ((uintptr_t)draft_logits % es)))
     return fail(SV_ERR_INVALID_ARG, "logit pointers must be aligned to the element size");
 
-  int nvec, nch;
-  row_geometry(V, dtype, &nvec, &nch);
-  if ((mode == SV_SAGUARO || prm.mode_per_req) && nch > 64)
-    return fail(SV_ERR_UNSUPPORTED, "saguaro supports V up to %d for this dtype",
-                64 * kChunkVecs * vec_elems(dtype));
+  int nvec, nseg;
+  row_geometry(V, dtype, &nvec, &nseg);
+  if (nseg > kMaxSegs)
+    return fail(SV_ERR_UNSUPPORTED, "V larger than %d is not supported for this dtype",
+                kMaxSegs * kSegVecs * vec_elems(dtype));
   const long long slots = 2LL * D_max + 1;
-  if ((long long)B * slots * nch > 0x7FFFFFFFLL)
-    return fail(SV_ERR_UNSUPPORTED, "B * (2*D_max+1) * chunks exceeds the grid limit");
+  if ((long long)B * slots * nseg > 0x7FFFFFFFLL)
+    return fail(SV_ERR_UNSUPPORTED, "B * (2*D_max+1) * segments exceeds 2^31");
+  const bool saguaro_possible = mode == SV_SAGUARO || prm.mode_per_req != nullptr;
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
 
-  const WsLayout L = ws_layout(B, D_max, V, dtype);
+  const WsLayout L = ws_layout(B, D_max, V, dtype, saguaro_possible);
   void* ws = prm.workspace;
   unsigned int* status = nullptr;
+  const bool fused = prm.variant == SV_VARIANT_FUSED;
+  int grid = 0;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     int rc = status_word(dev, &status);
     if (rc) return rc;
+    if ((rc = persistent_grid(dev, dtype, fused, &grid))) return rc;
     if (ws) {
       if (prm.workspace_bytes < L.total)
         return fail(SV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes",
@@ -185,17 +208,22 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.out_row_lse = prm.out_row_lse;
   a.out_flags = prm.out_flags;
   a.status = status;
-  a.cstat = (ChunkStat*)((char*)ws + L.cstat);
+  a.pstat = (PartStat*)((char*)ws + L.pstat);
+  a.tpart = (TopPart*)((char*)ws + L.tpart);
   a.rdesc = (RaceDesc*)((char*)ws + L.rdesc);
   a.rpart = (RacePart*)((char*)ws + L.rpart);
   a.rcount = (unsigned int*)((char*)ws + L.rcount);
+  a.fstate = (FusedState*)((char*)ws + L.fstate);
+  a.done = (unsigned int*)((char*)ws + L.done);
+  a.ready = (unsigned int*)((char*)ws + L.ready);
+  a.rclaim = (unsigned int*)((char*)ws + L.rclaim);
   a.seed = seed;
   a.B = B;
   a.D_max = D_max;
   a.V = V;
   a.dtype = dtype;
   a.nvec = nvec;
-  a.nch = nch;
+  a.nseg = nseg;
   a.slots = (int)slots;
   a.mode = mode;
   a.temperature = temperature;
@@ -205,8 +233,17 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
 
   cudaStream_t s = (cudaStream_t)prm.stream;
   cudaEvent_t* ev = (cudaEvent_t*)prm.timing_events;
+  if (fused) {
+    // the fused kernel's tickets, cursor and per-request counters start at zero
+    if ((e = cudaMemsetAsync((char*)ws + L.zero, 0, L.total - L.zero, s)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync(counters)");
+    if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = launch_fused(a, s, grid)) != cudaSuccess) return cuda_fail(e, "fused launch");
+    if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    return SV_OK;
+  }
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  if ((e = launch_row_stats(a, s)) != cudaSuccess) return cuda_fail(e, "row statistics launch");
+  if ((e = launch_row_stats(a, s, grid)) != cudaSuccess) return cuda_fail(e, "row statistics launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if ((e = launch_accept_scan(a, s)) != cudaSuccess) return cuda_fail(e, "accept scan launch");
   if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");

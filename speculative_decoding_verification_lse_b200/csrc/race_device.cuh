@@ -1,0 +1,302 @@
+// race_device.cuh -- device code of the residual / bonus race, shared by the
+// split race kernel and the fused kernel.
+//
+// After a rejection at position n the token is drawn from norm(max(0, p - q))
+// ("Speculative Speculative Decoding – асинхронизируй это.", rule item 3);
+// when every draft was accepted it is drawn from p at position D_b, the extra
+// token the target gives for free ("Accélérer Sonar par la Spéculation",
+// section "Décodage spéculatif").  Both draws are exponential races: the token
+// is the argmax over candidates x of r(x) / E_x with E_x unit exponentials from
+// Philox keyed by (seed, request, token), which picks x with probability
+// r(x) / sum r and does not depend on the order of any sum.
+//
+// Exactness.  The decision is taken on the exact key ln r(x) - ln E_x in double
+// precision, with the same formulas as the plain definition, but only for the
+// few tokens that can win.  One warp handles an 8 KiB segment of the row:
+//   A. every lane computes, for each of its tokens, a single-precision UPPER
+//      BOUND of the key in log2 units (ex2/lg2 based, with explicit slack for
+//      every rounding and approximation error) and keeps its two largest;
+//   B. each lane evaluates the exact key of its best token; S1 = warp maximum;
+//   C. a lane whose second bound reaches S1 (less a margin that also covers
+//      the 1e-6 near-tie band) evaluates that token too, and if its second
+//      bound reached S1 its third might have as well, so it re-scans its tokens
+//      and evaluates every one whose bound reaches S1.
+// No token whose exact key is within the band of the segment's best is ever
+// skipped, so the segment's best and runner-up are those of the exact keys.
+//
+// Layout: one warp per (request, segment); the warp that completes the last
+// segment of a request (atomic counter, no waiting) merges the segment results
+// and writes the token.  The counter starts at zero: the split path's scan
+// clears it, the fused path clears it before the launch.
+#pragma once
+#include "philox.cuh"
+#include "stats_device.cuh"
+#include "sv_common.cuh"
+
+#include <float.h>
+#include <limits.h>
+#include <math.h>
+
+namespace sv {
+
+struct Best {
+  double best;
+  double second;
+  int idx;
+};
+
+__device__ __forceinline__ void offer(Best& B, double key, int x) {
+  if (key == -INFINITY) return;
+  if (B.idx < 0 || key > B.best || (key == B.best && x < B.idx)) {
+    B.second = B.best;
+    B.best = key;
+    B.idx = x;
+  } else if (key > B.second) {
+    B.second = key;
+  }
+}
+
+__device__ __forceinline__ Best combine(const Best& A, const Best& C) {
+  const bool c_wins =
+      C.idx >= 0 && (A.idx < 0 || C.best > A.best || (C.best == A.best && C.idx < A.idx));
+  const Best& w = c_wins ? C : A;
+  const Best& l = c_wins ? A : C;
+  Best r;
+  r.best = w.best;
+  r.idx = w.idx;
+  r.second = fmax(w.second, l.best);
+  return r;
+}
+
+__device__ __forceinline__ Best warp_combine(Best v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Best w;
+    w.best = __shfl_xor_sync(0xFFFFFFFFu, v.best, o);
+    w.second = __shfl_xor_sync(0xFFFFFFFFu, v.second, o);
+    w.idx = __shfl_xor_sync(0xFFFFFFFFu, v.idx, o);
+    v = combine(v, w);
+  }
+  return v;
+}
+
+// log2 of E = -ln(1 - W), W = (o + 1/2) 2^-32, within 2^-12 relative in E.
+__device__ __forceinline__ float approx_log2_E(uint32_t o) {
+  // W < 2^-10: E = W + W^2/2 (the rest of the series is below 2^-20 relative)
+  const float fa = __uint_as_float(0x4B000000u | (o & 0x7FFFFFu)) - 8388608.0f;
+  const float Ws = (fa + 0.5f) * 0x1p-32f;
+  const float Es = fmaf(0.5f * Ws, Ws, Ws);
+  // otherwise E = -ln(U), U = 1 - W: exactly (~o + 1/2) 2^-32 when ~o < 2^23,
+  // else 1 - (o >> 9) 2^-23 (absolute error < 2^-23, U >= 2^-9 there)
+  const uint32_t no = ~o;
+  const float fc = __uint_as_float(0x4B000000u | (no & 0x7FFFFFu)) - 8388608.0f;
+  const float fb = __uint_as_float(0x4B000000u | (o >> 9)) - 8388608.0f;
+  const float U = no < 0x800000u ? (fc + 0.5f) * 0x1p-32f : fmaf(-fb, 0x1p-23f, 1.0f);
+  const float El = -0.693147180559945f * lg2_approx(U);
+  return lg2_approx(o < 0x400000u ? Es : El);
+}
+
+// The exact key ln r(x) - ln E_x in double precision, the plain definition's
+// formulas; -inf if x is no candidate.
+static __device__ __noinline__ double exact_key(float zt, float zq, int x, uint32_t o,
+                                         const RaceDesc& rd, bool residual) {
+  const double lp = (double)zt / rd.T - rd.lse_t;
+  if (lp == -INFINITY) return -INFINITY;
+  double lr = lp;
+  if (residual) {
+    double lq = (double)zq / rd.T - rd.lse_q;
+    if (rd.ntop > 0 && lq != -INFINITY) {
+      bool in_k = false;
+      for (int i = 0; i < rd.ntop; ++i) in_k |= (rd.top[i] == x);
+      lq += (in_k ? rd.ln_c : 0.0) - rd.ln_Z;
+    }
+    if (!(lp > lq)) return -INFINITY;
+    if (lq != -INFINITY) lr = lp + log(-expm1(lq - lp));
+  }
+  const double W = ((double)o + 0.5) * 0x1p-32;
+  return lr - log(-log1p(-W));
+}
+
+template <int DT>
+__device__ __forceinline__ float logit_at(const char* row, int x) {
+  if (DT == kF32) return ((const float*)row)[x];
+  return __uint_as_float((uint32_t)((const uint16_t*)row)[x] << 16);
+}
+
+// The race word of token x.
+__device__ __forceinline__ uint32_t race_word(uint64_t seed, uint32_t g, int x) {
+  const uint4 w = race_words(seed, g, (uint32_t)x >> 2);
+  const int l = x & 3;
+  return l == 0 ? w.x : l == 1 ? w.y : l == 2 ? w.z : w.w;
+}
+
+__device__ __forceinline__ double exact_key_of(const VerifyArgs& a, const RaceDesc& rd,
+                                               const char* trow, const char* qrow,
+                                               bool residual, int x) {
+  const float zt = (a.dtype == kF32) ? logit_at<kF32>(trow, x) : logit_at<kBF16>(trow, x);
+  float zq = 0.0f;
+  if (residual) zq = (a.dtype == kF32) ? logit_at<kF32>(qrow, x) : logit_at<kBF16>(qrow, x);
+  return exact_key(zt, zq, x, race_word(a.seed, rd.g, x), rd, residual);
+}
+
+// Upper bounds of the keys (log2 units) of one lane's tokens in segment `seg`;
+// calls visit(bound, x) for each.
+template <int DT, typename Visit>
+__device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc& rd,
+                                            const char* trow, const char* qrow, bool residual,
+                                            int seg, Visit&& visit) {
+  constexpr int VEC = DT == kF32 ? 4 : 8;
+  const int lane = threadIdx.x & 31;
+  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
+  const float k2 = rd.k2;
+  const float l2t = rd.l2_t, l2q = rd.l2_q;
+  // slack for the rounding of z*k2 - l2: relative 2^-21 of each term, plus 2^-22
+  const float ks = k2 * 0x1p-21f;
+  const float st0 = fabsf(l2t) * 0x1p-21f + 0x1p-22f;
+  const float sq0 = fabsf(l2q) * 0x1p-21f + 0x1p-22f;
+  const int nfull = a.V / VEC;
+  const bool aligned =
+      ((uintptr_t)trow & 15u) == 0 && (!residual || ((uintptr_t)qrow & 15u) == 0);
+#pragma unroll 1
+  for (int j = 0; j < kLaneVecs; ++j) {
+    const int v = seg * kSegVecs + lane + 32 * j;
+    if (v >= a.nvec) break;
+    uint4 wt, wq = make_uint4(0u, 0u, 0u, 0u);
+    if (aligned && v < nfull) {
+      wt = ld_stream16(trow + (size_t)v * 16);
+      if (residual) wq = ld_stream16(qrow + (size_t)v * 16);
+    } else {
+      wt = load_vec_checked<DT>(trow, v, a.V, a.nvec, nfull, aligned);
+      if (residual) wq = load_vec_checked<DT>(qrow, v, a.V, a.nvec, nfull, aligned);
+    }
+#pragma unroll
+    for (int h = 0; h < VEC / 4; ++h) {
+      const uint32_t base = (uint32_t)(v * VEC + 4 * h);
+      const uint4 o4 = philox4x32_10(make_uint4(base >> 2, rd.g, 1u, 0u), k0, k1);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int x = (int)base + e;
+        const float zt = elem<DT>(wt, 4 * h + e);
+        const uint32_t o = e == 0 ? o4.x : e == 1 ? o4.y : e == 2 ? o4.z : o4.w;
+        // ln p(x) - ln E_x, upper bound in log2 units
+        const float sp = fmaf(fabsf(zt), ks, st0);
+        const float l2p = fmaf(zt, k2, -l2t);
+        float bound = (l2p + sp) - (approx_log2_E(o) - 0x1p-11f);
+        if (residual) {
+          // r = p (1 - q/p): add the upper bound of log2(1 - 2^d), d = l2q - l2p
+          const float zq = elem<DT>(wq, 4 * h + e);
+          const float sq = fmaf(fabsf(zq), ks, sq0);
+          const float dlo = (fmaf(zq, k2, -l2q) - sq) - (l2p + sp);
+          const float t = fmaf(-ex2_approx(dlo), 1.0f - 0x1p-20f, 1.0f);
+          bound = (dlo < 0.0f) ? bound + (lg2_approx(t) + 0x1p-20f) : -INFINITY;
+        }
+        if (x < a.V && zt > -INFINITY) visit(bound, x);
+      }
+    }
+  }
+}
+
+// The exact best and runner-up of segment `seg` (all lanes get the result).
+template <int DT>
+__device__ __forceinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
+                                             const char* trow, const char* qrow,
+                                             bool residual, int seg) {
+  // A. the two largest bounds of each lane
+  float u1 = -INFINITY, u2 = -INFINITY;
+  int i1 = -1, i2 = -1;
+  race_bounds<DT>(a, rd, trow, qrow, residual, seg, [&](float bound, int x) {
+    if (bound > u2) {
+      if (bound > u1) {
+        u2 = u1;
+        i2 = i1;
+        u1 = bound;
+        i1 = x;
+      } else {
+        u2 = bound;
+        i2 = x;
+      }
+    }
+  });
+  // B. the exact key of each lane's best token
+  Best B{-INFINITY, -INFINITY, -1};
+  if (i1 >= 0) offer(B, exact_key_of(a, rd, trow, qrow, residual, i1), i1);
+  double S1 = B.best;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S1 = fmax(S1, __shfl_xor_sync(0xFFFFFFFFu, S1, o));
+  // C. every token whose bound reaches S1 (less the margin) gets its exact key
+  const float thr = S1 == -INFINITY ? -INFINITY : (float)(S1 * 1.4426950408889634) - 0x1p-14f;
+  if (i2 >= 0 && u2 >= thr) {
+    offer(B, exact_key_of(a, rd, trow, qrow, residual, i2), i2);
+    // the third bound may have reached thr as well: visit them all
+    const int j1 = i1, j2 = i2;
+    race_bounds<DT>(a, rd, trow, qrow, residual, seg, [&](float bound, int x) {
+      if (bound >= thr && x != j1 && x != j2)
+        offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
+    });
+  }
+  return warp_combine(B);
+}
+
+// Copy a request's race description into the warp's shared slot.
+__device__ __forceinline__ void load_race_desc(const RaceDesc* src, RaceDesc* dst) {
+  const int lane = threadIdx.x & 31;
+  constexpr int n16 = sizeof(RaceDesc) / 16;
+  static_assert(sizeof(RaceDesc) % 16 == 0, "RaceDesc is copied in 16-byte pieces");
+  if (lane < n16)
+    reinterpret_cast<uint4*>(dst)[lane] = __ldcg(reinterpret_cast<const uint4*>(src) + lane);
+  __syncwarp();
+}
+
+// Race segment `seg` of request b, by one warp (rd in the warp's shared slot).
+// The warp that completes the request's last segment merges and writes the token.
+template <int DT>
+__device__ inline void race_item(const VerifyArgs& a, int b, int seg, const RaceDesc& rd) {
+  const int lane = threadIdx.x & 31;
+  const bool residual = rd.kind == kRaceResidual;
+  const char* trow = row_base(a, b, rd.n);
+  const char* qrow = residual ? row_base(a, b, a.D_max + 1 + rd.n) : nullptr;
+  const Best sb = race_segment<DT>(a, rd, trow, qrow, residual, seg);
+
+  unsigned prev = 0;
+  if (lane == 0) {
+    RacePart p;
+    p.best = sb.best;
+    p.second = sb.second;
+    p.idx = sb.idx;
+    p.pad = 0;
+    a.rpart[(size_t)b * a.nseg + seg] = p;
+    __threadfence();
+    prev = atomicAdd(&a.rcount[b], 1u);
+  }
+  prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+  if (prev != (unsigned)(a.nseg - 1)) return;
+
+  // the last segment of this request: merge every segment's result
+  __threadfence();
+  Best r{-INFINITY, -INFINITY, -1};
+  for (int s = lane; s < a.nseg; s += 32) {
+    const RacePart* pp = a.rpart + (size_t)b * a.nseg + s;
+    Best o;
+    o.best = __ldcg(&pp->best);
+    o.second = __ldcg(&pp->second);
+    o.idx = __ldcg(&pp->idx);
+    r = combine(r, o);
+  }
+  r = warp_combine(r);
+  uint32_t flags = rd.flags;
+  if (r.idx < 0 && residual) {
+    // {p > q} was empty through rounding: draw from p on the same row instead
+    flags |= kFlagResidualEmpty;
+    Best Bb{-INFINITY, -INFINITY, -1};
+    for (int s = 0; s < a.nseg; ++s) Bb = combine(Bb, race_segment<DT>(a, rd, trow, nullptr, false, s));
+    r = Bb;
+  }
+  if (lane == 0) {
+    if (r.best - r.second < 1e-6) flags |= kFlagRaceNearTie;
+    a.out_tokens[(size_t)b * (a.D_max + 1) + rd.n] = r.idx;
+    if (a.out_flags) a.out_flags[b] = flags;
+    if (flags & kFlagResidualEmpty) atomicOr(a.status, kFlagResidualEmpty);
+  }
+}
+
+}  // namespace sv

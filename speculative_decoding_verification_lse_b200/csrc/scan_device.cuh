@@ -1,0 +1,265 @@
+// scan_device.cuh -- device code of the per-request accept scan, shared by the
+// split accept-scan kernel and the fused kernel.
+//
+// One warp per request.  The warp merges the segment partials of each row it
+// reads in double precision (merge_row), then lane d tests draft position d:
+//   a_d = min(1, p_d(x_d) / q_d(x_d))  ("Speculative Speculative Decoding –
+//   асинхронизируй это.", rule items 1-2, read as acceptance with probability
+//   min(1, p/q)), u_d from Philox, accept iff u_d < a_d;
+// a ballot gives n, the first rejected position ("NVIDIA: öt irányelv ...",
+// "Mit csinál a spekulatív dekódolás?": accept in order up to the first
+// mismatch), and AL = n + 1.
+// Greedy requests accept while x_d is the target row's argmax and emit the
+// argmax of row n.  Stochastic requests leave slot n to the race and describe
+// it in the workspace.  Saguaro requests use
+//   ln q'(x) = ln q(x) + [x in K] ln c - ln Z,  Z = 1 - (1 - c) sum_{x in K} q(x)
+// (saguaro recipe items 1-2: down-weight the draft's top tokens, renormalised).
+#pragma once
+#include "philox.cuh"
+#include "sv_common.cuh"
+
+#include <float.h>
+#include <limits.h>
+#include <math.h>
+
+namespace sv {
+
+constexpr double kLn2d = 0.69314718055994530942;
+
+struct RowRes {
+  double lse;   // natural-log LSE at T (stochastic rows)
+  double lnZ;   // saguaro draft rows: ln Z
+  int argmax;   // target rows
+  uint32_t bad;
+  int ntop;
+  int top[kMaxTopK];
+  float topv[kMaxTopK];
+};
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Merge the segment partials of one row, by the whole warp (lane l takes
+// segments l, l+32, ...; the partials were written by other warps, so they are
+// read through L2).  Every lane returns the same RowRes.
+//   LSE = ln2 * (Mk + log2 sum_s S_s 2^(m_s k2 - Mk)),  Mk = M k2, M = max_s m_s
+__device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg, bool lse,
+                                 float k2, int k, RowRes& r) {
+  const int lane = threadIdx.x & 31;
+  float mx = -INFINITY;
+  int am = INT_MAX;
+  uint32_t bad = 0;
+  double Sd = 0.0;  // relative to 2^(mx*k2)
+  for (int s = lane; s < nseg; s += 32) {
+    const float4 raw = __ldcg(reinterpret_cast<const float4*>(ps + s));
+    const float m = raw.x, S = raw.y;
+    const int ai = __float_as_int(raw.z);
+    bad |= __float_as_uint(raw.w);
+    if (m > mx) {  // segments ascend in index: strict '>' keeps the lowest index
+      if (lse && Sd > 0.0) Sd *= exp2((double)(mx * k2) - (double)(m * k2));
+      mx = m;
+      am = ai;
+    }
+    if (lse && S > 0.0f) Sd += (double)S * exp2((double)(m * k2) - (double)(mx * k2));
+  }
+  const unsigned long long key = value_index_key(mx, am == INT_MAX ? INT_MAX - 1 : am);
+  const unsigned long long win = warp_max_u64(key);
+  const float M = key_value(win);
+  const int Mi = key_index(win);
+  bad = __any_sync(0xFFFFFFFFu, bad) ? 1u : 0u;
+  if (M == -INFINITY) bad = 1u;  // every entry masked: no distribution
+  r.argmax = (Mi == INT_MAX - 1) ? INT_MAX : Mi;
+  r.lse = NAN;
+  if (lse) {
+    const double Mk = (double)(M * k2);
+    double part = 0.0;
+    if (Sd > 0.0) part = Sd * exp2((double)(mx * k2) - Mk);
+    const double S = warp_sum_d(part);
+    if (!bad) r.lse = (Mk + log2(S)) * kLn2d;
+  }
+  r.ntop = 0;
+  if (tp) {
+    // k rounds: each lane offers the best head of its segments' lists
+    int head[kMaxSegs / 32];
+    const int mine = (nseg - lane + 31) / 32;
+    for (int i = 0; i < mine; ++i) head[i] = 0;
+    for (int rd = 0; rd < k; ++rd) {
+      unsigned long long best = 0ull;
+      int bi = -1;
+      for (int i = 0; i < mine; ++i) {
+        if (head[i] >= k) continue;
+        const TopPart* t = tp + lane + 32 * i;
+        const int ci = __ldcg(&t->i[head[i]]);
+        if (ci == INT_MAX) continue;
+        const unsigned long long kk = value_index_key(__ldcg(&t->v[head[i]]), ci);
+        if (kk > best) {
+          best = kk;
+          bi = i;
+        }
+      }
+      const unsigned long long w = warp_max_u64(best);
+      if (w == 0ull) break;
+      if (best == w) ++head[bi];
+      r.top[r.ntop] = key_index(w);
+      r.topv[r.ntop] = key_value(w);
+      ++r.ntop;
+    }
+  }
+  r.bad = bad;
+}
+
+// The accept scan of request b by one full warp; rows: 2*D_max+1 entries of
+// shared memory.  Writes the outputs (slot n too for greedy), the flags, the
+// row LSEs and the race description; returns the race kind (same on all lanes).
+__device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
+  const int lane = threadIdx.x & 31;
+  const int Dm = a.D_max;
+  const ReqParams rp = load_req(a, b);
+  const uint32_t g = a.request_offset + (uint32_t)b;
+  int32_t* ot = a.out_tokens + (size_t)b * (Dm + 1);
+  uint32_t err = rp.err;
+
+  // draft tokens of the tested positions
+  int x = -1;
+  if (!err && lane < rp.Db) {
+    x = a.tokens[(size_t)b * Dm + lane];
+    if (x < 0 || x >= a.V) err |= kFlagBadToken;
+  }
+  err = __reduce_or_sync(0xFFFFFFFFu, err);
+
+  const bool greedy = rp.mode == kGreedy;
+  const bool saguaro = rp.mode == kSaguaro;
+  const double Td = (double)rp.T;
+  const double c = (double)a.saguaro_c;
+
+  // merge the rows this request reads, one row at a time with the whole warp
+  if (!err) {
+    const float k2 = greedy ? 0.0f : log2e_over_T(rp.T);
+    uint32_t nonfinite = 0;
+    for (int slot = 0; slot < a.slots; ++slot) {
+      const bool is_t = slot <= Dm;
+      const int d = is_t ? slot : slot - Dm - 1;
+      const bool needed = is_t ? d <= rp.Db : (d < rp.Db && !greedy);
+      if (!needed) continue;
+      const PartStat* ps = a.pstat + ((size_t)b * a.slots + slot) * a.nseg;
+      const TopPart* tp =
+          (!is_t && saguaro) ? a.tpart + ((size_t)b * Dm + d) * a.nseg : nullptr;
+      RowRes rr;
+      merge_row(ps, tp, a.nseg, !greedy, k2, a.saguaro_k, rr);
+      nonfinite |= rr.bad ? kFlagNonfinite : 0u;
+      if (tp && !rr.bad) {
+        // Z = 1 - (1 - c) * sum_{x in K} q(x)
+        double mass = 0.0;
+        for (int i = 0; i < rr.ntop; ++i) mass += exp((double)rr.topv[i] / Td - rr.lse);
+        rr.lnZ = log1p(-(1.0 - c) * mass);
+      }
+      if (lane == 0) rows[slot] = rr;
+    }
+    err |= nonfinite;
+  }
+  __syncwarp();
+
+  if (err) {
+    for (int j = lane; j <= Dm; j += 32) ot[j] = -1;
+    if (a.out_row_lse)
+      for (int s = lane; s < a.slots; s += 32) a.out_row_lse[(size_t)b * a.slots + s] = NAN;
+    if (lane == 0) {
+      a.out_al[b] = -1;
+      if (a.out_flags) a.out_flags[b] = err;
+      atomicOr(a.status, err);
+      a.rdesc[b].kind = kRaceNone;
+    }
+    return kRaceNone;
+  }
+
+  // test every draft position in parallel
+  bool accept = false, near = false;
+  if (lane < rp.Db) {
+    if (greedy) {
+      accept = (x == rows[lane].argmax);
+    } else {
+      const char* trow = row_base(a, b, lane);
+      const char* qrow = row_base(a, b, Dm + 1 + lane);
+      const RowRes& rq = rows[Dm + 1 + lane];
+      const double lp = (double)load_logit(a, trow, x) / Td - rows[lane].lse;
+      double lq = (double)load_logit(a, qrow, x) / Td - rq.lse;
+      if (saguaro && lq != -INFINITY) {
+        bool in_k = false;
+        for (int i = 0; i < rq.ntop; ++i) in_k |= (rq.top[i] == x);
+        lq += (in_k ? log(c) : 0.0) - rq.lnZ;
+      }
+      double acc;
+      if (lp == -INFINITY)
+        acc = 0.0;  // p(x) = 0: the target never emits x
+      else if (lq == -INFINITY)
+        acc = 1.0;
+      else
+        acc = fmin(1.0, exp(lp - lq));
+      const double u = (double)(accept_word(a.seed, g, (uint32_t)lane) >> 8) * 0x1p-24;
+      accept = u < acc;
+      near = fabs(u - acc) < 1e-5;
+    }
+  }
+  const uint32_t rej = __ballot_sync(0xFFFFFFFFu, lane < rp.Db && !accept);
+  const int n = rej ? __ffs(rej) - 1 : rp.Db;
+  const uint32_t nearm = __ballot_sync(0xFFFFFFFFu, near);
+  const uint32_t tested = (n < rp.Db) ? (uint32_t)((2ull << n) - 1ull)
+                                      : (uint32_t)((1ull << rp.Db) - 1ull);
+  const uint32_t flags = (nearm & tested) ? kFlagAcceptNearTie : 0u;
+  const int kind = greedy ? kRaceNone : (n < rp.Db ? kRaceResidual : kRaceBonus);
+
+  // outputs: accepted drafts, then slot n, then -1
+  for (int j = lane; j <= Dm; j += 32) {
+    int v = -1;
+    if (j < n)
+      v = a.tokens[(size_t)b * Dm + j];
+    else if (j == n && greedy)
+      v = rows[n].argmax;
+    ot[j] = v;
+  }
+  if (a.out_row_lse) {
+    for (int s = lane; s < a.slots; s += 32) {
+      const bool is_t = s <= Dm;
+      const int d = is_t ? s : s - Dm - 1;
+      const bool used = !greedy && (is_t ? d <= rp.Db : d < rp.Db);
+      a.out_row_lse[(size_t)b * a.slots + s] = used ? (float)rows[s].lse : NAN;
+    }
+  }
+  if (lane == 0) {
+    a.out_al[b] = n + 1;
+    if (a.out_flags) a.out_flags[b] = flags;
+    RaceDesc rd;
+    rd.kind = kind;
+    rd.n = n;
+    rd.g = g;
+    rd.flags = flags;
+    rd.T = Td;
+    rd.lse_t = rows[n].lse;
+    rd.k2 = log2e_over_T(rp.T);
+    rd.l2_t = (float)(rows[n].lse * 1.4426950408889634);
+    rd.l2_q = 0.0f;
+    rd.lse_q = 0.0;
+    rd.ln_c = log(c);
+    rd.ln_Z = 0.0;
+    rd.ntop = 0;
+    if (kind == kRaceResidual) {
+      const RowRes& rq = rows[Dm + 1 + n];
+      rd.lse_q = rq.lse;
+      double shift = rq.lse;
+      if (saguaro) {
+        rd.ln_Z = rq.lnZ;
+        rd.ntop = rq.ntop;
+        for (int i = 0; i < rq.ntop; ++i) rd.top[i] = rq.top[i];
+        shift = rq.lse - rd.ln_c + rq.lnZ;
+      }
+      rd.l2_q = (float)(shift * 1.4426950408889634);
+    }
+    a.rdesc[b] = rd;
+  }
+  return kind;
+}
+
+}  // namespace sv

@@ -1,0 +1,293 @@
+// stats_device.cuh -- device code of the per-row statistics pass, shared by the
+// split row_stats kernel and the fused kernel.
+//
+// For every row the rule reads (target rows 0..D_b, draft rows 0..D_b-1 of
+// non-greedy requests) one warp computes, per 8 KiB segment, the partial
+// log-sum-exp state of softmax(z / T), the lowest-index argmax (target rows)
+// and the k largest logits (saguaro draft rows).
+//
+// Sources: "Accélérer Sonar par la Spéculation", section "Cible-Brouillon"
+// (the sampler compares the full draft and target distributions, so both
+// normalisers are needed); "Speculative Speculative Decoding – асинхронизируй
+// это.", saguaro recipe item 1 (the draft's top tokens).
+//
+// Each lane issues its sixteen 16-byte loads at once (8 KiB in flight per
+// warp), takes its maximum on packed bf16 pairs, the warp agrees on the segment
+// maximum with five shuffles, and then every element costs one FFMA, one ex2
+// and one FADD relative to that maximum -- no per-element rescaling, no
+// barrier, no shared memory.
+#pragma once
+#include "sv_common.cuh"
+
+#include <float.h>
+#include <limits.h>
+
+namespace sv {
+
+constexpr uint32_t kNegInfBf2 = 0xFF80FF80u;  // two bf16 -inf
+constexpr uint32_t kNegInfF32 = 0xFF800000u;
+
+// Vector v of a row (VEC elements), -inf past V; element loads where the row
+// is not 16-byte aligned or the vector crosses the end of the row.
+template <int DT>
+__device__ __forceinline__ uint4 load_vec_checked(const char* row, int v, int V, int nvec,
+                                                  int nfull, bool aligned) {
+  const uint32_t fill = DT == kF32 ? kNegInfF32 : kNegInfBf2;
+  if (v >= nvec) return make_uint4(fill, fill, fill, fill);
+  if (aligned && v < nfull) return ld_stream16(row + (size_t)v * 16);
+  uint32_t w[4];
+  if (DT == kF32) {
+    const float* r = (const float*)row;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int x = v * 4 + e;
+      w[e] = x < V ? __float_as_uint(r[x]) : kNegInfF32;
+    }
+  } else {
+    const uint16_t* r = (const uint16_t*)row;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int x = v * 8 + 2 * e;
+      const uint32_t lo = x < V ? (uint32_t)r[x] : 0xFF80u;
+      const uint32_t hi = x + 1 < V ? (uint32_t)r[x + 1] : 0xFF80u;
+      w[e] = lo | (hi << 16);
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t w) {
+  __nv_bfloat162 r;
+  memcpy(&r, &w, 4);
+  return r;
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// Element e (0..VEC-1) of a loaded vector, widened to float.
+template <int DT>
+__device__ __forceinline__ float elem(const uint4& v, int e) {
+  if (DT == kF32) return __uint_as_float(word(v, e));
+  const uint32_t w = word(v, e >> 1);
+  return (e & 1) ? bf_hi(w) : bf_lo(w);
+}
+
+// Load the lane's kLaneVecs vectors of segment `seg`.
+template <int DT>
+__device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* row, int seg,
+                                             uint4 (&raw)[kLaneVecs]) {
+  constexpr int VEC = DT == kF32 ? 4 : 8;
+  const int lane = threadIdx.x & 31;
+  const int nfull = a.V / VEC;
+  const int v0 = seg * kSegVecs + lane;
+  const bool aligned = ((uintptr_t)row & 15u) == 0;
+  if (aligned && (seg + 1) * kSegVecs <= nfull) {
+    // whole segment inside the row: unchecked streaming loads
+#pragma unroll
+    for (int j = 0; j < kLaneVecs; ++j) raw[j] = ld_stream16(row + (size_t)(v0 + 32 * j) * 16);
+  } else {
+#pragma unroll
+    for (int j = 0; j < kLaneVecs; ++j)
+      raw[j] = load_vec_checked<DT>(row, v0 + 32 * j, a.V, a.nvec, nfull, aligned);
+  }
+}
+
+// Statistics of segment `seg` of one row, by one full warp.
+template <int DT, bool LSE, bool ARGMAX, bool TOP>
+__device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* row, int seg,
+                                              float k2, int topk, PartStat* out, TopPart* tout) {
+  constexpr int VEC = DT == kF32 ? 4 : 8;
+  const int lane = threadIdx.x & 31;
+  const int v0 = seg * kSegVecs + lane;
+  uint4 raw[kLaneVecs];
+  load_segment<DT>(a, row, seg, raw);
+
+  // ---- lane maximum, with NaN / +inf detection
+  float m_t;
+  uint32_t bad = 0;
+  if (DT == kBF16) {
+    __nv_bfloat162 mx = as_bf2(raw[0].x);
+#pragma unroll
+    for (int j = 0; j < kLaneVecs; ++j) {
+      mx = __hmax2_nan(mx, as_bf2(raw[j].x));
+      mx = __hmax2_nan(mx, as_bf2(raw[j].y));
+      mx = __hmax2_nan(mx, as_bf2(raw[j].z));
+      mx = __hmax2_nan(mx, as_bf2(raw[j].w));
+    }
+    const float lo = __low2float(mx), hi = __high2float(mx);
+    bad = (lo != lo) | (hi != hi) | (lo == INFINITY) | (hi == INFINITY);
+    m_t = fmaxf(lo, hi);
+  } else {
+    m_t = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kLaneVecs; ++j)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float z = elem<DT>(raw[j], e);
+        bad |= (z != z) | (z == INFINITY);
+        m_t = fmaxf(m_t, z);
+      }
+  }
+  const float m_w = warp_max(m_t);
+  const uint32_t bad_w = __any_sync(0xFFFFFFFFu, bad) ? 1u : 0u;
+
+  // ---- sum of 2^(z*k2 - mk): one FFMA, one ex2 and one FADD per element
+  float S_w = 0.0f;
+  if (LSE) {
+    float S_t = 0.0f;
+    if (m_w > -INFINITY) {
+      const float mk = m_w * k2;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < kLaneVecs; ++j)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e)
+          acc[(j * VEC + e) & 7] += ex2_approx(fmaf(elem<DT>(raw[j], e), k2, -mk));
+      S_t = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    }
+    S_w = warp_sum(S_t);
+  }
+
+  // ---- lowest index of the segment maximum (only lanes holding it search)
+  int idx_w = INT_MAX;
+  if (ARGMAX) {
+    int idx_t = INT_MAX;
+    if (m_t == m_w) {
+#pragma unroll
+      for (int j = kLaneVecs - 1; j >= 0; --j)
+#pragma unroll
+        for (int e = VEC - 1; e >= 0; --e)
+          if (elem<DT>(raw[j], e) == m_w) idx_t = (v0 + 32 * j) * VEC + e;
+    }
+    idx_w = warp_min_int(idx_t);
+  }
+
+  // ---- the k largest logits (value desc, index asc), saguaro draft rows
+  if (TOP) {
+    float tv[kMaxTopK];
+    int ti[kMaxTopK];
+#pragma unroll
+    for (int s = 0; s < kMaxTopK; ++s) {
+      tv[s] = -INFINITY;
+      ti[s] = INT_MAX;
+    }
+#pragma unroll
+    for (int j = 0; j < kLaneVecs; ++j)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float z = elem<DT>(raw[j], e);
+        if (z > tv[kMaxTopK - 1]) {
+          // elements arrive in increasing index order, so an equal value stays
+          // below the earlier (lower-index) one: strict comparisons throughout
+          tv[kMaxTopK - 1] = z;
+          ti[kMaxTopK - 1] = (v0 + 32 * j) * VEC + e;
+#pragma unroll
+          for (int s = kMaxTopK - 1; s > 0; --s) {
+            if (tv[s] > tv[s - 1]) {
+              const float fv = tv[s];
+              tv[s] = tv[s - 1];
+              tv[s - 1] = fv;
+              const int fi = ti[s];
+              ti[s] = ti[s - 1];
+              ti[s - 1] = fi;
+            }
+          }
+        }
+      }
+    int h = 0;
+    for (int r = 0; r < topk; ++r) {
+      float hv = -INFINITY;
+      int hi = INT_MAX;
+#pragma unroll
+      for (int s = 0; s < kMaxTopK; ++s)
+        if (s == h) {
+          hv = tv[s];
+          hi = ti[s];
+        }
+      const unsigned long long key = hi == INT_MAX ? 0ull : value_index_key(hv, hi);
+      const unsigned long long win = warp_max_u64(key);
+      if (win != 0ull && key == win) ++h;
+      if (lane == 0) {
+        tout->v[r] = win ? key_value(win) : -INFINITY;
+        tout->i[r] = win ? key_index(win) : INT_MAX;
+      }
+    }
+  }
+
+  if (lane == 0) {
+    PartStat p;
+    p.m = m_w;
+    p.S = S_w;
+    p.argmax = idx_w;
+    p.bad = bad_w;
+    *out = p;
+  }
+}
+
+// Whether row `slot` of a request with parameters rp is read by the rule.
+__device__ __forceinline__ bool row_needed(const VerifyArgs& a, int slot, const ReqParams& rp) {
+  if (rp.err) return false;
+  const bool is_target = slot <= a.D_max;
+  const int d = is_target ? slot : slot - a.D_max - 1;
+  return is_target ? d <= rp.Db : (d < rp.Db && rp.mode != kGreedy);
+}
+
+// Statistics of segment `seg` of row `slot` of request b (one full warp).
+template <int DT>
+__device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot, int seg,
+                                           const ReqParams& rp) {
+  const bool is_target = slot <= a.D_max;
+  const char* row = row_base(a, b, slot);
+  PartStat* out = a.pstat + ((size_t)b * a.slots + slot) * a.nseg + seg;
+  const float k2 = rp.mode == kGreedy ? 0.0f : log2e_over_T(rp.T);
+  if (is_target) {
+    if (rp.mode == kGreedy)
+      stats_segment<DT, false, true, false>(a, row, seg, k2, 0, out, nullptr);
+    else
+      stats_segment<DT, true, true, false>(a, row, seg, k2, 0, out, nullptr);
+  } else if (rp.mode == kSaguaro) {
+    TopPart* tout = a.tpart + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * a.nseg + seg;
+    stats_segment<DT, true, false, true>(a, row, seg, k2, a.saguaro_k, out, tout);
+  } else {
+    stats_segment<DT, true, false, false>(a, row, seg, k2, 0, out, nullptr);
+  }
+}
+
+// (b, slot, seg) of work item `it` of the request-major item order, advanced
+// in steps of `stride` items without divisions.
+struct ItemWalker {
+  int b, slot, seg;
+  int d_b, d_slot, d_seg;  // the stride decomposed the same way
+  __device__ __forceinline__ void init(const VerifyArgs& a, unsigned it, unsigned stride) {
+    const unsigned per_req = (unsigned)a.slots * (unsigned)a.nseg;
+    b = (int)(it / per_req);
+    const unsigned r = it % per_req;
+    slot = (int)(r / (unsigned)a.nseg);
+    seg = (int)(r % (unsigned)a.nseg);
+    d_b = (int)(stride / per_req);
+    const unsigned dr = stride % per_req;
+    d_slot = (int)(dr / (unsigned)a.nseg);
+    d_seg = (int)(dr % (unsigned)a.nseg);
+  }
+  __device__ __forceinline__ void advance(const VerifyArgs& a) {
+    seg += d_seg;
+    int carry = 0;
+    if (seg >= a.nseg) {
+      seg -= a.nseg;
+      carry = 1;
+    }
+    slot += d_slot + carry;
+    carry = 0;
+    if (slot >= a.slots) {
+      slot -= a.slots;
+      carry = 1;
+    }
+    b += d_b + carry;
+  }
+};
+
+}  // namespace sv

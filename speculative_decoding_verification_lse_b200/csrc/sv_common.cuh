@@ -1,11 +1,15 @@
 // sv_common.cuh -- layouts and device helpers shared by the libspecverify kernels.
 //
 // Row decomposition (fixed by V and dtype only, so that identical rows always
-// reduce in the same order and give bit-identical statistics):
+// reduce in the same order and give bit-identical statistics, whatever the
+// batch around them):
 //   a row of V logits is read as 16-byte vectors of VEC elements (8 bf16 or 4 fp32);
-//   a chunk is kChunkVecs = kThreads * kVecsPerThread consecutive vectors;
-//   thread t of the CTA handling chunk c owns vectors c*kChunkVecs + t + j*kThreads,
-//   j = 0..kVecsPerThread-1, so each warp reads 512 contiguous bytes per j.
+//   a segment is kSegVecs = 32 * kLaneVecs consecutive vectors (8 KiB), handled by
+//   one warp: lane l owns vectors seg*kSegVecs + l + 32*j, j = 0..kLaneVecs-1, so
+//   the warp reads 512 contiguous bytes per j.
+//   Each segment yields one partial (its maximum, the sum of 2^(z*k2 - max*k2),
+//   the lowest index of its maximum); a row's partials are merged in segment
+//   order by one warp in double precision.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -14,11 +18,13 @@
 
 namespace sv {
 
-constexpr int kThreads = 256;        // threads per statistics / race CTA
-constexpr int kVecsPerThread = 8;    // 16-byte vectors per thread per chunk
-constexpr int kChunkVecs = kThreads * kVecsPerThread;  // 2048 vectors = 32 KiB per chunk
+constexpr int kThreads = 256;        // threads per CTA (8 independent warps)
+constexpr int kWarps = kThreads / 32;
+constexpr int kLaneVecs = 16;        // 16-byte vectors per lane per segment
+constexpr int kSegVecs = 32 * kLaneVecs;  // 512 vectors = 8 KiB per segment
 constexpr int kMaxDraft = 32;
 constexpr int kMaxTopK = 8;
+constexpr int kMaxSegs = 1024;       // segments per row (V up to 2^21 bf16 / 2^20 fp32)
 constexpr int kScanWarps = 4;        // requests per accept-scan CTA
 
 enum : int { kF32 = 0, kBF16 = 1 };
@@ -36,23 +42,23 @@ enum : uint32_t {
   kFlagErrors = kFlagBadToken | kFlagBadRowD | kFlagNonfinite | kFlagBadParam
 };
 
-// Partial statistics of one chunk of one row.
-//   m   : largest logit in the chunk (raw, as float); -inf if every entry is -inf
-//   mk  : fl(m * k2), k2 = fl(log2(e) / T): the offset the chunk's exponents used
-//   S   : sum over the chunk of 2^(fl(z*k2 - mk))   (so S * 2^mk = sum 2^(z*k2))
-//   argmax: lowest index of m inside the chunk (INT_MAX if none)
-//   bad : nonzero if a NaN or +inf was seen
-//   top : the chunk's largest logits (value desc, index asc), saguaro draft rows only
-struct __align__(16) ChunkStat {
+// Partial statistics of one segment of one row (16 bytes).
+//   m     : largest logit in the segment (raw, as float); -inf if all are -inf
+//   S     : sum over the segment of 2^(fl(z*k2 - mk)), mk = fl(m*k2),
+//           k2 = fl(log2(e) / T); so S * 2^mk = sum 2^(z*k2)
+//   argmax: lowest index of m inside the segment
+//   bad   : nonzero if a NaN or +inf was seen
+struct __align__(16) PartStat {
   float m;
-  float mk;
   float S;
   int argmax;
   uint32_t bad;
-  int ntop;
-  float topv[kMaxTopK];
-  int topi[kMaxTopK];
-  int pad[2];
+};
+
+// The k largest logits of one segment (value desc, index asc), saguaro draft rows.
+struct __align__(16) TopPart {
+  float v[kMaxTopK];
+  int i[kMaxTopK];
 };
 
 // What the race of one request needs; written by the accept scan.
@@ -68,16 +74,26 @@ struct __align__(16) RaceDesc {
   double ln_Z;       // saguaro: ln Z of draft row n
   float k2;          // fl(log2(e) / T)
   float l2_t;        // fl(lse_t * log2(e))
+  float l2_q;        // fl((lse_q - ln c + ln Z) * log2(e)) (saguaro), fl(lse_q * log2(e)) else:
+                     // z*k2 - l2_q is then a lower bound of log2 q'(x) for every x
   int ntop;          // saguaro: size of K (0 otherwise)
   int top[kMaxTopK]; // saguaro: K of draft row n
 };
 
-// One race chunk's result: the best and second-best exact keys and the winner.
+// One race segment's result: the best and second-best exact keys and the winner.
 struct __align__(16) RacePart {
   double best;
   double second;
-  int idx;           // -1 if the chunk had no candidate
+  int idx;           // -1 if the segment had no candidate
   int pad;
+};
+
+// Counters of the fused kernel (each on its own 128-byte line).
+struct __align__(128) FusedState {
+  unsigned int next_ticket;   // next statistics item
+  unsigned int pad0[31];
+  unsigned int cursor;        // request whose race chunks are being claimed
+  unsigned int pad1[31];
 };
 
 // Everything a kernel needs, passed by value.
@@ -93,13 +109,18 @@ struct VerifyArgs {
   float* out_row_lse;
   uint32_t* out_flags;
   unsigned int* status;    // the device status word
-  ChunkStat* cstat;        // [B, slots, nch]
+  PartStat* pstat;         // [B, slots, nseg]
+  TopPart* tpart;          // [B, D_max, nseg] (saguaro draft rows)
   RaceDesc* rdesc;         // [B]
-  RacePart* rpart;         // [B, nch]
-  unsigned int* rcount;    // [B]
+  RacePart* rpart;         // [B, nseg]
+  unsigned int* rcount;    // [B] race segments finished
+  FusedState* fstate;      // fused kernel: tickets and race cursor
+  unsigned int* done;      // [B] fused kernel: statistics items finished
+  unsigned int* ready;     // [B] fused kernel: 0 running, 1 race published, 2 nothing to race
+  unsigned int* rclaim;    // [B] fused kernel: race segments claimed
   uint64_t seed;
   int B, D_max, V, dtype;
-  int nvec, nch, slots;
+  int nvec, nseg, slots;
   int mode;
   float temperature;
   int saguaro_k;
@@ -108,35 +129,47 @@ struct VerifyArgs {
 };
 
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
+// [zero, total) holds the counters that must read zero when a fused launch starts.
 struct WsLayout {
-  size_t cstat, rdesc, rpart, rcount, total;
+  size_t pstat, tpart, rdesc, rpart, zero, fstate, rcount, done, ready, rclaim, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline int vec_elems(int dtype) { return dtype == kF32 ? 4 : 8; }
 
-inline void row_geometry(int V, int dtype, int* nvec, int* nch) {
+inline void row_geometry(int V, int dtype, int* nvec, int* nseg) {
   const int ve = vec_elems(dtype);
   *nvec = (V + ve - 1) / ve;
-  *nch = (*nvec + kChunkVecs - 1) / kChunkVecs;
+  *nseg = (*nvec + kSegVecs - 1) / kSegVecs;
 }
 
-inline WsLayout ws_layout(int B, int D_max, int V, int dtype) {
-  int nvec, nch;
-  row_geometry(V, dtype, &nvec, &nch);
+inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
+  int nvec, nseg;
+  row_geometry(V, dtype, &nvec, &nseg);
   const size_t slots = 2 * (size_t)D_max + 1;
   WsLayout L;
   size_t off = 0;
-  L.cstat = off;
-  off = align_up(off + (size_t)B * slots * nch * sizeof(ChunkStat), 256);
+  L.pstat = off;
+  off = align_up(off + (size_t)B * slots * nseg * sizeof(PartStat), 256);
+  L.tpart = off;
+  off = align_up(off + (saguaro ? (size_t)B * D_max * nseg * sizeof(TopPart) : 0), 256);
   L.rdesc = off;
   off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
   L.rpart = off;
-  off = align_up(off + (size_t)B * nch * sizeof(RacePart), 256);
+  off = align_up(off + (size_t)B * nseg * sizeof(RacePart), 256);
+  L.zero = off;
+  L.fstate = off;
+  off = align_up(off + sizeof(FusedState), 256);
   L.rcount = off;
   off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
-  L.total = off > 0 ? off : 256;
+  L.done = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.ready = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.rclaim = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.total = off;
   return L;
 }
 
@@ -225,9 +258,9 @@ struct ReqParams {
 
 __device__ __forceinline__ ReqParams load_req(const VerifyArgs& a, int b) {
   ReqParams r;
-  r.Db = a.row_D ? a.row_D[b] : a.D_max;
-  r.mode = a.mode_per_req ? (int)a.mode_per_req[b] : a.mode;
-  r.T = a.temp_per_req ? a.temp_per_req[b] : a.temperature;
+  r.Db = a.row_D ? __ldg(&a.row_D[b]) : a.D_max;
+  r.mode = a.mode_per_req ? (int)__ldg(&a.mode_per_req[b]) : a.mode;
+  r.T = a.temp_per_req ? __ldg(&a.temp_per_req[b]) : a.temperature;
   r.err = 0;
   if (r.Db < 0 || r.Db > a.D_max) r.err |= kFlagBadRowD;
   if (r.mode != kStochastic && r.mode != kGreedy && r.mode != kSaguaro) r.err |= kFlagBadParam;
@@ -235,6 +268,9 @@ __device__ __forceinline__ ReqParams load_req(const VerifyArgs& a, int b) {
   if (r.mode != kGreedy && a.draft == nullptr && r.Db > 0) r.err |= kFlagBadParam;
   return r;
 }
+
+// k2 = fl(log2(e) / T): the one scale every kernel applies to logits.
+__device__ __forceinline__ float log2e_over_T(float T) { return __fdiv_rn(1.44269504088896341f, T); }
 
 __device__ __forceinline__ const char* row_base(const VerifyArgs& a, int b, int slot) {
   const size_t es = a.dtype == kF32 ? 4 : 2;
@@ -252,7 +288,11 @@ __device__ __forceinline__ float load_logit(const VerifyArgs& a, const char* row
 
 // Host-side launchers (one per kernel file), called from the C ABI.
 namespace sv {
-cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s, int grid);
+int row_stats_blocks_per_sm(int dtype);
 cudaError_t launch_accept_scan(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
+size_t fused_smem_bytes(int D_max);
+int fused_blocks_per_sm(int dtype);
 }  // namespace sv
