@@ -173,7 +173,9 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
 
-  const WsLayout L = ws_layout(B, D_max, V, dtype, saguaro_possible);
+  // the same layout sv_workspace_bytes reports, whatever the modes
+  const WsLayout L = ws_layout(B, D_max, V, dtype, true);
+  (void)saguaro_possible;
   void* ws = prm.workspace;
   unsigned int* status = nullptr;
   const bool fused = prm.variant == SV_VARIANT_FUSED;

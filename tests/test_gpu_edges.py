@@ -15,6 +15,9 @@ from speculative_decoding_verification_lse_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
+VARIANTS = pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED],
+                                   ids=["split", "fused"])
+
 
 def make_random(B, D, V, dtype=sv.SV_BF16, seed=0, draft_sd=1.0, T=1.0, mode=0):
     w = wl.make("tiny", "cuda", B=B, D=D, V=V, seed=seed, dtype=dtype, T=T, mode=mode,
@@ -22,25 +25,28 @@ def make_random(B, D, V, dtype=sv.SV_BF16, seed=0, draft_sd=1.0, T=1.0, mode=0):
     return w
 
 
-@pytest.mark.parametrize("V", [1, 2, 5, 7, 8, 9, 100, 1023, 16384, 16384 * 8 + 1, 16384 * 8 + 9])
+@VARIANTS
+@pytest.mark.parametrize("V", [1, 2, 5, 7, 8, 9, 100, 1023, 4096, 4096 * 8 + 1, 4096 * 8 + 9])
 @pytest.mark.parametrize("dtype", [sv.SV_F32, sv.SV_BF16])
-def test_vocab_sizes_and_alignment(sv, V, dtype):
+def test_vocab_sizes_and_alignment(sv, V, dtype, variant):
     # odd V makes every row after the first start off a 16-byte boundary
     w = make_random(5, 3, V, dtype=dtype, seed=V)
     for mode in (0, 1, 2):
         w.mode = mode
-        compare(w, gpu_run(w, seed=mode), oracle_on(w, seed=mode))
+        compare(w, gpu_run(w, seed=mode, variant=variant), oracle_on(w, seed=mode))
 
 
+@VARIANTS
 @pytest.mark.parametrize("D", [0, 1, 32])
-def test_draft_lengths(sv, D):
+def test_draft_lengths(sv, D, variant):
     w = make_random(6, D, 3000, seed=D)
     for mode in (0, 1, 2):
         w.mode = mode
-        compare(w, gpu_run(w), oracle_on(w))
+        compare(w, gpu_run(w, variant=variant), oracle_on(w))
 
 
-def test_row_D_with_zero_and_nan_padding(sv):
+@VARIANTS
+def test_row_D_with_zero_and_nan_padding(sv, variant):
     w = make_random(8, 5, 5000, seed=3)
     row_D = torch.tensor([0, 5, 1, 0, 3, 5, 2, 4], dtype=torch.int32, device="cuda")
     for b, d in enumerate(row_D.tolist()):
@@ -50,7 +56,7 @@ def test_row_D_with_zero_and_nan_padding(sv):
     w.row_D = row_D
     for mode in (0, 1, 2):
         w.mode = mode
-        got = gpu_run(w)
+        got = gpu_run(w, variant=variant)
         assert np.all((got["flags"] & sv.SV_FLAG_ERRORS) == 0)
         compare(w, got, oracle_on(w))
     assert sv.sv_get_device_status() == 0
@@ -77,14 +83,15 @@ def test_masked_tokens(sv):
     assert np.all(emitted % 3 != 0)  # p = 0 tokens are never emitted
 
 
-def test_invalid_device_inputs_set_flags_and_status(sv):
+@VARIANTS
+def test_invalid_device_inputs_set_flags_and_status(sv, variant):
     w = make_random(6, 3, 3000, seed=6)
     assert sv.sv_get_device_status() == 0
     w.tokens[1, 0] = 3000
     w.target[2, 1, 17] = float("nan")
     w.draft[3, 2, 5] = float("inf")
     w.target[4, 0, :] = float("-inf")
-    got = gpu_run(w)
+    got = gpu_run(w, variant=variant)
     compare(w, got, oracle_on(w))
     assert got["flags"][1] & sv.SV_FLAG_BAD_TOKEN
     assert got["flags"][2] & sv.SV_FLAG_NONFINITE
@@ -97,12 +104,13 @@ def test_invalid_device_inputs_set_flags_and_status(sv):
     assert sv.sv_get_device_status() == 0  # cleared by the read
 
 
-def test_bad_row_D_and_per_request_parameters(sv):
+@VARIANTS
+def test_bad_row_D_and_per_request_parameters(sv, variant):
     w = make_random(6, 3, 3000, seed=7)
     w.row_D = torch.tensor([3, 4, -1, 2, 3, 3], dtype=torch.int32, device="cuda")
     w.temperature_per_req = torch.tensor([1.0, 1.0, 1.0, 0.0, 0.5, 1.0], device="cuda")
     w.mode_per_req = torch.tensor([0, 0, 0, 0, 1, 7], dtype=torch.int8, device="cuda")
-    got = gpu_run(w)
+    got = gpu_run(w, variant=variant)
     compare(w, got, oracle_on(w))
     assert got["flags"][1] & sv.SV_FLAG_BAD_ROW_D
     assert got["flags"][2] & sv.SV_FLAG_BAD_ROW_D
@@ -162,8 +170,9 @@ def test_explicit_workspace_and_stream(sv):
         sv.verify_workload(w, workspace=small)
 
 
+@VARIANTS
 @pytest.mark.parametrize("mode", [0, 2], ids=["plain", "saguaro"])
-def test_emitted_marginals_equal_target_1e6_requests(sv, mode):
+def test_emitted_marginals_equal_target_1e6_requests(sv, mode, variant):
     """V=8, D=2: 10^6 requests in one call (independent Philox streams): the
     emitted tokens follow p within 3 sigma per cell, as the oracle's do."""
     from svtest_util import sample_categorical, softmax
@@ -181,7 +190,7 @@ def test_emitted_marginals_equal_target_1e6_requests(sv, mode):
     tok = np.stack([sample_categorical(rng, qd[d], N) for d in range(D)], axis=1)
     T = torch.from_numpy(np.ascontiguousarray(np.broadcast_to(zt, (N, D + 1, V)))).cuda()
     Q = torch.from_numpy(np.ascontiguousarray(np.broadcast_to(zq, (N, D, V)))).cuda()
-    out = sv.verify(T, Q, torch.from_numpy(tok).cuda(), mode=mode, seed=31)
+    out = sv.verify(T, Q, torch.from_numpy(tok).cuda(), mode=mode, seed=31, variant=variant)
     torch.cuda.synchronize()
     AL = out["accept_len"].cpu().numpy()
     toks = out["tokens"].cpu().numpy()

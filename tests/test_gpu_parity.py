@@ -16,30 +16,36 @@ from gpu_util import compare, gpu_run, oracle_on
 
 pytestmark = pytest.mark.gpu
 
+VARIANTS = pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED],
+                                   ids=["split", "fused"])
 
+
+@VARIANTS
 @pytest.mark.parametrize("mode", [0, 1, 2], ids=["stochastic", "greedy", "saguaro"])
-def test_tiny_workload(sv, mode):
+def test_tiny_workload(sv, mode, variant):
     w = wl.make("tiny", "cuda", mode=mode)
     for seed in range(20):
-        got = gpu_run(w, seed=seed)
+        got = gpu_run(w, seed=seed, variant=variant)
         s = compare(w, got, oracle_on(w, seed=seed))
         assert s["checked"] + s["exempt"] == 1
 
 
+@VARIANTS
 @pytest.mark.parametrize("name", sorted(wl.CONFIGS))
 @pytest.mark.parametrize("V", [40000 + 13, 16384 * 2 + 7])
-def test_reduced_workloads(sv, name, V):
+def test_reduced_workloads(sv, name, V, variant):
     B = {"tiny": 3, "b32": 32, "b256": 24, "ragged": 24, "saguaro": 24}[name]
     w = wl.make(name, "cuda", B=B, V=V)
-    s = compare(w, gpu_run(w), oracle_on(w))
+    s = compare(w, gpu_run(w, variant=variant), oracle_on(w))
     assert s["checked"] >= B - 1
 
 
+@VARIANTS
 @pytest.mark.parametrize("name,sample", [("b32", None), ("b256", 24), ("ragged", None),
                                           ("saguaro", 24)])
-def test_full_size_workloads(sv, name, sample):
+def test_full_size_workloads(sv, name, sample, variant):
     w = wl.make(name, "cuda")
-    got = gpu_run(w)
+    got = gpu_run(w, variant=variant)
     reqs = None
     if sample:
         rng = np.random.default_rng(5)
@@ -50,23 +56,28 @@ def test_full_size_workloads(sv, name, sample):
     print(name, s)
 
 
+@VARIANTS
 @pytest.mark.parametrize("name", ["b32", "b256", "ragged", "saguaro"])
-def test_near_tie_rate_below_1e4_of_rows(sv, name):
+def test_near_tie_rate_below_1e4_of_rows(sv, name, variant):
     w = wl.make(name, "cuda")
     flagged = rows = 0
     for seed in range(8):
-        got = gpu_run(w, seed=seed)
+        got = gpu_run(w, seed=seed, variant=variant)
         flagged += int(np.count_nonzero(got["flags"] & sv.SV_FLAG_NEAR_TIE))
         rows += w.verified_rows()
     assert flagged <= max(1, 1e-4 * rows), (flagged, rows)
 
 
-def test_full_size_is_deterministic(sv):
+def test_full_size_is_deterministic_and_variants_agree(sv):
     w = wl.make("b256", "cuda")
-    a = gpu_run(w, seed=3)
-    b = gpu_run(w, seed=3)
+    a = gpu_run(w, seed=3, variant=sv.SV_VARIANT_SPLIT)
+    b = gpu_run(w, seed=3, variant=sv.SV_VARIANT_SPLIT)
+    c = gpu_run(w, seed=3, variant=sv.SV_VARIANT_FUSED)
+    d = gpu_run(w, seed=3, variant=sv.SV_VARIANT_FUSED)
     for k in a:
         assert np.array_equal(a[k], b[k], equal_nan=True), k
+        assert np.array_equal(a[k], c[k], equal_nan=True), k
+        assert np.array_equal(c[k], d[k], equal_nan=True), k
 
 
 def test_accept_length_mean_is_plausible(sv):
