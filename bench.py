@@ -213,6 +213,7 @@ def run_ours(args):
 
     import speculative_decoding_verification_lse_b200 as sv
     from speculative_decoding_verification_lse_b200 import workloads
+    from speculative_decoding_verification_lse_b200.sharding import max_over_ranks
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -272,12 +273,8 @@ def run_ours(args):
     clocks.active = False
     barrier()
     clocks.stop()
-    ms = t_start.elapsed_time(t_stop)
+    ms = max_over_ranks(t_start.elapsed_time(t_stop), dev)
     k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
     ms_per_step = ms / args.steps
     rows_total = w.verified_rows() * args.steps * world
     value = rows_total / (ms / 1e3)
@@ -314,11 +311,7 @@ def run_ours(args):
             e2e_step(1 + i)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
         h2d = h_t.numel() * h_t.element_size() + h_q.numel() * h_q.element_size() + h_x.numel() * 4
         d2h = o_t.numel() * 4 + o_a.numel() * 4
         e2e = {"value": w.verified_rows() * args.e2e_steps * world / (ems / 1e3), "unit": "rows/s",

@@ -45,4 +45,65 @@ __device__ __forceinline__ uint4 race_words(uint64_t seed, uint32_t g, uint32_t 
   return philox4x32_10(make_uint4(i, g, 1u, 0u), (uint32_t)seed, (uint32_t)(seed >> 32));
 }
 
+// The ten round keys of one seed (warp-uniform; computed once per work item).
+struct PhiloxKey {
+  uint32_t k0[10], k1[10];
+};
+
+__device__ __forceinline__ PhiloxKey philox_key(uint64_t seed) {
+  PhiloxKey K;
+  uint32_t a = (uint32_t)seed, b = (uint32_t)(seed >> 32);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    K.k0[r] = a;
+    K.k1[r] = b;
+    a += kWeylA;
+    b += kWeylB;
+  }
+  return K;
+}
+
+__device__ __forceinline__ void philox_round(uint4& c, uint32_t k0, uint32_t k1) {
+  const unsigned long long pa = (unsigned long long)kPhiloxMulA * c.x;
+  const unsigned long long pb = (unsigned long long)kPhiloxMulB * c.z;
+  c = make_uint4((uint32_t)(pb >> 32) ^ c.y ^ k0, (uint32_t)pb, (uint32_t)(pa >> 32) ^ c.w ^ k1,
+                 (uint32_t)pa);
+}
+
+// The race words of counter (i, g, 1, 0) for many i and one request g.  Words 2
+// and 3 of the counter are constants, so round 1 needs one per-thread product
+// instead of two, and so does round 2 (its first product is the same for every
+// i); the rest of the rounds are the published ones.
+struct RaceStream {
+  PhiloxKey K;
+  uint32_t x1;    // round-1 word 0: hi(B*1) ^ g ^ k0[0] = g ^ k0[0]
+  uint32_t y2c;   // round-2 word 0 term: lo(B*1) ^ k0[1] = B ^ k0[1]
+  uint32_t z2c;   // round-2 word 2 term: hi(A*x1) ^ k1[1]
+  uint32_t w2;    // round-2 word 3: lo(A*x1)
+};
+
+__device__ __forceinline__ RaceStream race_stream(uint64_t seed, uint32_t g) {
+  RaceStream R;
+  R.K = philox_key(seed);
+  R.x1 = g ^ R.K.k0[0];
+  R.y2c = kPhiloxMulB ^ R.K.k0[1];
+  const unsigned long long pa = (unsigned long long)kPhiloxMulA * R.x1;
+  R.z2c = (uint32_t)(pa >> 32) ^ R.K.k1[1];
+  R.w2 = (uint32_t)pa;
+  return R;
+}
+
+__device__ __forceinline__ uint4 race_words_fast(const RaceStream& R, uint32_t i) {
+  // round 1 on (i, g, 1, 0)
+  const unsigned long long pa = (unsigned long long)kPhiloxMulA * i;
+  const uint32_t z1 = (uint32_t)(pa >> 32) ^ R.K.k1[0];
+  const uint32_t w1 = (uint32_t)pa;
+  // round 2 on (x1, lo(B), z1, w1)
+  const unsigned long long pb = (unsigned long long)kPhiloxMulB * z1;
+  uint4 c = make_uint4((uint32_t)(pb >> 32) ^ R.y2c, (uint32_t)pb, w1 ^ R.z2c, R.w2);
+#pragma unroll
+  for (int r = 2; r < 10; ++r) philox_round(c, R.K.k0[r], R.K.k1[r]);
+  return c;
+}
+
 }  // namespace sv

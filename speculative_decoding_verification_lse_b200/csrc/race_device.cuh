@@ -15,7 +15,8 @@
 // few tokens that can win.  One warp handles an 8 KiB segment of the row:
 //   A. every lane computes, for each of its tokens, a single-precision UPPER
 //      BOUND of the key in log2 units (ex2/lg2 based, with explicit slack for
-//      every rounding and approximation error) and keeps its two largest;
+//      every rounding and approximation error; race_bounds) and keeps its two
+//      largest;
 //   B. each lane evaluates the exact key of its best token; S1 = warp maximum;
 //   C. a lane whose second bound reaches S1 (less a margin that also covers
 //      the 1e-6 near-tie band) evaluates that token too, and if its second
@@ -80,20 +81,18 @@ __device__ __forceinline__ Best warp_combine(Best v) {
   return v;
 }
 
-// log2 of E = -ln(1 - W), W = (o + 1/2) 2^-32, within 2^-12 relative in E.
-__device__ __forceinline__ float approx_log2_E(uint32_t o) {
-  // W < 2^-10: E = W + W^2/2 (the rest of the series is below 2^-20 relative)
-  const float fa = __uint_as_float(0x4B000000u | (o & 0x7FFFFFu)) - 8388608.0f;
-  const float Ws = (fa + 0.5f) * 0x1p-32f;
-  const float Es = fmaf(0.5f * Ws, Ws, Ws);
-  // otherwise E = -ln(U), U = 1 - W: exactly (~o + 1/2) 2^-32 when ~o < 2^23,
-  // else 1 - (o >> 9) 2^-23 (absolute error < 2^-23, U >= 2^-9 there)
-  const uint32_t no = ~o;
-  const float fc = __uint_as_float(0x4B000000u | (no & 0x7FFFFFu)) - 8388608.0f;
+// A lower bound of E = -ln(1 - W), W = (o + 1/2) 2^-32, within 2^-12 of it.
+//   W < 2^-10 (o < 2^22): E >= W, and W is exact from the low 22 bits of o.
+//   otherwise: U = 1 - W <= Uup = 1 - (o >> 9) 2^-23 (exact in single precision),
+//   so E >= -ln Uup >= ln2 (-lg2(Uup) - 2^-16) (lg2's error, taken as at most
+//   2^-22 (1 + |result|), is below 2^-16 for Uup in [2^-23, 1 - 2^-10]).
+__device__ __forceinline__ float E_lower(uint32_t o) {
+  const float fa = __uint_as_float(0x4B000000u | (o & 0x3FFFFFu)) - 8388608.0f;
+  const float Ws = fmaf(fa, 0x1p-32f, 0x1p-33f);
   const float fb = __uint_as_float(0x4B000000u | (o >> 9)) - 8388608.0f;
-  const float U = no < 0x800000u ? (fc + 0.5f) * 0x1p-32f : fmaf(-fb, 0x1p-23f, 1.0f);
-  const float El = -0.693147180559945f * lg2_approx(U);
-  return lg2_approx(o < 0x400000u ? Es : El);
+  const float Uup = fmaf(fb, -0x1p-23f, 1.0f);
+  const float El = fmaf(lg2_approx(Uup), -0.693147180559945f, -0.693147180559945f * 0x1p-16f);
+  return o < 0x400000u ? Ws : El;
 }
 
 // The exact key ln r(x) - ln E_x in double precision, the plain definition's
@@ -140,20 +139,25 @@ __device__ __forceinline__ double exact_key_of(const VerifyArgs& a, const RaceDe
 }
 
 // Upper bounds of the keys (log2 units) of one lane's tokens in segment `seg`;
-// calls visit(bound, x) for each.
+// calls visit(bound, x) for each.  Every rounding and approximation error is
+// covered by explicit slack:
+//   l2p = z*k2 - l2_t is within (|z| k2 + |l2_t|) 2^-22 of log2 p(x);
+//   log2 E >= lg2(E_lower) - 2^-16;
+//   residual, x outside K: d = log2 q'(x) - log2 p(x) >= dlo, and
+//     log2(1 - 2^d) <= lg2(1 - ex2(dlo)(1 - 2^-21)) + 2^-16;
+//   residual, x possibly in K (draft logit >= the smallest logit of K): r <= p.
 template <int DT, typename Visit>
 __device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc& rd,
-                                            const char* trow, const char* qrow, bool residual,
-                                            int seg, Visit&& visit) {
+                                            const RaceStream& R, const char* trow,
+                                            const char* qrow, bool residual, int seg,
+                                            Visit&& visit) {
   constexpr int VEC = DT == kF32 ? 4 : 8;
   const int lane = threadIdx.x & 31;
-  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
   const float k2 = rd.k2;
-  const float l2t = rd.l2_t, l2q = rd.l2_q;
-  // slack for the rounding of z*k2 - l2: relative 2^-21 of each term, plus 2^-22
-  const float ks = k2 * 0x1p-21f;
-  const float st0 = fabsf(l2t) * 0x1p-21f + 0x1p-22f;
-  const float sq0 = fabsf(l2q) * 0x1p-21f + 0x1p-22f;
+  const float l2t = rd.l2_t, l2q = rd.l2_q, kmin = rd.kmin;
+  const float ks = k2 * 0x1p-22f;
+  const float st = fmaf(fabsf(l2t), 0x1p-22f, 0x1p-16f);  // + the log2 E slack
+  const float sq = fabsf(l2q) * 0x1p-22f;
   const int nfull = a.V / VEC;
   const bool aligned =
       ((uintptr_t)trow & 15u) == 0 && (!residual || ((uintptr_t)qrow & 15u) == 0);
@@ -172,23 +176,22 @@ __device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc&
 #pragma unroll
     for (int h = 0; h < VEC / 4; ++h) {
       const uint32_t base = (uint32_t)(v * VEC + 4 * h);
-      const uint4 o4 = philox4x32_10(make_uint4(base >> 2, rd.g, 1u, 0u), k0, k1);
+      const uint4 o4 = race_words_fast(R, base >> 2);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int x = (int)base + e;
         const float zt = elem<DT>(wt, 4 * h + e);
         const uint32_t o = e == 0 ? o4.x : e == 1 ? o4.y : e == 2 ? o4.z : o4.w;
-        // ln p(x) - ln E_x, upper bound in log2 units
-        const float sp = fmaf(fabsf(zt), ks, st0);
-        const float l2p = fmaf(zt, k2, -l2t);
-        float bound = (l2p + sp) - (approx_log2_E(o) - 0x1p-11f);
+        // log2 p(x) + slack, an upper bound (the log2 E slack is folded into st)
+        const float l2pu = fmaf(zt, k2, -l2t) + fmaf(fabsf(zt), ks, st);
+        float bound = l2pu - lg2_approx(E_lower(o));
         if (residual) {
-          // r = p (1 - q/p): add the upper bound of log2(1 - 2^d), d = l2q - l2p
+          // r = p (1 - q'/p): add an upper bound of log2(1 - 2^d), d = log2 q' - log2 p
           const float zq = elem<DT>(wq, 4 * h + e);
-          const float sq = fmaf(fabsf(zq), ks, sq0);
-          const float dlo = (fmaf(zq, k2, -l2q) - sq) - (l2p + sp);
-          const float t = fmaf(-ex2_approx(dlo), 1.0f - 0x1p-20f, 1.0f);
-          bound = (dlo < 0.0f) ? bound + (lg2_approx(t) + 0x1p-20f) : -INFINITY;
+          const float dlo = (fmaf(zq, k2, -l2q) - fmaf(fabsf(zq), ks, sq)) - l2pu;
+          const float t = fmaf(-ex2_approx(dlo), 1.0f - 0x1p-21f, 1.0f);
+          const float res = (dlo < 0.0f) ? bound + (lg2_approx(t) + 0x1p-16f) : -INFINITY;
+          bound = zq >= kmin ? bound : res;  // a token of K keeps the bound r <= p
         }
         if (x < a.V && zt > -INFINITY) visit(bound, x);
       }
@@ -202,9 +205,10 @@ __device__ __forceinline__ Best race_segment(const VerifyArgs& a, const RaceDesc
                                              const char* trow, const char* qrow,
                                              bool residual, int seg) {
   // A. the two largest bounds of each lane
+  const RaceStream R = race_stream(a.seed, rd.g);
   float u1 = -INFINITY, u2 = -INFINITY;
   int i1 = -1, i2 = -1;
-  race_bounds<DT>(a, rd, trow, qrow, residual, seg, [&](float bound, int x) {
+  race_bounds<DT>(a, rd, R, trow, qrow, residual, seg, [&](float bound, int x) {
     if (bound > u2) {
       if (bound > u1) {
         u2 = u1;
@@ -229,7 +233,7 @@ __device__ __forceinline__ Best race_segment(const VerifyArgs& a, const RaceDesc
     offer(B, exact_key_of(a, rd, trow, qrow, residual, i2), i2);
     // the third bound may have reached thr as well: visit them all
     const int j1 = i1, j2 = i2;
-    race_bounds<DT>(a, rd, trow, qrow, residual, seg, [&](float bound, int x) {
+    race_bounds<DT>(a, rd, R, trow, qrow, residual, seg, [&](float bound, int x) {
       if (bound >= thr && x != j1 && x != j2)
         offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
     });

@@ -241,6 +241,7 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
     rd.k2 = log2e_over_T(rp.T);
     rd.l2_t = (float)(rows[n].lse * 1.4426950408889634);
     rd.l2_q = 0.0f;
+    rd.kmin = INFINITY;
     rd.lse_q = 0.0;
     rd.ln_c = log(c);
     rd.ln_Z = 0.0;
@@ -253,7 +254,8 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
         rd.ln_Z = rq.lnZ;
         rd.ntop = rq.ntop;
         for (int i = 0; i < rq.ntop; ++i) rd.top[i] = rq.top[i];
-        shift = rq.lse - rd.ln_c + rq.lnZ;
+        shift = rq.lse + rq.lnZ;
+        if (rq.ntop > 0) rd.kmin = rq.topv[rq.ntop - 1];
       }
       rd.l2_q = (float)(shift * 1.4426950408889634);
     }

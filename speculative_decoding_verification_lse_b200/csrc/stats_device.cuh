@@ -13,9 +13,9 @@
 //
 // Each lane issues its sixteen 16-byte loads at once (8 KiB in flight per
 // warp), takes its maximum on packed bf16 pairs, the warp agrees on the segment
-// maximum with five shuffles, and then every element costs one FFMA, one ex2
-// and one FADD relative to that maximum -- no per-element rescaling, no
-// barrier, no shared memory.
+// maximum with five shuffles, and then every pair of elements costs one packed
+// FFMA, two ex2 and one packed FADD relative to that maximum -- no per-element
+// rescaling, no barrier, no shared memory.
 #pragma once
 #include "sv_common.cuh"
 
@@ -133,21 +133,28 @@ __device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* r
   const float m_w = warp_max(m_t);
   const uint32_t bad_w = __any_sync(0xFFFFFFFFu, bad) ? 1u : 0u;
 
-  // ---- sum of 2^(z*k2 - mk): one FFMA, one ex2 and one FADD per element
+  // ---- sum of 2^(z*k2 - mk): per pair of elements one packed FFMA, two ex2 and
+  // one packed FADD (fixed accumulation order: four float2 accumulators)
   float S_w = 0.0f;
   if (LSE) {
     float S_t = 0.0f;
     if (m_w > -INFINITY) {
       const float mk = m_w * k2;
-      float acc[8];
+      const float2 kk = make_float2(k2, k2), nm = make_float2(-mk, -mk);
+      float2 acc[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+      for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int j = 0; j < kLaneVecs; ++j)
 #pragma unroll
-        for (int e = 0; e < VEC; ++e)
-          acc[(j * VEC + e) & 7] += ex2_approx(fmaf(elem<DT>(raw[j], e), k2, -mk));
-      S_t = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        for (int e = 0; e < VEC; e += 2) {
+          const float2 t = __ffma2_rn(make_float2(elem<DT>(raw[j], e), elem<DT>(raw[j], e + 1)), kk, nm);
+          const int q = ((j * VEC + e) >> 1) & 3;
+          acc[q] = __fadd2_rn(acc[q], make_float2(ex2_approx(t.x), ex2_approx(t.y)));
+        }
+      const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 s = __fadd2_rn(s01, s23);
+      S_t = s.x + s.y;
     }
     S_w = warp_sum(S_t);
   }
@@ -245,10 +252,11 @@ __device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot,
   PartStat* out = a.pstat + ((size_t)b * a.slots + slot) * a.nseg + seg;
   const float k2 = rp.mode == kGreedy ? 0.0f : log2e_over_T(rp.T);
   if (is_target) {
+    // the argmax is only used by greedy requests
     if (rp.mode == kGreedy)
       stats_segment<DT, false, true, false>(a, row, seg, k2, 0, out, nullptr);
     else
-      stats_segment<DT, true, true, false>(a, row, seg, k2, 0, out, nullptr);
+      stats_segment<DT, true, false, false>(a, row, seg, k2, 0, out, nullptr);
   } else if (rp.mode == kSaguaro) {
     TopPart* tout = a.tpart + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * a.nseg + seg;
     stats_segment<DT, true, false, true>(a, row, seg, k2, a.saguaro_k, out, tout);

@@ -74,8 +74,10 @@ struct __align__(16) RaceDesc {
   double ln_Z;       // saguaro: ln Z of draft row n
   float k2;          // fl(log2(e) / T)
   float l2_t;        // fl(lse_t * log2(e))
-  float l2_q;        // fl((lse_q - ln c + ln Z) * log2(e)) (saguaro), fl(lse_q * log2(e)) else:
-                     // z*k2 - l2_q is then a lower bound of log2 q'(x) for every x
+  float l2_q;        // fl((lse_q + ln Z) * log2(e)): z*k2 - l2_q approximates log2 q'(x)
+                     // for every x outside K (ln Z = 0 unless saguaro)
+  float kmin;        // saguaro: the smallest logit in K (a token with a smaller draft
+                     // logit is not in K); +inf otherwise
   int ntop;          // saguaro: size of K (0 otherwise)
   int top[kMaxTopK]; // saguaro: K of draft row n
 };
