@@ -165,8 +165,8 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     return fail(SV_ERR_UNSUPPORTED, "V larger than %d is not supported for this dtype",
                 kMaxSegs * kSegVecs * vec_elems(dtype));
   const long long slots = 2LL * D_max + 1;
-  if ((long long)B * slots * nseg > 0x7FFFFFFFLL)
-    return fail(SV_ERR_UNSUPPORTED, "B * (2*D_max+1) * segments exceeds 2^31");
+  if ((long long)B * (slots + 1) * nseg > 0x7FFFFFFFLL)
+    return fail(SV_ERR_UNSUPPORTED, "B * (2*D_max+2) * segments exceeds 2^31");
   const bool saguaro_possible = mode == SV_SAGUARO || prm.mode_per_req != nullptr;
 
   int dev = 0;
@@ -215,10 +215,11 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.rdesc = (RaceDesc*)((char*)ws + L.rdesc);
   a.rpart = (RacePart*)((char*)ws + L.rpart);
   a.rcount = (unsigned int*)((char*)ws + L.rcount);
+  a.rowres = (RowRes*)((char*)ws + L.rowres);
   a.fstate = (FusedState*)((char*)ws + L.fstate);
-  a.done = (unsigned int*)((char*)ws + L.done);
+  a.row_done = (unsigned int*)((char*)ws + L.row_done);
+  a.req_rows = (unsigned int*)((char*)ws + L.req_rows);
   a.ready = (unsigned int*)((char*)ws + L.ready);
-  a.rclaim = (unsigned int*)((char*)ws + L.rclaim);
   a.seed = seed;
   a.B = B;
   a.D_max = D_max;

@@ -1,20 +1,23 @@
 // fused_verify.cu -- the whole verification step in one launch.
 //
-// Every warp of a persistent grid is an independent worker that repeats:
-//   1. claim a published race segment, if any, and run it (race_device.cuh);
-//   2. otherwise take the next statistics ticket -- (request, row, segment) in
-//      request-major order -- and compute that segment's statistics
-//      (stats_device.cuh);
-//   3. the warp that finishes the last segment of a request runs that
-//      request's accept scan (scan_device.cuh) and publishes its race.
-// Race work is claimed through a cursor over requests: a warp claims segments
-// of the request under the cursor only when that request is published, and
-// moves the cursor on once every segment is claimed.  Nothing ever waits for
-// another warp: a warp that finds no published race work takes a ticket, and
-// one that finds no ticket left exits.  Whoever publishes the request under
-// the cursor carries on with every published request behind it, so no race is
-// left unclaimed.  The sampled rows of a request were streamed moments earlier,
-// so the race mostly reads them again from L2, while other warps keep HBM busy.
+// Every warp of a persistent grid takes tickets from one ordered ticket space
+// and does what its ticket names:
+//   * a statistics ticket: one 8 KiB segment of one row (stats_device.cuh); the
+//     warp that finishes a row's last segment merges that row, and the warp
+//     that merges a request's last row runs that request's accept scan
+//     (scan_device.cuh) and publishes it;
+//   * a race ticket: one segment of one request's race (race_device.cuh).
+// The ticket space lists, request after request, the statistics segments of
+// request r followed by the race segments of request r - L, with a lag of L
+// requests (about 64 MiB of logits) so that a race ticket is normally taken
+// after its request has been published, while that request's sampled rows are
+// still in L2.  A warp holding a race ticket whose request is not yet published
+// waits for it, polling with a sleep and a bounded number of polls (an expired
+// wait sets SV_STATUS_TIMEOUT and leaves that token at -1).  The wait always
+// ends: the request's statistics tickets all come earlier in the order, so they
+// were taken by warps that are running, and statistics work never waits.  For
+// the same reason a warp prefetches its next ticket only while it works on a
+// statistics segment, never while it waits.
 //
 // All counters live in a workspace region cleared before the launch.
 #include "race_device.cuh"
@@ -28,6 +31,8 @@ namespace {
 constexpr unsigned kReadyNone = 0u;   // request not finished yet
 constexpr unsigned kReadyRace = 1u;   // race published
 constexpr unsigned kReadyDone = 2u;   // finished, nothing to race (greedy or error)
+constexpr unsigned kLagTickets = 8192;  // statistics tickets (64 MiB) between a request and its race
+constexpr int kWaitPolls = 1 << 20;     // with a 128 ns sleep each: well over 0.1 s
 
 __device__ __forceinline__ unsigned load_acquire(const unsigned* p) {
   unsigned v;
@@ -39,29 +44,60 @@ __device__ __forceinline__ void store_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Number of statistics items request b completes with.
-__device__ __forceinline__ unsigned items_needed(const VerifyArgs& a, const ReqParams& rp) {
-  const int rows = (rp.Db + 1) + (rp.mode == kGreedy ? 0 : rp.Db);
-  return (unsigned)rows * (unsigned)a.nseg;
-}
-
-// Lane 0: claim one published race segment; returns the request (or -1).
-__device__ int claim_race(const VerifyArgs& a, int* seg) {
-  for (int guard = 0; guard < 4 * a.B + 8; ++guard) {  // each pass moves the cursor or returns
-    const unsigned r = load_acquire(&a.fstate->cursor);
-    if (r >= (unsigned)a.B) return -1;
-    const unsigned st = load_acquire(&a.ready[r]);
-    if (st == kReadyNone) return -1;  // not published yet: its publisher will run it
-    if (st == kReadyRace) {
-      const unsigned s = atomicAdd(&a.rclaim[r], 1u);
-      if (s < (unsigned)a.nseg) {
-        *seg = (int)s;
-        return (int)r;
-      }
-    }
-    atomicCAS(&a.fstate->cursor, r, r + 1);  // fully claimed (or nothing to race): move on
+// The ordered ticket space.
+struct Tickets {
+  unsigned S, R, L, B;      // stats and race tickets per request, lag, requests
+  unsigned p1, p2, total;   // ends of the three phases
+  __device__ __forceinline__ void init(const VerifyArgs& a) {
+    S = (unsigned)a.slots * (unsigned)a.nseg;
+    R = (unsigned)a.nseg;
+    B = (unsigned)a.B;
+    L = (kLagTickets + S - 1) / S;
+    if (L < 1) L = 1;
+    if (L > B) L = B;
+    p1 = L * S;                      // requests [0, L): statistics only
+    p2 = p1 + (B - L) * (S + R);     // requests [L, B): statistics of r, race of r - L
+    total = p2 + L * R;              // the races of the last L requests
   }
-  return -1;
+  // false: race ticket (b, seg); true: statistics ticket (b, slot, seg)
+  __device__ __forceinline__ bool decode(const VerifyArgs& a, unsigned t, int& b, int& slot,
+                                         int& seg) const {
+    unsigned r, off;
+    bool stats;
+    if (t < p1) {
+      r = t / S;
+      off = t % S;
+      stats = true;
+    } else if (t < p2) {
+      const unsigned u = t - p1;
+      r = L + u / (S + R);
+      off = u % (S + R);
+      stats = off < S;
+      if (!stats) {
+        r -= L;
+        off -= S;
+      }
+    } else {
+      const unsigned u = t - p2;
+      r = B - L + u / R;
+      off = u % R;
+      stats = false;
+    }
+    b = (int)r;
+    if (stats) {
+      slot = (int)(off / (unsigned)a.nseg);
+      seg = (int)(off % (unsigned)a.nseg);
+    } else {
+      slot = 0;
+      seg = (int)off;
+    }
+    return stats;
+  }
+};
+
+// Number of rows request b reads.
+__device__ __forceinline__ unsigned rows_needed(const ReqParams& rp) {
+  return (unsigned)((rp.Db + 1) + (rp.mode == kGreedy ? 0 : rp.Db));
 }
 
 // The scan of request b by this warp, then its publication.
@@ -75,55 +111,74 @@ __device__ __forceinline__ void finish_request(const VerifyArgs& a, int b, RowRe
   __syncwarp();
 }
 
+// Lane 0: the publication state of request b, waiting (bounded) until it is set.
+__device__ unsigned wait_ready(const VerifyArgs& a, int b) {
+  unsigned st = load_acquire(&a.ready[b]);
+  for (int i = 0; st == kReadyNone && i < kWaitPolls; ++i) {
+    __nanosleep(128);
+    st = load_acquire(&a.ready[b]);
+  }
+  if (st == kReadyNone) atomicOr(a.status, kStatusTimeout);
+  return st;
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads) fused_kernel(VerifyArgs a) {
   extern __shared__ __align__(16) unsigned char s_dyn[];
   __shared__ RaceDesc s_rd[kWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   RowRes* rows = reinterpret_cast<RowRes*>(s_dyn) + (size_t)warp * a.slots;
-  const unsigned per_req = (unsigned)a.slots * (unsigned)a.nseg;
-  const unsigned total = (unsigned)a.B * per_req;
+  Tickets T;
+  T.init(a);
 
-  for (;;) {
-    // 1. published race work first
-    int rb = -1, rs = 0;
-    if (lane == 0) rb = claim_race(a, &rs);
-    rb = __shfl_sync(0xFFFFFFFFu, rb, 0);
-    if (rb >= 0) {
-      rs = __shfl_sync(0xFFFFFFFFu, rs, 0);
-      __threadfence();
-      load_race_desc(a.rdesc + rb, &s_rd[warp]);
-      race_item<DT>(a, rb, rs, s_rd[warp]);
-      continue;
+  unsigned t = 0;
+  if (lane == 0) t = atomicAdd(&a.fstate->next_ticket, 1u);
+  t = __shfl_sync(0xFFFFFFFFu, t, 0);
+  while (t < T.total) {
+    int b, slot, seg;
+    if (T.decode(a, t, b, slot, seg)) {
+      // a statistics segment: fetch the next ticket now, use it afterwards
+      unsigned tn = 0;
+      if (lane == 0) tn = atomicAdd(&a.fstate->next_ticket, 1u);
+      const ReqParams rp = load_req(a, b);
+      if (rp.err) {
+        // invalid request parameters: the request's first ticket reports them
+        if (slot == 0 && seg == 0) finish_request(a, b, rows);
+      } else if (row_needed(a, slot, rp)) {
+        stats_item<DT>(a, b, slot, seg, rp);
+        // the warp finishing the row's last segment merges the row ...
+        unsigned prev = 0;
+        if (lane == 0) {
+          __threadfence();
+          prev = atomicAdd(&a.row_done[(size_t)b * a.slots + slot], 1u);
+        }
+        prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+        if (prev + 1u == (unsigned)a.nseg) {
+          __threadfence();
+          merge_row_global(a, b, slot, rp);
+          // ... and the warp merging the request's last row runs the scan
+          if (lane == 0) {
+            __threadfence();
+            prev = atomicAdd(&a.req_rows[b], 1u);
+          }
+          prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+          if (prev + 1u == rows_needed(rp)) finish_request(a, b, rows);
+        }
+      }
+      t = __shfl_sync(0xFFFFFFFFu, tn, 0);
+    } else {
+      // a race segment: its request must have been published
+      unsigned st = 0;
+      if (lane == 0) st = wait_ready(a, b);
+      st = __shfl_sync(0xFFFFFFFFu, st, 0);
+      if (st == kReadyRace) {
+        __threadfence();
+        load_race_desc(a.rdesc + b, &s_rd[warp]);
+        race_item<DT>(a, b, seg, s_rd[warp]);
+      }
+      if (lane == 0) t = atomicAdd(&a.fstate->next_ticket, 1u);
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
     }
-
-    // 2. the next statistics item
-    unsigned tk = 0;
-    if (lane == 0) tk = atomicAdd(&a.fstate->next_ticket, 1u);
-    tk = __shfl_sync(0xFFFFFFFFu, tk, 0);
-    if (tk >= total) break;
-    const int b = (int)(tk / per_req);
-    const unsigned rem = tk % per_req;
-    const int slot = (int)(rem / (unsigned)a.nseg);
-    const int seg = (int)(rem % (unsigned)a.nseg);
-    const ReqParams rp = load_req(a, b);
-
-    if (rp.err) {
-      // invalid request parameters: its first ticket reports them
-      if (slot == 0 && seg == 0) finish_request(a, b, rows);
-      continue;
-    }
-    if (!row_needed(a, slot, rp)) continue;
-    stats_item<DT>(a, b, slot, seg, rp);
-
-    // 3. the warp finishing a request's last item runs its scan and publishes
-    unsigned prev = 0;
-    if (lane == 0) {
-      __threadfence();
-      prev = atomicAdd(&a.done[b], 1u);
-    }
-    prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-    if (prev + 1u == items_needed(a, rp)) finish_request(a, b, rows);
   }
 }
 

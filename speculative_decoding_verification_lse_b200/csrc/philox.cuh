@@ -45,6 +45,13 @@ __device__ __forceinline__ uint4 race_words(uint64_t seed, uint32_t g, uint32_t 
   return philox4x32_10(make_uint4(i, g, 1u, 0u), (uint32_t)seed, (uint32_t)(seed >> 32));
 }
 
+// Full 64-bit product of two 32-bit words.
+__device__ __forceinline__ unsigned long long mul_wide(uint32_t a, uint32_t b) {
+  unsigned long long r;
+  asm("mul.wide.u32 %0, %1, %2;" : "=l"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // The ten round keys of one seed (warp-uniform; computed once per work item).
 struct PhiloxKey {
   uint32_t k0[10], k1[10];
@@ -64,8 +71,8 @@ __device__ __forceinline__ PhiloxKey philox_key(uint64_t seed) {
 }
 
 __device__ __forceinline__ void philox_round(uint4& c, uint32_t k0, uint32_t k1) {
-  const unsigned long long pa = (unsigned long long)kPhiloxMulA * c.x;
-  const unsigned long long pb = (unsigned long long)kPhiloxMulB * c.z;
+  const unsigned long long pa = mul_wide(kPhiloxMulA, c.x);
+  const unsigned long long pb = mul_wide(kPhiloxMulB, c.z);
   c = make_uint4((uint32_t)(pb >> 32) ^ c.y ^ k0, (uint32_t)pb, (uint32_t)(pa >> 32) ^ c.w ^ k1,
                  (uint32_t)pa);
 }
@@ -95,11 +102,11 @@ __device__ __forceinline__ RaceStream race_stream(uint64_t seed, uint32_t g) {
 
 __device__ __forceinline__ uint4 race_words_fast(const RaceStream& R, uint32_t i) {
   // round 1 on (i, g, 1, 0)
-  const unsigned long long pa = (unsigned long long)kPhiloxMulA * i;
+  const unsigned long long pa = mul_wide(kPhiloxMulA, i);
   const uint32_t z1 = (uint32_t)(pa >> 32) ^ R.K.k1[0];
   const uint32_t w1 = (uint32_t)pa;
   // round 2 on (x1, lo(B), z1, w1)
-  const unsigned long long pb = (unsigned long long)kPhiloxMulB * z1;
+  const unsigned long long pb = mul_wide(kPhiloxMulB, z1);
   uint4 c = make_uint4((uint32_t)(pb >> 32) ^ R.y2c, (uint32_t)pb, w1 ^ R.z2c, R.w2);
 #pragma unroll
   for (int r = 2; r < 10; ++r) philox_round(c, R.K.k0[r], R.K.k1[r]);

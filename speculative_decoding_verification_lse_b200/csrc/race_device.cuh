@@ -81,18 +81,25 @@ __device__ __forceinline__ Best warp_combine(Best v) {
   return v;
 }
 
-// A lower bound of E = -ln(1 - W), W = (o + 1/2) 2^-32, within 2^-12 of it.
+// A lower bound of E = -ln(1 - W), W = (o + 1/2) 2^-32, within 2^-12 of it, for
+// two words at once.
 //   W < 2^-10 (o < 2^22): E >= W, and W is exact from the low 22 bits of o.
 //   otherwise: U = 1 - W <= Uup = 1 - (o >> 9) 2^-23 (exact in single precision),
 //   so E >= -ln Uup >= ln2 (-lg2(Uup) - 2^-16) (lg2's error, taken as at most
 //   2^-22 (1 + |result|), is below 2^-16 for Uup in [2^-23, 1 - 2^-10]).
-__device__ __forceinline__ float E_lower(uint32_t o) {
-  const float fa = __uint_as_float(0x4B000000u | (o & 0x3FFFFFu)) - 8388608.0f;
-  const float Ws = fmaf(fa, 0x1p-32f, 0x1p-33f);
-  const float fb = __uint_as_float(0x4B000000u | (o >> 9)) - 8388608.0f;
-  const float Uup = fmaf(fb, -0x1p-23f, 1.0f);
-  const float El = fmaf(lg2_approx(Uup), -0.693147180559945f, -0.693147180559945f * 0x1p-16f);
-  return o < 0x400000u ? Ws : El;
+__device__ __forceinline__ float2 E_lower2(uint32_t o0, uint32_t o1) {
+  const float2 fa = __fadd2_rn(make_float2(__uint_as_float(0x4B000000u | (o0 & 0x3FFFFFu)),
+                                           __uint_as_float(0x4B000000u | (o1 & 0x3FFFFFu))),
+                               make_float2(-8388608.0f, -8388608.0f));
+  const float2 Ws = __ffma2_rn(fa, make_float2(0x1p-32f, 0x1p-32f), make_float2(0x1p-33f, 0x1p-33f));
+  const float2 fb = __fadd2_rn(make_float2(__uint_as_float(0x4B000000u | (o0 >> 9)),
+                                           __uint_as_float(0x4B000000u | (o1 >> 9))),
+                               make_float2(-8388608.0f, -8388608.0f));
+  const float2 Uup = __ffma2_rn(fb, make_float2(-0x1p-23f, -0x1p-23f), make_float2(1.0f, 1.0f));
+  const float2 El = __ffma2_rn(make_float2(lg2_approx(Uup.x), lg2_approx(Uup.y)),
+                               make_float2(-0.693147180559945f, -0.693147180559945f),
+                               make_float2(-0.693147180559945f * 0x1p-16f, -0.693147180559945f * 0x1p-16f));
+  return make_float2(o0 < 0x400000u ? Ws.x : El.x, o1 < 0x400000u ? Ws.y : El.y);
 }
 
 // The exact key ln r(x) - ln E_x in double precision, the plain definition's
@@ -146,6 +153,7 @@ __device__ __forceinline__ double exact_key_of(const VerifyArgs& a, const RaceDe
 //   residual, x outside K: d = log2 q'(x) - log2 p(x) >= dlo, and
 //     log2(1 - 2^d) <= lg2(1 - ex2(dlo)(1 - 2^-21)) + 2^-16;
 //   residual, x possibly in K (draft logit >= the smallest logit of K): r <= p.
+// Pairs of tokens share packed fp32x2 arithmetic.
 template <int DT, typename Visit>
 __device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc& rd,
                                             const RaceStream& R, const char* trow,
@@ -155,9 +163,15 @@ __device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc&
   const int lane = threadIdx.x & 31;
   const float k2 = rd.k2;
   const float l2t = rd.l2_t, l2q = rd.l2_q, kmin = rd.kmin;
-  const float ks = k2 * 0x1p-22f;
-  const float st = fmaf(fabsf(l2t), 0x1p-22f, 0x1p-16f);  // + the log2 E slack
-  const float sq = fabsf(l2q) * 0x1p-22f;
+  const float2 kk = make_float2(k2, k2);
+  const float2 ks = make_float2(k2 * 0x1p-22f, k2 * 0x1p-22f);
+  const float2 nt = make_float2(-l2t, -l2t), nq = make_float2(-l2q, -l2q);
+  const float st1 = fmaf(fabsf(l2t), 0x1p-22f, 0x1p-16f);  // + the log2 E slack
+  const float2 st = make_float2(st1, st1);
+  const float sq1 = fabsf(l2q) * 0x1p-22f;
+  const float2 sq = make_float2(sq1, sq1);
+  const float2 shrink = make_float2(-(1.0f - 0x1p-21f), -(1.0f - 0x1p-21f));
+  const float2 one = make_float2(1.0f, 1.0f);
   const int nfull = a.V / VEC;
   const bool aligned =
       ((uintptr_t)trow & 15u) == 0 && (!residual || ((uintptr_t)qrow & 15u) == 0);
@@ -178,22 +192,31 @@ __device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc&
       const uint32_t base = (uint32_t)(v * VEC + 4 * h);
       const uint4 o4 = race_words_fast(R, base >> 2);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int x = (int)base + e;
-        const float zt = elem<DT>(wt, 4 * h + e);
-        const uint32_t o = e == 0 ? o4.x : e == 1 ? o4.y : e == 2 ? o4.z : o4.w;
+      for (int e = 0; e < 4; e += 2) {
+        const float2 zt = make_float2(elem<DT>(wt, 4 * h + e), elem<DT>(wt, 4 * h + e + 1));
+        const float2 El = e == 0 ? E_lower2(o4.x, o4.y) : E_lower2(o4.z, o4.w);
         // log2 p(x) + slack, an upper bound (the log2 E slack is folded into st)
-        const float l2pu = fmaf(zt, k2, -l2t) + fmaf(fabsf(zt), ks, st);
-        float bound = l2pu - lg2_approx(E_lower(o));
+        const float2 l2pu = __fadd2_rn(__ffma2_rn(zt, kk, nt),
+                                       __ffma2_rn(make_float2(fabsf(zt.x), fabsf(zt.y)), ks, st));
+        float2 bound = __fadd2_rn(l2pu, make_float2(-lg2_approx(El.x), -lg2_approx(El.y)));
         if (residual) {
           // r = p (1 - q'/p): add an upper bound of log2(1 - 2^d), d = log2 q' - log2 p
-          const float zq = elem<DT>(wq, 4 * h + e);
-          const float dlo = (fmaf(zq, k2, -l2q) - fmaf(fabsf(zq), ks, sq)) - l2pu;
-          const float t = fmaf(-ex2_approx(dlo), 1.0f - 0x1p-21f, 1.0f);
-          const float res = (dlo < 0.0f) ? bound + (lg2_approx(t) + 0x1p-16f) : -INFINITY;
-          bound = zq >= kmin ? bound : res;  // a token of K keeps the bound r <= p
+          const float2 zq = make_float2(elem<DT>(wq, 4 * h + e), elem<DT>(wq, 4 * h + e + 1));
+          const float2 dlo = __fadd2_rn(
+              __fadd2_rn(__ffma2_rn(zq, kk, nq),
+                         __fmul2_rn(__ffma2_rn(make_float2(fabsf(zq.x), fabsf(zq.y)), ks, sq),
+                                    make_float2(-1.0f, -1.0f))),
+              make_float2(-l2pu.x, -l2pu.y));
+          const float2 t = __ffma2_rn(make_float2(ex2_approx(dlo.x), ex2_approx(dlo.y)), shrink, one);
+          const float2 res = __fadd2_rn(bound, make_float2(lg2_approx(t.x) + 0x1p-16f,
+                                                           lg2_approx(t.y) + 0x1p-16f));
+          // a token of K keeps the bound r <= p; q' >= p excludes the token
+          bound.x = zq.x >= kmin ? bound.x : (dlo.x < 0.0f ? res.x : -INFINITY);
+          bound.y = zq.y >= kmin ? bound.y : (dlo.y < 0.0f ? res.y : -INFINITY);
         }
-        if (x < a.V && zt > -INFINITY) visit(bound, x);
+        const int x = (int)base + e;
+        if (x < a.V && zt.x > -INFINITY) visit(bound.x, x);
+        if (x + 1 < a.V && zt.y > -INFINITY) visit(bound.y, x + 1);
       }
     }
   }
@@ -209,17 +232,12 @@ __device__ __forceinline__ Best race_segment(const VerifyArgs& a, const RaceDesc
   float u1 = -INFINITY, u2 = -INFINITY;
   int i1 = -1, i2 = -1;
   race_bounds<DT>(a, rd, R, trow, qrow, residual, seg, [&](float bound, int x) {
-    if (bound > u2) {
-      if (bound > u1) {
-        u2 = u1;
-        i2 = i1;
-        u1 = bound;
-        i1 = x;
-      } else {
-        u2 = bound;
-        i2 = x;
-      }
-    }
+    // branch-free: ties keep the earlier (lower) index
+    const bool gt1 = bound > u1, gt2 = bound > u2;
+    u2 = gt1 ? u1 : (gt2 ? bound : u2);
+    i2 = gt1 ? i1 : (gt2 ? x : i2);
+    u1 = gt1 ? bound : u1;
+    i1 = gt1 ? x : i1;
   });
   // B. the exact key of each lane's best token
   Best B{-INFINITY, -INFINITY, -1};

@@ -26,16 +26,6 @@ namespace sv {
 
 constexpr double kLn2d = 0.69314718055994530942;
 
-struct RowRes {
-  double lse;   // natural-log LSE at T (stochastic rows)
-  double lnZ;   // saguaro draft rows: ln Z
-  int argmax;   // target rows
-  uint32_t bad;
-  int ntop;
-  int top[kMaxTopK];
-  float topv[kMaxTopK];
-};
-
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
@@ -111,9 +101,41 @@ __device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg
   r.bad = bad;
 }
 
-// The accept scan of request b by one full warp; rows: 2*D_max+1 entries of
-// shared memory.  Writes the outputs (slot n too for greedy), the flags, the
-// row LSEs and the race description; returns the race kind (same on all lanes).
+// Whether row `slot` of a request with parameters rp is read by the rule.
+__device__ __forceinline__ bool slot_needed(const VerifyArgs& a, int slot, const ReqParams& rp) {
+  if (rp.err) return false;
+  const bool is_t = slot <= a.D_max;
+  const int d = is_t ? slot : slot - a.D_max - 1;
+  return is_t ? d <= rp.Db : (d < rp.Db && rp.mode != kGreedy);
+}
+
+// Merge row `slot` of request b (one full warp) into a.rowres.
+__device__ inline void merge_row_global(const VerifyArgs& a, int b, int slot, const ReqParams& rp) {
+  const int Dm = a.D_max;
+  const bool greedy = rp.mode == kGreedy;
+  const bool is_t = slot <= Dm;
+  const int d = is_t ? slot : slot - Dm - 1;
+  const float k2 = greedy ? 0.0f : log2e_over_T(rp.T);
+  const PartStat* ps = a.pstat + ((size_t)b * a.slots + slot) * a.nseg;
+  const TopPart* tp =
+      (!is_t && rp.mode == kSaguaro) ? a.tpart + ((size_t)b * Dm + d) * a.nseg : nullptr;
+  RowRes rr;
+  merge_row(ps, tp, a.nseg, !greedy, k2, a.saguaro_k, rr);
+  rr.lnZ = 0.0;
+  if (tp && !rr.bad) {
+    // Z = 1 - (1 - c) * sum_{x in K} q(x)
+    const double Td = (double)rp.T;
+    double mass = 0.0;
+    for (int i = 0; i < rr.ntop; ++i) mass += exp((double)rr.topv[i] / Td - rr.lse);
+    rr.lnZ = log1p(-(1.0 - (double)a.saguaro_c) * mass);
+  }
+  if ((threadIdx.x & 31) == 0) a.rowres[(size_t)b * a.slots + slot] = rr;
+}
+
+// The accept scan of request b by one full warp, once every row it reads has
+// been merged into a.rowres; rows: 2*D_max+1 entries of shared memory (a copy).
+// Writes the outputs (slot n too for greedy), the flags, the row LSEs and the
+// race description; returns the race kind (same on all lanes).
 __device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
   const int lane = threadIdx.x & 31;
   const int Dm = a.D_max;
@@ -135,30 +157,18 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
   const double Td = (double)rp.T;
   const double c = (double)a.saguaro_c;
 
-  // merge the rows this request reads, one row at a time with the whole warp
+  // the merged rows this request reads (written by other warps: read through L2)
   if (!err) {
-    const float k2 = greedy ? 0.0f : log2e_over_T(rp.T);
     uint32_t nonfinite = 0;
-    for (int slot = 0; slot < a.slots; ++slot) {
-      const bool is_t = slot <= Dm;
-      const int d = is_t ? slot : slot - Dm - 1;
-      const bool needed = is_t ? d <= rp.Db : (d < rp.Db && !greedy);
-      if (!needed) continue;
-      const PartStat* ps = a.pstat + ((size_t)b * a.slots + slot) * a.nseg;
-      const TopPart* tp =
-          (!is_t && saguaro) ? a.tpart + ((size_t)b * Dm + d) * a.nseg : nullptr;
-      RowRes rr;
-      merge_row(ps, tp, a.nseg, !greedy, k2, a.saguaro_k, rr);
-      nonfinite |= rr.bad ? kFlagNonfinite : 0u;
-      if (tp && !rr.bad) {
-        // Z = 1 - (1 - c) * sum_{x in K} q(x)
-        double mass = 0.0;
-        for (int i = 0; i < rr.ntop; ++i) mass += exp((double)rr.topv[i] / Td - rr.lse);
-        rr.lnZ = log1p(-(1.0 - c) * mass);
-      }
-      if (lane == 0) rows[slot] = rr;
+    for (int slot = lane; slot < a.slots; slot += 32) {
+      if (!slot_needed(a, slot, rp)) continue;
+      const uint4* src = reinterpret_cast<const uint4*>(a.rowres + (size_t)b * a.slots + slot);
+      uint4* dst = reinterpret_cast<uint4*>(rows + slot);
+#pragma unroll
+      for (int i = 0; i < (int)(sizeof(RowRes) / 16); ++i) dst[i] = __ldcg(src + i);
+      nonfinite |= rows[slot].bad ? kFlagNonfinite : 0u;
     }
-    err |= nonfinite;
+    err |= __reduce_or_sync(0xFFFFFFFFu, nonfinite);
   }
   __syncwarp();
 

@@ -39,7 +39,8 @@ enum : uint32_t {
   kFlagBadRowD = 1u << 9,
   kFlagNonfinite = 1u << 10,
   kFlagBadParam = 1u << 11,
-  kFlagErrors = kFlagBadToken | kFlagBadRowD | kFlagNonfinite | kFlagBadParam
+  kFlagErrors = kFlagBadToken | kFlagBadRowD | kFlagNonfinite | kFlagBadParam,
+  kStatusTimeout = 1u << 12   // a bounded wait of the fused kernel expired
 };
 
 // Partial statistics of one segment of one row (16 bytes).
@@ -59,6 +60,17 @@ struct __align__(16) PartStat {
 struct __align__(16) TopPart {
   float v[kMaxTopK];
   int i[kMaxTopK];
+};
+
+// One row's merged statistics (written by the warp that merges the row).
+struct __align__(16) RowRes {
+  double lse;   // natural-log LSE at T (stochastic rows)
+  double lnZ;   // saguaro draft rows: ln Z
+  int argmax;   // greedy target rows
+  uint32_t bad;
+  int ntop;
+  int top[kMaxTopK];
+  float topv[kMaxTopK];
 };
 
 // What the race of one request needs; written by the accept scan.
@@ -90,12 +102,10 @@ struct __align__(16) RacePart {
   int pad;
 };
 
-// Counters of the fused kernel (each on its own 128-byte line).
+// Counters of the fused kernel (on its own 128-byte line).
 struct __align__(128) FusedState {
-  unsigned int next_ticket;   // next statistics item
+  unsigned int next_ticket;   // next ticket
   unsigned int pad0[31];
-  unsigned int cursor;        // request whose race chunks are being claimed
-  unsigned int pad1[31];
 };
 
 // Everything a kernel needs, passed by value.
@@ -116,10 +126,11 @@ struct VerifyArgs {
   RaceDesc* rdesc;         // [B]
   RacePart* rpart;         // [B, nseg]
   unsigned int* rcount;    // [B] race segments finished
-  FusedState* fstate;      // fused kernel: tickets and race cursor
-  unsigned int* done;      // [B] fused kernel: statistics items finished
+  RowRes* rowres;          // [B, slots] merged rows
+  FusedState* fstate;      // fused kernel: ticket counter
+  unsigned int* row_done;  // [B, slots] fused kernel: segments of the row finished
+  unsigned int* req_rows;  // [B] fused kernel: rows of the request merged
   unsigned int* ready;     // [B] fused kernel: 0 running, 1 race published, 2 nothing to race
-  unsigned int* rclaim;    // [B] fused kernel: race segments claimed
   uint64_t seed;
   int B, D_max, V, dtype;
   int nvec, nseg, slots;
@@ -133,7 +144,7 @@ struct VerifyArgs {
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
 // [zero, total) holds the counters that must read zero when a fused launch starts.
 struct WsLayout {
-  size_t pstat, tpart, rdesc, rpart, zero, fstate, rcount, done, ready, rclaim, total;
+  size_t pstat, tpart, rowres, rdesc, rpart, zero, fstate, rcount, row_done, req_rows, ready, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -156,6 +167,8 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   off = align_up(off + (size_t)B * slots * nseg * sizeof(PartStat), 256);
   L.tpart = off;
   off = align_up(off + (saguaro ? (size_t)B * D_max * nseg * sizeof(TopPart) : 0), 256);
+  L.rowres = off;
+  off = align_up(off + (size_t)B * slots * sizeof(RowRes), 256);
   L.rdesc = off;
   off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
   L.rpart = off;
@@ -165,11 +178,11 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   off = align_up(off + sizeof(FusedState), 256);
   L.rcount = off;
   off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
-  L.done = off;
+  L.row_done = off;
+  off = align_up(off + (size_t)B * slots * sizeof(unsigned int), 256);
+  L.req_rows = off;
   off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
   L.ready = off;
-  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
-  L.rclaim = off;
   off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
   L.total = off;
   return L;
@@ -196,6 +209,11 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// Ask L2 to fetch `bytes` (a multiple of 16) from a 16-byte aligned address.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // bf16 halves of a 32-bit word as floats (exact widening).
