@@ -3,9 +3,7 @@
 // A persistent grid of warps walks the (request, row, segment) items in
 // request-major order, warp w taking items w, w + W, w + 2W, ... so that at any
 // moment the whole device streams one contiguous stretch of the logits; each
-// item is one warp's 8 KiB segment (stats_device.cuh).  While a warp reduces a
-// segment, L2 already fetches its next one (a bulk prefetch issued by one lane),
-// so HBM stays busy through the warp's compute phase.
+// item is one warp's 8 KiB segment (stats_device.cuh).
 #include "stats_device.cuh"
 
 namespace sv {
@@ -21,12 +19,6 @@ __global__ void __launch_bounds__(kThreads) row_stats_kernel(VerifyArgs a) {
   ItemWalker it;
   it.init(a, w0, W);
   for (unsigned i = w0; i < total; i += W, it.advance(a)) {
-    // while this segment is read and reduced, let L2 fetch the next one
-    if (i + W < total) {
-      ItemWalker nx = it;
-      nx.advance(a);
-      if (row_needed(a, nx.slot, load_req(a, nx.b))) prefetch_segment<DT>(a, nx.b, nx.slot, nx.seg);
-    }
     const ReqParams rp = load_req(a, it.b);
     if (!row_needed(a, it.slot, rp)) continue;  // parameter errors are reported by the scan
     stats_item<DT>(a, it.b, it.slot, it.seg, rp);

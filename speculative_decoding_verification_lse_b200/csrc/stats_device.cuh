@@ -265,20 +265,6 @@ __device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot,
   }
 }
 
-// Lane 0 asks L2 for segment `seg` of row `slot` of request b (aligned rows only).
-template <int DT>
-__device__ __forceinline__ void prefetch_segment(const VerifyArgs& a, int b, int slot, int seg) {
-  if ((threadIdx.x & 31) != 0) return;
-  const char* row = row_base(a, b, slot);
-  if (((uintptr_t)row & 15u) != 0) return;
-  const long long row_bytes = (long long)a.V * (DT == kF32 ? 4 : 2);
-  const long long off = (long long)seg * kSegVecs * 16;
-  long long n = row_bytes - off;
-  if (n > kSegVecs * 16) n = kSegVecs * 16;
-  n &= ~15ll;
-  if (n > 0) prefetch_l2_bulk(row + off, (uint32_t)n);
-}
-
 // (b, slot, seg) of work item `it` of the request-major item order, advanced
 // in steps of `stride` items without divisions.
 struct ItemWalker {
