@@ -173,6 +173,35 @@ SV_API int sv_verify_ex(const void* target_logits, const void* draft_logits,
                  int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
                  int32_t* out_accept_len, const sv_params* p);
 
+/*
+ * sv_verify_static: sv_verify_ex that allocates nothing.  (The pages have no
+ * counterpart; this is a service for callers.)
+ *
+ * For callers that must not allocate device memory, e.g. because the process's
+ * memory already belongs to a caching allocator that the library must not
+ * bypass, or because cudaMalloc/cudaFree can synchronise the device in a
+ * latency-critical decode loop.  The caller still passes every input and
+ * output; the scratch is a fixed array of SV_STATIC_WORKSPACE_BYTES in the
+ * library's own device memory, which every GPU that loads the library keeps
+ * until the process exits.  sv_params.workspace and workspace_bytes are ignored.
+ *   - Sizes whose sv_workspace_bytes(B, D_max, V, dtype) exceeds
+ *     SV_STATIC_WORKSPACE_BYTES are rejected with SV_ERR_UNSUPPORTED (nothing
+ *     launched; sv_last_error says why).  8 MiB covers B=256, D=7, V=128256.
+ *   - The first call on a device looks up the array's device address (and does
+ *     the same one-time device queries as sv_verify_ex); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     each call clears what must start at zero itself.  Calls that overlap on
+ *     the GPU (other streams, other host threads) race on it: run them on one
+ *     stream, or give each its own workspace through sv_verify_ex.
+ * Otherwise identical to sv_verify_ex (same arguments, results and errors).
+ */
+#define SV_STATIC_WORKSPACE_BYTES (8u << 20)
+SV_API int sv_verify_static(const void* target_logits, const void* draft_logits,
+                            const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max,
+                            int V, int dtype, float temperature, int mode, uint64_t seed,
+                            int32_t* out_tokens, int32_t* out_accept_len, const sv_params* p);
+
 /* Bytes of scratch one call with these sizes needs (for sv_params.workspace). */
 SV_API size_t sv_workspace_bytes(int B, int D_max, int V, int dtype);
 

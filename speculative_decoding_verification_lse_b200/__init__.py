@@ -76,6 +76,8 @@ def load(build_if_needed=True):
     L.sv_verify.restype = ctypes.c_int
     L.sv_verify_ex.argtypes = _VERIFY_ARGS + [ctypes.POINTER(SvParams)]
     L.sv_verify_ex.restype = ctypes.c_int
+    L.sv_verify_static.argtypes = _VERIFY_ARGS + [ctypes.POINTER(SvParams)]
+    L.sv_verify_static.restype = ctypes.c_int
     L.sv_verify_greedy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_void_p, ctypes.c_void_p]
@@ -130,6 +132,18 @@ def sv_verify_ex(target_logits, draft_logits, draft_tokens, row_D, B, D_max, V, 
                                B, D_max, V, dtype, temperature, mode, seed & (2**64 - 1),
                                _p(out_tokens), _p(out_accept_len),
                                ctypes.byref(params) if params is not None else None)
+
+
+def sv_verify_static(target_logits, draft_logits, draft_tokens, row_D, B, D_max, V, dtype,
+                     temperature, mode, seed, out_tokens, out_accept_len, params=None):
+    """sv_verify_ex without any device allocation (fixed in-library scratch)."""
+    return load().sv_verify_static(_p(target_logits), _p(draft_logits), _p(draft_tokens),
+                                   _p(row_D), B, D_max, V, dtype, temperature, mode,
+                                   seed & (2**64 - 1), _p(out_tokens), _p(out_accept_len),
+                                   ctypes.byref(params) if params is not None else None)
+
+
+SV_STATIC_WORKSPACE_BYTES = 8 << 20
 
 
 def sv_workspace_bytes(B, D_max, V, dtype):

@@ -105,6 +105,9 @@ int cached_workspace(int dev, size_t bytes, void** out) {
 }
 
 }  // namespace
+
+int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 }  // namespace sv
 
 using namespace sv;
