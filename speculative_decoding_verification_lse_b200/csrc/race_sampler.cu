@@ -7,7 +7,7 @@ namespace sv {
 namespace {
 
 template <int DT>
-__global__ void __launch_bounds__(kThreads) race_kernel(VerifyArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) race_kernel(VerifyArgs a) {
   __shared__ RaceDesc s_rd[kWarps];
   const int warp = threadIdx.x >> 5;
   const long long item = (long long)blockIdx.x * kWarps + warp;

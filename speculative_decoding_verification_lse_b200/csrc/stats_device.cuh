@@ -94,16 +94,14 @@ __device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* ro
   }
 }
 
-// Statistics of segment `seg` of one row, by one full warp.
+// Statistics of one segment whose lane vectors are raw[0..kLaneVecs-1] (the
+// vectors seg*kSegVecs + lane + 32 j of the row), by one full warp.
 template <int DT, bool LSE, bool ARGMAX, bool TOP>
-__device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* row, int seg,
-                                              float k2, int topk, PartStat* out, TopPart* tout) {
+__device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], int seg, float k2,
+                                             int topk, PartStat* out, TopPart* tout) {
   constexpr int VEC = DT == kF32 ? 4 : 8;
   const int lane = threadIdx.x & 31;
   const int v0 = seg * kSegVecs + lane;
-  uint4 raw[kLaneVecs];
-  load_segment<DT>(a, row, seg, raw);
-
   // ---- lane maximum, with NaN / +inf detection
   float m_t;
   uint32_t bad = 0;
@@ -235,6 +233,30 @@ __device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* r
   }
 }
 
+// Statistics of segment `seg` of one row, by one full warp, loading through registers.
+template <int DT, bool LSE, bool ARGMAX, bool TOP>
+__device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* row, int seg,
+                                              float k2, int topk, PartStat* out, TopPart* tout) {
+  uint4 raw[kLaneVecs];
+  load_segment<DT>(a, row, seg, raw);
+  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, seg, k2, topk, out, tout);
+}
+
+// The same from a copy of the segment in shared memory (vector i of the
+// segment at smem[i], nv vectors valid; the rest of the buffer is stale and
+// reads as -inf).
+template <int DT, bool LSE, bool ARGMAX, bool TOP>
+__device__ __forceinline__ void stats_segment_smem(const uint4* smem, int nv, int seg, float k2,
+                                                   int topk, PartStat* out, TopPart* tout) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t fill = DT == kF32 ? kNegInfF32 : kNegInfBf2;
+  uint4 raw[kLaneVecs];
+#pragma unroll
+  for (int j = 0; j < kLaneVecs; ++j)
+    raw[j] = lane + 32 * j < nv ? smem[lane + 32 * j] : make_uint4(fill, fill, fill, fill);
+  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, seg, k2, topk, out, tout);
+}
+
 // Whether row `slot` of a request with parameters rp is read by the rule.
 __device__ __forceinline__ bool row_needed(const VerifyArgs& a, int slot, const ReqParams& rp) {
   if (rp.err) return false;
@@ -263,6 +285,41 @@ __device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot,
   } else {
     stats_segment<DT, true, false, false>(a, row, seg, k2, 0, out, nullptr);
   }
+}
+
+// Statistics of segment `seg` of row `slot` of request b from its copy in
+// shared memory (one full warp).
+template <int DT>
+__device__ __forceinline__ void stats_item_smem(const VerifyArgs& a, const uint4* smem, int nv,
+                                                int b, int slot, int seg, const ReqParams& rp) {
+  const bool is_target = slot <= a.D_max;
+  PartStat* out = a.pstat + ((size_t)b * a.slots + slot) * a.nseg + seg;
+  const float k2 = rp.mode == kGreedy ? 0.0f : log2e_over_T(rp.T);
+  if (is_target) {
+    if (rp.mode == kGreedy)
+      stats_segment_smem<DT, false, true, false>(smem, nv, seg, k2, 0, out, nullptr);
+    else
+      stats_segment_smem<DT, true, false, false>(smem, nv, seg, k2, 0, out, nullptr);
+  } else if (rp.mode == kSaguaro) {
+    TopPart* tout = a.tpart + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * a.nseg + seg;
+    stats_segment_smem<DT, true, false, true>(smem, nv, seg, k2, a.saguaro_k, out, tout);
+  } else {
+    stats_segment_smem<DT, true, false, false>(smem, nv, seg, k2, 0, out, nullptr);
+  }
+}
+
+// Bytes of segment `seg` of a row that one bulk copy can bring to shared
+// memory, or 0 when the segment must be read through registers (a row not
+// 16-byte aligned, or a last segment whose length is not a multiple of 16).
+template <int DT>
+__device__ __forceinline__ uint32_t bulk_bytes(const VerifyArgs& a, const char* row, int seg) {
+  if (((uintptr_t)row & 15u) != 0) return 0u;
+  const long long row_bytes = (long long)a.V * (DT == kF32 ? 4 : 2);
+  const long long off = (long long)seg * kSegVecs * 16;
+  long long n = row_bytes - off;
+  if (n > kSegVecs * 16) n = kSegVecs * 16;
+  if (n <= 0 || (n & 15)) return 0u;
+  return (uint32_t)n;
 }
 
 // (b, slot, seg) of work item `it` of the request-major item order, advanced
