@@ -5,22 +5,39 @@
 
 using namespace sv;
 
+template <int DT, bool RES, bool SAG>
+__device__ void probe_segment(const VerifyArgs& a, const RaceDesc& rd, const char* trow,
+                              const char* qrow, int seg, float* bounds, double* exact) {
+  const RaceStream R = race_stream(a.seed, rd.g);
+  race_bounds<DT, RES, SAG>(a, rd, R, trow, qrow, seg, [&](float b, int x) {
+    if (x < a.V) {
+      bounds[x] = b;
+      exact[x] = exact_key_of(a, rd, trow, qrow, RES, x);
+    }
+  });
+}
+
+template <int DT>
+__device__ void probe_dispatch(const VerifyArgs& a, const RaceDesc& rd, const char* trow,
+                               const char* qrow, int residual, int seg, float* bounds,
+                               double* exact) {
+  if (!residual)
+    probe_segment<DT, false, false>(a, rd, trow, qrow, seg, bounds, exact);
+  else if (rd.ntop > 0)
+    probe_segment<DT, true, true>(a, rd, trow, qrow, seg, bounds, exact);
+  else
+    probe_segment<DT, true, false>(a, rd, trow, qrow, seg, bounds, exact);
+}
+
 __global__ void probe_kernel(VerifyArgs a, RaceDesc rd, const char* trow, const char* qrow,
                              int residual, float* bounds, double* exact) {
   const int warp = threadIdx.x >> 5;
   const int seg = blockIdx.x * (blockDim.x >> 5) + warp;
   if (seg >= a.nseg) return;
-  const RaceStream R = race_stream(a.seed, rd.g);
   if (a.dtype == kF32)
-    race_bounds<kF32>(a, rd, R, trow, qrow, residual != 0, seg, [&](float b, int x) {
-      bounds[x] = b;
-      exact[x] = exact_key_of(a, rd, trow, qrow, residual != 0, x);
-    });
+    probe_dispatch<kF32>(a, rd, trow, qrow, residual, seg, bounds, exact);
   else
-    race_bounds<kBF16>(a, rd, R, trow, qrow, residual != 0, seg, [&](float b, int x) {
-      bounds[x] = b;
-      exact[x] = exact_key_of(a, rd, trow, qrow, residual != 0, x);
-    });
+    probe_dispatch<kBF16>(a, rd, trow, qrow, residual, seg, bounds, exact);
 }
 
 // All pointers are device pointers; lse values are natural-log LSEs at T.
