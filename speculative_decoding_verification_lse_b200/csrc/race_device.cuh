@@ -145,93 +145,93 @@ __device__ __forceinline__ double exact_key_of(const VerifyArgs& a, const RaceDe
   return exact_key(zt, zq, x, race_word(a.seed, rd.g, x), rd, residual);
 }
 
-// Four consecutive logits starting at token x (x a multiple of 4), widened to
-// float; -inf past the end of the row.  An 8-byte (bf16) or 16-byte (fp32) load
-// when the row allows it.
-template <int DT>
-__device__ __forceinline__ float4 load4(const char* row, int x, int V, bool aligned) {
-  if (aligned && x + 4 <= V) {
-    if (DT == kF32) return __ldcs(reinterpret_cast<const float4*>(row) + (x >> 2));
-    const uint2 w = __ldcs(reinterpret_cast<const uint2*>(row) + (x >> 2));
-    return make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
-  }
-  float f[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) f[e] = x + e < V ? logit_at<DT>(row, x + e) : -INFINITY;
-  return make_float4(f[0], f[1], f[2], f[3]);
-}
-
-// Upper bounds of the keys (log2 units) of one lane's tokens in segment `seg`:
-// the lane takes groups of four consecutive tokens (one Philox call each), the
-// warp covering 128 tokens per step.  Calls visit(bound, x) for each token; a
-// masked token, or one past the end of the row, gets a NaN bound, which never
-// compares true.  Every rounding and approximation error is covered by slack:
+// Upper bounds of the keys (log2 units) of one lane's tokens in segment `seg`;
+// calls visit(bound, x) for each.  Every rounding and approximation error is
+// covered by explicit slack:
 //   l2p = z*k2 - l2_t is within (|z| k2 + |l2_t|) 2^-22 of log2 p(x);
 //   log2 E >= lg2(E_lower) - 2^-16;
 //   residual, x outside K: d = log2 q'(x) - log2 p(x) >= dlo, and
 //     log2(1 - 2^d) <= lg2(1 - ex2(dlo)(1 - 2^-21)) + 2^-16;
 //   residual, x possibly in K (draft logit >= the smallest logit of K): r <= p.
-template <int DT, bool RESIDUAL, bool SAGUARO, typename Visit>
+// Pairs of tokens share packed fp32x2 arithmetic.
+template <int DT, typename Visit>
 __device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc& rd,
                                             const RaceStream& R, const char* trow,
-                                            const char* qrow, int seg, Visit&& visit) {
+                                            const char* qrow, bool residual, int seg,
+                                            Visit&& visit) {
+  constexpr int VEC = DT == kF32 ? 4 : 8;
   const int lane = threadIdx.x & 31;
-  const float k2 = rd.k2, l2t = rd.l2_t, l2q = rd.l2_q, kmin = rd.kmin;
-  const float ks = k2 * 0x1p-22f;
-  const float st = fmaf(fabsf(l2t), 0x1p-22f, 0x1p-16f);  // + the log2 E slack
-  const float sq = fabsf(l2q) * 0x1p-22f;
-  const bool aligned = ((uintptr_t)trow & (DT == kF32 ? 15u : 7u)) == 0 &&
-                       (!RESIDUAL || ((uintptr_t)qrow & (DT == kF32 ? 15u : 7u)) == 0);
-  const int x_begin = seg * kSegVecs * (DT == kF32 ? 4 : 8);
-  const int x_end = min(a.V, x_begin + kSegVecs * (DT == kF32 ? 4 : 8));
+  const float k2 = rd.k2;
+  const float l2t = rd.l2_t, l2q = rd.l2_q, kmin = rd.kmin;
+  const float2 kk = make_float2(k2, k2);
+  const float2 ks = make_float2(k2 * 0x1p-22f, k2 * 0x1p-22f);
+  const float2 nt = make_float2(-l2t, -l2t), nq = make_float2(-l2q, -l2q);
+  const float st1 = fmaf(fabsf(l2t), 0x1p-22f, 0x1p-16f);  // + the log2 E slack
+  const float2 st = make_float2(st1, st1);
+  const float sq1 = fabsf(l2q) * 0x1p-22f;
+  const float2 sq = make_float2(sq1, sq1);
+  const float2 shrink = make_float2(-(1.0f - 0x1p-21f), -(1.0f - 0x1p-21f));
+  const float2 one = make_float2(1.0f, 1.0f);
+  const int nfull = a.V / VEC;
+  const bool aligned =
+      ((uintptr_t)trow & 15u) == 0 && (!residual || ((uintptr_t)qrow & 15u) == 0);
 #pragma unroll 1
-  for (int x0 = x_begin + 4 * lane; x0 < x_end; x0 += 128) {
-    const float4 zt4 = load4<DT>(trow, x0, a.V, aligned);
-    float4 zq4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (RESIDUAL) zq4 = load4<DT>(qrow, x0, a.V, aligned);
-    const uint4 o4 = race_words_fast(R, (uint32_t)x0 >> 2);
+  for (int j = 0; j < kLaneVecs; ++j) {
+    const int v = seg * kSegVecs + lane + 32 * j;
+    if (v >= a.nvec) break;
+    uint4 wt, wq = make_uint4(0u, 0u, 0u, 0u);
+    if (aligned && v < nfull) {
+      wt = ld_stream16(trow + (size_t)v * 16);
+      if (residual) wq = ld_stream16(qrow + (size_t)v * 16);
+    } else {
+      wt = load_vec_checked<DT>(trow, v, a.V, a.nvec, nfull, aligned);
+      if (residual) wq = load_vec_checked<DT>(qrow, v, a.V, a.nvec, nfull, aligned);
+    }
 #pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-      const float2 zt = e == 0 ? make_float2(zt4.x, zt4.y) : make_float2(zt4.z, zt4.w);
-      const float2 El = e == 0 ? E_lower2(o4.x, o4.y) : E_lower2(o4.z, o4.w);
-      // log2 p(x) + slack, an upper bound (the log2 E slack is folded into st)
-      const float2 l2pu = __fadd2_rn(
-          __ffma2_rn(zt, make_float2(k2, k2), make_float2(-l2t, -l2t)),
-          __ffma2_rn(make_float2(fabsf(zt.x), fabsf(zt.y)), make_float2(ks, ks), make_float2(st, st)));
-      float2 bound = __fadd2_rn(l2pu, make_float2(-lg2_approx(El.x), -lg2_approx(El.y)));
-      if (RESIDUAL) {
-        // r = p (1 - q'/p): add an upper bound of log2(1 - 2^d), d = log2 q' - log2 p
-        const float2 zq = e == 0 ? make_float2(zq4.x, zq4.y) : make_float2(zq4.z, zq4.w);
-        // dlo = (zq k2 - l2q) - (|zq| ks + sq) - l2pu
-        const float2 sl = __ffma2_rn(make_float2(fabsf(zq.x), fabsf(zq.y)), make_float2(ks, ks),
-                                     make_float2(sq, sq));
-        const float2 l2ql = __ffma2_rn(zq, make_float2(k2, k2),
-                                       make_float2(-l2q - sl.x, -l2q - sl.y));
-        const float2 dlo = __fadd2_rn(l2ql, make_float2(-l2pu.x, -l2pu.y));
-        const float2 t = __ffma2_rn(make_float2(ex2_approx(dlo.x), ex2_approx(dlo.y)),
-                                    make_float2(-(1.0f - 0x1p-21f), -(1.0f - 0x1p-21f)),
-                                    make_float2(1.0f, 1.0f));
-        const float rx = dlo.x < 0.0f ? bound.x + (lg2_approx(t.x) + 0x1p-16f) : -INFINITY;
-        const float ry = dlo.y < 0.0f ? bound.y + (lg2_approx(t.y) + 0x1p-16f) : -INFINITY;
-        // a token that may belong to K keeps the bound r <= p
-        bound.x = (SAGUARO && zq.x >= kmin) ? bound.x : rx;
-        bound.y = (SAGUARO && zq.y >= kmin) ? bound.y : ry;
+    for (int h = 0; h < VEC / 4; ++h) {
+      const uint32_t base = (uint32_t)(v * VEC + 4 * h);
+      const uint4 o4 = race_words_fast(R, base >> 2);
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const float2 zt = make_float2(elem<DT>(wt, 4 * h + e), elem<DT>(wt, 4 * h + e + 1));
+        const float2 El = e == 0 ? E_lower2(o4.x, o4.y) : E_lower2(o4.z, o4.w);
+        // log2 p(x) + slack, an upper bound (the log2 E slack is folded into st)
+        const float2 l2pu = __fadd2_rn(__ffma2_rn(zt, kk, nt),
+                                       __ffma2_rn(make_float2(fabsf(zt.x), fabsf(zt.y)), ks, st));
+        float2 bound = __fadd2_rn(l2pu, make_float2(-lg2_approx(El.x), -lg2_approx(El.y)));
+        if (residual) {
+          // r = p (1 - q'/p): add an upper bound of log2(1 - 2^d), d = log2 q' - log2 p
+          const float2 zq = make_float2(elem<DT>(wq, 4 * h + e), elem<DT>(wq, 4 * h + e + 1));
+          const float2 dlo = __fadd2_rn(
+              __fadd2_rn(__ffma2_rn(zq, kk, nq),
+                         __fmul2_rn(__ffma2_rn(make_float2(fabsf(zq.x), fabsf(zq.y)), ks, sq),
+                                    make_float2(-1.0f, -1.0f))),
+              make_float2(-l2pu.x, -l2pu.y));
+          const float2 t = __ffma2_rn(make_float2(ex2_approx(dlo.x), ex2_approx(dlo.y)), shrink, one);
+          const float2 res = __fadd2_rn(bound, make_float2(lg2_approx(t.x) + 0x1p-16f,
+                                                           lg2_approx(t.y) + 0x1p-16f));
+          // a token of K keeps the bound r <= p; q' >= p excludes the token
+          bound.x = zq.x >= kmin ? bound.x : (dlo.x < 0.0f ? res.x : -INFINITY);
+          bound.y = zq.y >= kmin ? bound.y : (dlo.y < 0.0f ? res.y : -INFINITY);
+        }
+        const int x = (int)base + e;
+        if (x < a.V && zt.x > -INFINITY) visit(bound.x, x);
+        if (x + 1 < a.V && zt.y > -INFINITY) visit(bound.y, x + 1);
       }
-      visit(bound.x, x0 + e);
-      visit(bound.y, x0 + e + 1);
     }
   }
 }
 
 // The exact best and runner-up of segment `seg` (all lanes get the result).
-template <int DT, bool RESIDUAL, bool SAGUARO>
-__device__ __noinline__ Best race_segment_t(const VerifyArgs& a, const RaceDesc& rd,
-                                            const char* trow, const char* qrow, int seg) {
+template <int DT>
+__device__ __forceinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
+                                             const char* trow, const char* qrow,
+                                             bool residual, int seg) {
+  // A. the two largest bounds of each lane
   const RaceStream R = race_stream(a.seed, rd.g);
-  // A. the two largest bounds of each lane (NaN bounds never compare true)
   float u1 = -INFINITY, u2 = -INFINITY;
   int i1 = -1, i2 = -1;
-  race_bounds<DT, RESIDUAL, SAGUARO>(a, rd, R, trow, qrow, seg, [&](float bound, int x) {
+  race_bounds<DT>(a, rd, R, trow, qrow, residual, seg, [&](float bound, int x) {
     // branch-free: ties keep the earlier (lower) index
     const bool gt1 = bound > u1, gt2 = bound > u2;
     u2 = gt1 ? u1 : (gt2 ? bound : u2);
@@ -241,31 +241,22 @@ __device__ __noinline__ Best race_segment_t(const VerifyArgs& a, const RaceDesc&
   });
   // B. the exact key of each lane's best token
   Best B{-INFINITY, -INFINITY, -1};
-  if (i1 >= 0) offer(B, exact_key_of(a, rd, trow, qrow, RESIDUAL, i1), i1);
+  if (i1 >= 0) offer(B, exact_key_of(a, rd, trow, qrow, residual, i1), i1);
   double S1 = B.best;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) S1 = fmax(S1, __shfl_xor_sync(0xFFFFFFFFu, S1, o));
   // C. every token whose bound reaches S1 (less the margin) gets its exact key
   const float thr = S1 == -INFINITY ? -INFINITY : (float)(S1 * 1.4426950408889634) - 0x1p-14f;
   if (i2 >= 0 && u2 >= thr) {
-    offer(B, exact_key_of(a, rd, trow, qrow, RESIDUAL, i2), i2);
+    offer(B, exact_key_of(a, rd, trow, qrow, residual, i2), i2);
     // the third bound may have reached thr as well: visit them all
     const int j1 = i1, j2 = i2;
-    race_bounds<DT, RESIDUAL, SAGUARO>(a, rd, R, trow, qrow, seg, [&](float bound, int x) {
+    race_bounds<DT>(a, rd, R, trow, qrow, residual, seg, [&](float bound, int x) {
       if (bound >= thr && x != j1 && x != j2)
-        offer(B, exact_key_of(a, rd, trow, qrow, RESIDUAL, x), x);
+        offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
     });
   }
   return warp_combine(B);
-}
-
-template <int DT>
-__device__ __forceinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
-                                             const char* trow, const char* qrow,
-                                             bool residual, int seg) {
-  if (!residual) return race_segment_t<DT, false, false>(a, rd, trow, qrow, seg);
-  if (rd.ntop > 0) return race_segment_t<DT, true, true>(a, rd, trow, qrow, seg);
-  return race_segment_t<DT, true, false>(a, rd, trow, qrow, seg);
 }
 
 // Copy a request's race description into the warp's shared slot.

@@ -9,7 +9,7 @@ template <int DT, bool RES, bool SAG>
 __device__ void probe_segment(const VerifyArgs& a, const RaceDesc& rd, const char* trow,
                               const char* qrow, int seg, float* bounds, double* exact) {
   const RaceStream R = race_stream(a.seed, rd.g);
-  race_bounds<DT, RES, SAG>(a, rd, R, trow, qrow, seg, [&](float b, int x) {
+  race_bounds<DT>(a, rd, R, trow, qrow, RES, seg, [&](float b, int x) {
     if (x < a.V) {
       bounds[x] = b;
       exact[x] = exact_key_of(a, rd, trow, qrow, RES, x);
