@@ -215,14 +215,7 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.status = status;
   a.pstat = (PartStat*)((char*)ws + L.pstat);
   a.tpart = (TopPart*)((char*)ws + L.tpart);
-  a.rdesc = (RaceDesc*)((char*)ws + L.rdesc);
-  a.rpart = (RacePart*)((char*)ws + L.rpart);
-  a.rcount = (unsigned int*)((char*)ws + L.rcount);
-  a.rowres = (RowRes*)((char*)ws + L.rowres);
-  a.fstate = (FusedState*)((char*)ws + L.fstate);
-  a.row_done = (unsigned int*)((char*)ws + L.row_done);
-  a.req_rows = (unsigned int*)((char*)ws + L.req_rows);
-  a.ready = (unsigned int*)((char*)ws + L.ready);
+  a.barrier = (unsigned int*)((char*)ws + L.barrier);
   a.seed = seed;
   a.B = B;
   a.D_max = D_max;
@@ -240,9 +233,9 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   cudaStream_t s = (cudaStream_t)prm.stream;
   cudaEvent_t* ev = (cudaEvent_t*)prm.timing_events;
   if (fused) {
-    // the fused kernel's tickets, cursor and per-request counters start at zero
+    // the fused kernel's grid barrier starts at zero
     if ((e = cudaMemsetAsync((char*)ws + L.zero, 0, L.total - L.zero, s)) != cudaSuccess)
-      return cuda_fail(e, "cudaMemsetAsync(counters)");
+      return cuda_fail(e, "cudaMemsetAsync(barrier)");
     if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_fused(a, s, grid)) != cudaSuccess) return cuda_fail(e, "fused launch");
     if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -251,8 +244,7 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if ((e = launch_row_stats(a, s, grid)) != cudaSuccess) return cuda_fail(e, "row statistics launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  if ((e = launch_accept_scan(a, s)) != cudaSuccess) return cuda_fail(e, "accept scan launch");
-  if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");
+  if ((e = launch_tail(a, s)) != cudaSuccess) return cuda_fail(e, "scan and race launch");
   return SV_OK;
 }
 

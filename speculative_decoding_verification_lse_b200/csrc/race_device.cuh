@@ -1,5 +1,5 @@
 // race_device.cuh -- device code of the residual / bonus race, shared by the
-// split race kernel and the fused kernel.
+// split race kernel, the accept scan (its reference key) and the fused kernel.
 //
 // After a rejection at position n the token is drawn from norm(max(0, p - q))
 // ("Speculative Speculative Decoding – асинхронизируй это.", rule item 3);
@@ -10,25 +10,27 @@
 // Philox keyed by (seed, request, token), which picks x with probability
 // r(x) / sum r and does not depend on the order of any sum.
 //
-// Exactness.  The decision is taken on the exact key ln r(x) - ln E_x in double
-// precision, with the same formulas as the plain definition, but only for the
-// few tokens that can win.  One warp handles an 8 KiB segment of the row:
-//   A. every lane computes, for each of its tokens, a single-precision UPPER
-//      BOUND of the key in log2 units (ex2/lg2 based, with explicit slack for
-//      every rounding and approximation error; race_bounds) and keeps its two
-//      largest;
-//   B. each lane evaluates the exact key of its best token; S1 = warp maximum;
-//   C. a lane whose second bound reaches S1 (less a margin that also covers
-//      the 1e-6 near-tie band) evaluates that token too, and if its second
-//      bound reached S1 its third might have as well, so it re-scans its tokens
-//      and evaluates every one whose bound reaches S1.
-// No token whose exact key is within the band of the segment's best is ever
-// skipped, so the segment's best and runner-up are those of the exact keys.
+// Exactness.  The decision is taken on the exact key
+//   key(x) = ln r(x) - ln E_x,   E_x = -ln(1 - W_x),   W_x = (o_x + 1/2) 2^-32
+// in double precision, with the same formulas as the plain definition, but only
+// for the tokens that can matter.  Since r(x) <= p(x) and E_x >= W_x,
+//   key(x) <= ln p(x) - ln W_x,
+// so once the exact key K0 of any one real token is known, a token whose key
+// reaches K0 - delta must have a small Philox word:
+//   o_x + 1/2 <= 2^L(x),   L(x) = log2 p(x) + 32 - (K0 - delta) log2(e) = z_x k2 + C.
+// The word filter (word_filter) tests this with four instructions per token:
+// a packed FMA and add for L (its single-precision error is covered by slack
+// folded into C: filter_offset), a count of leading zeros of o_x, and an
+// integer add whose sign bit says "drop".  The race's best key is >= K0, so
+// every token within the near-tie band delta of the best survives the filter;
+// the survivors (a handful per row) get exact keys.
 //
-// Layout: one warp per (request, segment); the warp that completes the last
-// segment of a request (atomic counter, no waiting) merges the segment results
-// and writes the token.  The counter starts at zero: the split path's scan
-// clears it, the fused path clears it before the launch.
+// K0 comes from a search in the segment holding the sampled row's largest
+// logit (race_ref_key_warp), and grows as segments finish; where none is known
+// (K0 = -inf) a segment first takes the best exact key of its 32 lane-wise
+// largest logits, and if that is -inf too every token survives the filter.
+// One warp handles an 8 KiB segment (race_segment_in); the CTA that owns the
+// request combines the segments (tail_device.cuh).
 #pragma once
 #include "philox.cuh"
 #include "stats_device.cuh"
@@ -81,31 +83,10 @@ __device__ __forceinline__ Best warp_combine(Best v) {
   return v;
 }
 
-// A lower bound of E = -ln(1 - W), W = (o + 1/2) 2^-32, within 2^-12 of it, for
-// two words at once.
-//   W < 2^-10 (o < 2^22): E >= W, and W is exact from the low 22 bits of o.
-//   otherwise: U = 1 - W <= Uup = 1 - (o >> 9) 2^-23 (exact in single precision),
-//   so E >= -ln Uup >= ln2 (-lg2(Uup) - 2^-16) (lg2's error, taken as at most
-//   2^-22 (1 + |result|), is below 2^-16 for Uup in [2^-23, 1 - 2^-10]).
-__device__ __forceinline__ float2 E_lower2(uint32_t o0, uint32_t o1) {
-  const float2 fa = __fadd2_rn(make_float2(__uint_as_float(0x4B000000u | (o0 & 0x3FFFFFu)),
-                                           __uint_as_float(0x4B000000u | (o1 & 0x3FFFFFu))),
-                               make_float2(-8388608.0f, -8388608.0f));
-  const float2 Ws = __ffma2_rn(fa, make_float2(0x1p-32f, 0x1p-32f), make_float2(0x1p-33f, 0x1p-33f));
-  const float2 fb = __fadd2_rn(make_float2(__uint_as_float(0x4B000000u | (o0 >> 9)),
-                                           __uint_as_float(0x4B000000u | (o1 >> 9))),
-                               make_float2(-8388608.0f, -8388608.0f));
-  const float2 Uup = __ffma2_rn(fb, make_float2(-0x1p-23f, -0x1p-23f), make_float2(1.0f, 1.0f));
-  const float2 El = __ffma2_rn(make_float2(lg2_approx(Uup.x), lg2_approx(Uup.y)),
-                               make_float2(-0.693147180559945f, -0.693147180559945f),
-                               make_float2(-0.693147180559945f * 0x1p-16f, -0.693147180559945f * 0x1p-16f));
-  return make_float2(o0 < 0x400000u ? Ws.x : El.x, o1 < 0x400000u ? Ws.y : El.y);
-}
-
 // The exact key ln r(x) - ln E_x in double precision, the plain definition's
 // formulas; -inf if x is no candidate.
 static __device__ __noinline__ double exact_key(float zt, float zq, int x, uint32_t o,
-                                         const RaceDesc& rd, bool residual) {
+                                                const RaceDesc& rd, bool residual) {
   const double lp = (double)zt / rd.T - rd.lse_t;
   if (lp == -INFINITY) return -INFINITY;
   double lr = lp;
@@ -145,180 +126,235 @@ __device__ __forceinline__ double exact_key_of(const VerifyArgs& a, const RaceDe
   return exact_key(zt, zq, x, race_word(a.seed, rd.g, x), rd, residual);
 }
 
-// Upper bounds of the keys (log2 units) of one lane's tokens in segment `seg`;
-// calls visit(bound, x) for each.  Every rounding and approximation error is
-// covered by explicit slack:
-//   l2p = z*k2 - l2_t is within (|z| k2 + |l2_t|) 2^-22 of log2 p(x);
-//   log2 E >= lg2(E_lower) - 2^-16;
-//   residual, x outside K: d = log2 q'(x) - log2 p(x) >= dlo, and
-//     log2(1 - 2^d) <= lg2(1 - ex2(dlo)(1 - 2^-21)) + 2^-16;
-//   residual, x possibly in K (draft logit >= the smallest logit of K): r <= p.
-// Pairs of tokens share packed fp32x2 arithmetic.
-template <int DT, typename Visit>
-__device__ __forceinline__ void race_bounds(const VerifyArgs& a, const RaceDesc& rd,
-                                            const RaceStream& R, const char* trow,
-                                            const char* qrow, bool residual, int seg,
-                                            Visit&& visit) {
-  constexpr int VEC = DT == kF32 ? 4 : 8;
-  const int lane = threadIdx.x & 31;
-  const float k2 = rd.k2;
-  const float l2t = rd.l2_t, l2q = rd.l2_q, kmin = rd.kmin;
-  const float2 kk = make_float2(k2, k2);
-  const float2 ks = make_float2(k2 * 0x1p-22f, k2 * 0x1p-22f);
-  const float2 nt = make_float2(-l2t, -l2t), nq = make_float2(-l2q, -l2q);
-  const float st1 = fmaf(fabsf(l2t), 0x1p-22f, 0x1p-16f);  // + the log2 E slack
-  const float2 st = make_float2(st1, st1);
-  const float sq1 = fabsf(l2q) * 0x1p-22f;
-  const float2 sq = make_float2(sq1, sq1);
-  const float2 shrink = make_float2(-(1.0f - 0x1p-21f), -(1.0f - 0x1p-21f));
-  const float2 one = make_float2(1.0f, 1.0f);
-  const int nfull = a.V / VEC;
-  const bool aligned =
-      ((uintptr_t)trow & 15u) == 0 && (!residual || ((uintptr_t)qrow & 15u) == 0);
-#pragma unroll 1
-  for (int j = 0; j < kLaneVecs; ++j) {
-    const int v = seg * kSegVecs + lane + 32 * j;
-    if (v >= a.nvec) break;
-    uint4 wt, wq = make_uint4(0u, 0u, 0u, 0u);
-    if (aligned && v < nfull) {
-      wt = ld_stream16(trow + (size_t)v * 16);
-      if (residual) wq = ld_stream16(qrow + (size_t)v * 16);
-    } else {
-      wt = load_vec_checked<DT>(trow, v, a.V, a.nvec, nfull, aligned);
-      if (residual) wq = load_vec_checked<DT>(qrow, v, a.V, a.nvec, nfull, aligned);
-    }
+constexpr double kRaceBand = 1e-5;  // delta: the 1e-6 near-tie band plus every rounding error
+
+// The word filter's offset C for the reference key K0 of a race on a target
+// row with LSE lse_t, raised by the filter's own error bound:
+//   C = 32 + (delta - lse_t - K0) log2(e).
+// The filter computes L = fl(fma(z, k2, C)).  k2 is within 2^-23 of log2(e)/T
+// (relative), the FMA rounds once, and |z k2| <= |L| + |C|, so where the
+// outcome depends on L (|L| <= 64) its error is below (64 + |C|) 2^-21.
+// +inf (keep every token) when K0 is -inf or C is too large to resolve.
+__device__ __forceinline__ float filter_offset(double K0, double lse_t) {
+  if (!(K0 > -INFINITY) || !(fabs(lse_t) < INFINITY)) return INFINITY;
+  const double C = 32.0 + (kRaceBand - lse_t - K0) * 1.4426950408889634;
+  if (!(fabs(C) < 0x1p24)) return INFINITY;
+  return __double2float_ru(C + (64.0 + fabs(C)) * 0x1p-21 + 0x1p-20);
+}
+
+// Tokens per lane in a segment, and the 32-bit words of their flags.
+template <int DT>
+struct Lanes {
+  static constexpr int VEC = DT == kF32 ? 4 : 8;
+  static constexpr int TOK = kLaneVecs * VEC;
+  static constexpr int WORDS = TOK / 32;
+};
+
+// The index of the most significant set bit of o, -1 for o = 0.
+__device__ __forceinline__ int msb_index(uint32_t o) {
+  int r;
+  asm("bfind.u32 %0, %1;" : "=r"(r) : "r"(o));
+  return r;
+}
+
+// The word filter over one group of 32 tokens of a lane: vectors j0 .. j0 +
+// 32/VEC - 1 of the lane (vector j of the lane is vector v0 + 32 j of the row),
+// logits in raw.  Returns the drop word: bit 31 - t is set when token t of the
+// group (element t mod VEC of vector j0 + t / VEC) cannot reach K0 - delta.
+// A token is kept iff o < 2^(rint(L) + 1) (>= 2^(L + 1/2)); with o's top set
+// bit at position m (m = -1 for o = 0) that is  m + 1 <= rint(L) + 1, i.e.
+//   bits(L + 1.5 * 2^23) - m - bits(1.5 * 2^23) >= 0:
+// for |L| < 2^22 the float sum holds rint(L) in its low bits, and below or
+// above that range (-inf included) the comparison still comes out right.
+template <int DT>
+__device__ __forceinline__ uint32_t word_filter(const uint4 (&raw)[32 / Lanes<DT>::VEC], int j0,
+                                                const RaceStream& R, int v0, float k2, float cup) {
+  constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC;
+  const float2 kk = make_float2(k2, k2), cc = make_float2(cup, cup);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  uint32_t drop = 0u;
+#pragma unroll
+  for (int jj = 0; jj < QV; ++jj) {
 #pragma unroll
     for (int h = 0; h < VEC / 4; ++h) {
-      const uint32_t base = (uint32_t)(v * VEC + 4 * h);
+      const uint32_t base = (uint32_t)((v0 + 32 * (j0 + jj)) * VEC + 4 * h);
       const uint4 o4 = race_words_fast(R, base >> 2);
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
-        const float2 zt = make_float2(elem<DT>(wt, 4 * h + e), elem<DT>(wt, 4 * h + e + 1));
-        const float2 El = e == 0 ? E_lower2(o4.x, o4.y) : E_lower2(o4.z, o4.w);
-        // log2 p(x) + slack, an upper bound (the log2 E slack is folded into st)
-        const float2 l2pu = __fadd2_rn(__ffma2_rn(zt, kk, nt),
-                                       __ffma2_rn(make_float2(fabsf(zt.x), fabsf(zt.y)), ks, st));
-        float2 bound = __fadd2_rn(l2pu, make_float2(-lg2_approx(El.x), -lg2_approx(El.y)));
-        if (residual) {
-          // r = p (1 - q'/p): add an upper bound of log2(1 - 2^d), d = log2 q' - log2 p
-          const float2 zq = make_float2(elem<DT>(wq, 4 * h + e), elem<DT>(wq, 4 * h + e + 1));
-          const float2 dlo = __fadd2_rn(
-              __fadd2_rn(__ffma2_rn(zq, kk, nq),
-                         __fmul2_rn(__ffma2_rn(make_float2(fabsf(zq.x), fabsf(zq.y)), ks, sq),
-                                    make_float2(-1.0f, -1.0f))),
-              make_float2(-l2pu.x, -l2pu.y));
-          const float2 t = __ffma2_rn(make_float2(ex2_approx(dlo.x), ex2_approx(dlo.y)), shrink, one);
-          const float2 res = __fadd2_rn(bound, make_float2(lg2_approx(t.x) + 0x1p-16f,
-                                                           lg2_approx(t.y) + 0x1p-16f));
-          // a token of K keeps the bound r <= p; q' >= p excludes the token
-          bound.x = zq.x >= kmin ? bound.x : (dlo.x < 0.0f ? res.x : -INFINITY);
-          bound.y = zq.y >= kmin ? bound.y : (dlo.y < 0.0f ? res.y : -INFINITY);
-        }
-        const int x = (int)base + e;
-        if (x < a.V && zt.x > -INFINITY) visit(bound.x, x);
-        if (x + 1 < a.V && zt.y > -INFINITY) visit(bound.y, x + 1);
+        const float2 z = make_float2(elem<DT>(raw[jj], 4 * h + e), elem<DT>(raw[jj], 4 * h + e + 1));
+        const float2 F = __fadd2_rn(__ffma2_rn(z, kk, cc), magic);
+        const uint32_t oa = e == 0 ? o4.x : o4.z, ob = e == 0 ? o4.y : o4.w;
+        const int ta = __float_as_int(F.x) - msb_index(oa) - 0x4B400000;
+        const int tb = __float_as_int(F.y) - msb_index(ob) - 0x4B400000;
+        drop = __funnelshift_l((uint32_t)ta, drop, 1);
+        drop = __funnelshift_l((uint32_t)tb, drop, 1);
       }
     }
   }
+  return drop;
 }
 
-// The exact best and runner-up of segment `seg` (all lanes get the result).
-template <int DT>
-__device__ __forceinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
-                                             const char* trow, const char* qrow,
-                                             bool residual, int seg) {
-  // A. the two largest bounds of each lane
-  const RaceStream R = race_stream(a.seed, rd.g);
-  float u1 = -INFINITY, u2 = -INFINITY;
-  int i1 = -1, i2 = -1;
-  race_bounds<DT>(a, rd, R, trow, qrow, residual, seg, [&](float bound, int x) {
-    // branch-free: ties keep the earlier (lower) index
-    const bool gt1 = bound > u1, gt2 = bound > u2;
-    u2 = gt1 ? u1 : (gt2 ? bound : u2);
-    i2 = gt1 ? i1 : (gt2 ? x : i2);
-    u1 = gt1 ? bound : u1;
-    i1 = gt1 ? x : i1;
-  });
-  // B. the exact key of each lane's best token
-  Best B{-INFINITY, -INFINITY, -1};
-  if (i1 >= 0) offer(B, exact_key_of(a, rd, trow, qrow, residual, i1), i1);
-  double S1 = B.best;
+// Vectors j0 .. j0 + NJ - 1 of one lane's part of segment `seg` (-inf past the
+// end of the row).
+template <int DT, int NJ>
+__device__ __forceinline__ void load_part(const VerifyArgs& a, const char* row, int seg, int j0,
+                                          uint4 (&raw)[NJ]) {
+  constexpr int VEC = Lanes<DT>::VEC;
+  const int nfull = a.V / VEC;
+  const int v0 = seg * kSegVecs + (threadIdx.x & 31) + 32 * j0;
+  const bool aligned = ((uintptr_t)row & 15u) == 0;
+  if (aligned && v0 + 32 * (NJ - 1) < nfull) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) S1 = fmax(S1, __shfl_xor_sync(0xFFFFFFFFu, S1, o));
-  // C. every token whose bound reaches S1 (less the margin) gets its exact key
-  const float thr = S1 == -INFINITY ? -INFINITY : (float)(S1 * 1.4426950408889634) - 0x1p-14f;
-  if (i2 >= 0 && u2 >= thr) {
-    offer(B, exact_key_of(a, rd, trow, qrow, residual, i2), i2);
-    // the third bound may have reached thr as well: visit them all
-    const int j1 = i1, j2 = i2;
-    race_bounds<DT>(a, rd, R, trow, qrow, residual, seg, [&](float bound, int x) {
-      if (bound >= thr && x != j1 && x != j2)
-        offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
-    });
+    for (int j = 0; j < NJ; ++j) raw[j] = ld_stream16(row + (size_t)(v0 + 32 * j) * 16);
+  } else {
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) raw[j] = load_vec_checked<DT>(row, v0 + 32 * j, a.V, a.nvec, nfull, aligned);
+  }
+}
+
+// The best exact key among the lanes' largest target logits of a segment (one
+// token per lane, the lowest index on ties), over the warp; -inf if none.
+template <int DT>
+__device__ __noinline__ double lane_max_key(const VerifyArgs& a, const RaceDesc& rd,
+                                            const char* trow, const char* qrow, bool residual,
+                                            int seg) {
+  constexpr int VEC = Lanes<DT>::VEC;
+  const int v0 = seg * kSegVecs + (threadIdx.x & 31);
+  float mv = -INFINITY;
+  int xi = -1;
+#pragma unroll 1
+  for (int j0 = 0; j0 < kLaneVecs; j0 += kLaneVecs / 2) {
+    uint4 raw[kLaneVecs / 2];
+    load_part<DT>(a, trow, seg, j0, raw);
+#pragma unroll
+    for (int j = 0; j < kLaneVecs / 2; ++j)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float z = elem<DT>(raw[j], e);
+        if (z > mv) {
+          mv = z;
+          xi = (v0 + 32 * (j0 + j)) * VEC + e;
+        }
+      }
+  }
+  double k = -INFINITY;
+  if (xi >= 0 && xi < a.V) k = exact_key_of(a, rd, trow, qrow, residual, xi);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) k = fmax(k, __shfl_xor_sync(0xFFFFFFFFu, k, o));
+  return k;
+}
+
+// The exact best and runner-up of segment `seg` among the tokens that can reach
+// K0 - delta (all lanes get the result); K0 and its filter offset cup come
+// from the caller, K0 = -inf when unknown.  A runner-up below best - delta may
+// come out lower than it is; no decision depends on it.  R is the race's
+// Philox stream.  The lane walks its part of the segment in groups of 32
+// tokens, loading the next group while it filters the current one, and takes
+// exact keys of a group's survivors (rare) right away, so the loop body stays
+// small enough for the instruction cache.
+template <int DT>
+__device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceDesc& rd,
+                                                const RaceStream& R, const char* trow,
+                                                const char* qrow, bool residual, int seg,
+                                                double K0, float cup) {
+  constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC, NG = kLaneVecs / QV;
+  const int v0 = seg * kSegVecs + (threadIdx.x & 31);
+  if (!(K0 > -INFINITY))
+    cup = filter_offset(lane_max_key<DT>(a, rd, trow, qrow, residual, seg), rd.lse_t);
+
+  Best B{-INFINITY, -INFINITY, -1};
+  uint4 cur[QV], nxt[QV];
+  load_part<DT>(a, trow, seg, 0, cur);
+#pragma unroll 1
+  for (int gi = 0; gi < NG; ++gi) {
+    if (gi + 1 < NG) load_part<DT>(a, trow, seg, (gi + 1) * QV, nxt);
+    uint32_t keep = ~word_filter<DT>(cur, gi * QV, R, v0, rd.k2, cup);
+    // exact keys of the survivors, one token per lane at a time
+    while (__any_sync(0xFFFFFFFFu, keep != 0u)) {
+      if (keep) {
+        const int t = __clz((int)keep);
+        keep &= ~(0x80000000u >> t);
+        const int x = (v0 + 32 * (gi * QV + t / VEC)) * VEC + t % VEC;
+        if (x < a.V) offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
+      }
+    }
+    if (gi + 1 < NG) {
+#pragma unroll
+      for (int j = 0; j < QV; ++j) cur[j] = nxt[j];
+    }
   }
   return warp_combine(B);
 }
 
-// Copy a request's race description into the warp's shared slot.
-__device__ __forceinline__ void load_race_desc(const RaceDesc* src, RaceDesc* dst) {
-  const int lane = threadIdx.x & 31;
-  constexpr int n16 = sizeof(RaceDesc) / 16;
-  static_assert(sizeof(RaceDesc) % 16 == 0, "RaceDesc is copied in 16-byte pieces");
-  if (lane < n16)
-    reinterpret_cast<uint4*>(dst)[lane] = __ldcg(reinterpret_cast<const uint4*>(src) + lane);
-  __syncwarp();
+template <int DT>
+__device__ __noinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
+                                          const char* trow, const char* qrow, bool residual,
+                                          int seg, double K0, float cup) {
+  return race_segment_in<DT>(a, rd, race_stream(a.seed, rd.g), trow, qrow, residual, seg, K0, cup);
 }
 
-// Race segment `seg` of request b, by one warp (rd in the warp's shared slot).
-// The warp that completes the request's last segment merges and writes the token.
+// A quick approximate key (natural-log units) with the hardware's approximate
+// exp and log; it only ranks tokens in the search for a reference key.
+__device__ __forceinline__ float approx_key_fast(float zt, float zq, uint32_t o, float invT,
+                                                 float lse_t, float lse_q, bool residual) {
+  const float lp = zt * invT - lse_t;
+  float lr = lp;
+  if (residual) {
+    const float lq = zq * invT - lse_q;
+    lr = lq < lp ? lp + __logf(1.0f - __expf(lq - lp)) : -INFINITY;
+  }
+  const float W = ((float)o + 0.5f) * 0x1p-32f;
+  const float E = fmaxf(W, -__logf(1.0f - W));  // E >= W always holds
+  return lr - __logf(E);
+}
+
+// A reference key for the race of rd (request b), by one warp among nw: the
+// warp ranks its share of the 16-byte vectors of segment `seg` of the sampled
+// row (vectors warp*32 + lane, + 32 nw, ...) by approximate key and returns
+// the exact key of its best token (the same on every lane); -inf if none.
 template <int DT>
-__device__ inline void race_item(const VerifyArgs& a, int b, int seg, const RaceDesc& rd) {
+__device__ __forceinline__ double race_ref_key_warp(const VerifyArgs& a, const RaceDesc& rd,
+                                                    const RaceStream& R, int b, int seg,
+                                                    int warp, int nw) {
+  constexpr int VEC = Lanes<DT>::VEC;
   const int lane = threadIdx.x & 31;
   const bool residual = rd.kind == kRaceResidual;
   const char* trow = row_base(a, b, rd.n);
   const char* qrow = residual ? row_base(a, b, a.D_max + 1 + rd.n) : nullptr;
-  const Best sb = race_segment<DT>(a, rd, trow, qrow, residual, seg);
-
-  unsigned prev = 0;
-  if (lane == 0) {
-    RacePart p;
-    p.best = sb.best;
-    p.second = sb.second;
-    p.idx = sb.idx;
-    p.pad = 0;
-    a.rpart[(size_t)b * a.nseg + seg] = p;
-    __threadfence();
-    prev = atomicAdd(&a.rcount[b], 1u);
+  const int nfull = a.V / VEC;
+  const bool aligned =
+      ((uintptr_t)trow & 15u) == 0 && (!residual || ((uintptr_t)qrow & 15u) == 0);
+  const float invT = (float)(1.0 / rd.T), lse_t = (float)rd.lse_t;
+  const float lse_q = (float)(rd.lse_q + rd.ln_Z);
+  float best = -INFINITY;
+  int bx = INT_MAX;
+  const int vend = min(a.nvec, (seg + 1) * kSegVecs);
+  for (int v = seg * kSegVecs + 32 * warp + lane; v < vend; v += 32 * nw) {
+    const uint4 wt = load_vec_checked<DT>(trow, v, a.V, a.nvec, nfull, aligned);
+    uint4 wq = make_uint4(0u, 0u, 0u, 0u);
+    if (residual) wq = load_vec_checked<DT>(qrow, v, a.V, a.nvec, nfull, aligned);
+#pragma unroll
+    for (int h = 0; h < VEC / 4; ++h) {
+      const uint4 o4 = race_words_fast(R, (uint32_t)(v * VEC + 4 * h) >> 2);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int x = v * VEC + 4 * h + e;
+        const float zt = elem<DT>(wt, 4 * h + e);
+        const uint32_t o = e == 0 ? o4.x : e == 1 ? o4.y : e == 2 ? o4.z : o4.w;
+        const float k = approx_key_fast(zt, residual ? elem<DT>(wq, 4 * h + e) : 0.0f, o, invT,
+                                        lse_t, lse_q, residual);
+        if (x < a.V && zt > -INFINITY && k > best) {
+          best = k;
+          bx = x;
+        }
+      }
+    }
   }
-  prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-  if (prev != (unsigned)(a.nseg - 1)) return;
-
-  // the last segment of this request: merge every segment's result
-  __threadfence();
-  Best r{-INFINITY, -INFINITY, -1};
-  for (int s = lane; s < a.nseg; s += 32) {
-    const RacePart* pp = a.rpart + (size_t)b * a.nseg + s;
-    Best o;
-    o.best = __ldcg(&pp->best);
-    o.second = __ldcg(&pp->second);
-    o.idx = __ldcg(&pp->idx);
-    r = combine(r, o);
-  }
-  r = warp_combine(r);
-  uint32_t flags = rd.flags;
-  if (r.idx < 0 && residual) {
-    // {p > q} was empty through rounding: draw from p on the same row instead
-    flags |= kFlagResidualEmpty;
-    Best Bb{-INFINITY, -INFINITY, -1};
-    for (int s = 0; s < a.nseg; ++s) Bb = combine(Bb, race_segment<DT>(a, rd, trow, nullptr, false, s));
-    r = Bb;
-  }
-  if (lane == 0) {
-    if (r.best - r.second < 1e-6) flags |= kFlagRaceNearTie;
-    a.out_tokens[(size_t)b * (a.D_max + 1) + rd.n] = r.idx;
-    if (a.out_flags) a.out_flags[b] = flags;
-    if (flags & kFlagResidualEmpty) atomicOr(a.status, kFlagResidualEmpty);
-  }
+  // the warp's best (ties: the lower index), then its exact key on every lane
+  const unsigned long long w = warp_max_u64(value_index_key(best, bx));
+  const int x = key_index(w);
+  if (x == INT_MAX || !(key_value(w) > -INFINITY)) return -INFINITY;
+  return exact_key_of(a, rd, trow, qrow, residual, x);
 }
 
 }  // namespace sv

@@ -1,9 +1,6 @@
-// row_stats.cu -- the per-row statistics pass of the split path.
-//
-// A persistent grid of warps walks the (request, row, segment) items in
-// request-major order, warp w taking items w, w + W, w + 2W, ... so that at any
-// moment the whole device streams one contiguous stretch of the logits; each
-// item is one warp's 8 KiB segment (stats_device.cuh).
+// row_stats.cu -- the first kernel of the split path: the per-row statistics
+// pass (stats_device.cuh) on a persistent grid of warps, each item one warp's
+// 8 KiB segment of a row.
 #include "stats_device.cuh"
 
 namespace sv {
@@ -12,17 +9,7 @@ namespace {
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads) row_stats_kernel(VerifyArgs a) {
-  const unsigned W = gridDim.x * kWarps;
-  const unsigned w0 = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const unsigned total = (unsigned)a.B * (unsigned)a.slots * (unsigned)a.nseg;
-  if (w0 >= total) return;
-  ItemWalker it;
-  it.init(a, w0, W);
-  for (unsigned i = w0; i < total; i += W, it.advance(a)) {
-    const ReqParams rp = load_req(a, it.b);
-    if (!row_needed(a, it.slot, rp)) continue;  // parameter errors are reported by the scan
-    stats_item<DT>(a, it.b, it.slot, it.seg, rp);
-  }
+  stats_pass<DT>(a, blockIdx.x * kWarps + (threadIdx.x >> 5), gridDim.x * kWarps);
 }
 
 }  // namespace

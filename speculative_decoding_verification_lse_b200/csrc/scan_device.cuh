@@ -40,7 +40,7 @@ __device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg
                                  float k2, int k, RowRes& r) {
   const int lane = threadIdx.x & 31;
   float mx = -INFINITY;
-  int am = INT_MAX;
+  int am = INT_MAX, ms = nseg;
   uint32_t bad = 0;
   double Sd = 0.0;  // relative to 2^(mx*k2)
   for (int s = lane; s < nseg; s += 32) {
@@ -48,20 +48,24 @@ __device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg
     const float m = raw.x, S = raw.y;
     const int ai = __float_as_int(raw.z);
     bad |= __float_as_uint(raw.w);
-    if (m > mx) {  // segments ascend in index: strict '>' keeps the lowest index
+    if (m > mx || ms == nseg) {  // segments ascend: strict '>' keeps the lowest one
       if (lse && Sd > 0.0) Sd *= exp2((double)(mx * k2) - (double)(m * k2));
       mx = m;
       am = ai;
+      ms = s;
     }
     if (lse && S > 0.0f) Sd += (double)S * exp2((double)(m * k2) - (double)(mx * k2));
   }
-  const unsigned long long key = value_index_key(mx, am == INT_MAX ? INT_MAX - 1 : am);
-  const unsigned long long win = warp_max_u64(key);
+  // the lowest segment holding the largest value; its partial has the argmax
+  const unsigned long long win = warp_max_u64(value_index_key(mx, ms));
   const float M = key_value(win);
-  const int Mi = key_index(win);
+  const int Ms = key_index(win);
+  const unsigned src = __ffs(__ballot_sync(0xFFFFFFFFu, ms == Ms)) - 1;
+  const int Mi = __shfl_sync(0xFFFFFFFFu, am, src);
   bad = __any_sync(0xFFFFFFFFu, bad) ? 1u : 0u;
   if (M == -INFINITY) bad = 1u;  // every entry masked: no distribution
-  r.argmax = (Mi == INT_MAX - 1) ? INT_MAX : Mi;
+  r.argmax = Mi;
+  r.mseg = Ms < nseg ? Ms : 0;
   r.lse = NAN;
   if (lse) {
     const double Mk = (double)(M * k2);
@@ -109,8 +113,9 @@ __device__ __forceinline__ bool slot_needed(const VerifyArgs& a, int slot, const
   return is_t ? d <= rp.Db : (d < rp.Db && rp.mode != kGreedy);
 }
 
-// Merge row `slot` of request b (one full warp) into a.rowres.
-__device__ inline void merge_row_global(const VerifyArgs& a, int b, int slot, const ReqParams& rp) {
+// Merge row `slot` of request b (one full warp); lane 0 writes the result to dst.
+__device__ inline void merge_row_into(const VerifyArgs& a, int b, int slot, const ReqParams& rp,
+                                      RowRes* dst) {
   const int Dm = a.D_max;
   const bool greedy = rp.mode == kGreedy;
   const bool is_t = slot <= Dm;
@@ -129,14 +134,15 @@ __device__ inline void merge_row_global(const VerifyArgs& a, int b, int slot, co
     for (int i = 0; i < rr.ntop; ++i) mass += exp((double)rr.topv[i] / Td - rr.lse);
     rr.lnZ = log1p(-(1.0 - (double)a.saguaro_c) * mass);
   }
-  if ((threadIdx.x & 31) == 0) a.rowres[(size_t)b * a.slots + slot] = rr;
+  if ((threadIdx.x & 31) == 0) *dst = rr;
 }
 
 // The accept scan of request b by one full warp, once every row it reads has
-// been merged into a.rowres; rows: 2*D_max+1 entries of shared memory (a copy).
-// Writes the outputs (slot n too for greedy), the flags, the row LSEs and the
-// race description; returns the race kind (same on all lanes).
-__device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
+// been merged into rows (2*D_max+1 entries of shared memory).  Writes the
+// outputs (slot n too for greedy), the flags and the row LSEs, and lane 0
+// writes the race description to *rd; returns the race kind (same on all
+// lanes).
+__device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* rows, RaceDesc* rd) {
   const int lane = threadIdx.x & 31;
   const int Dm = a.D_max;
   const ReqParams rp = load_req(a, b);
@@ -157,20 +163,13 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
   const double Td = (double)rp.T;
   const double c = (double)a.saguaro_c;
 
-  // the merged rows this request reads (written by other warps: read through L2)
+  // the merged rows this request reads
   if (!err) {
     uint32_t nonfinite = 0;
-    for (int slot = lane; slot < a.slots; slot += 32) {
-      if (!slot_needed(a, slot, rp)) continue;
-      const uint4* src = reinterpret_cast<const uint4*>(a.rowres + (size_t)b * a.slots + slot);
-      uint4* dst = reinterpret_cast<uint4*>(rows + slot);
-#pragma unroll
-      for (int i = 0; i < (int)(sizeof(RowRes) / 16); ++i) dst[i] = __ldcg(src + i);
-      nonfinite |= rows[slot].bad ? kFlagNonfinite : 0u;
-    }
+    for (int slot = lane; slot < a.slots; slot += 32)
+      if (slot_needed(a, slot, rp) && rows[slot].bad) nonfinite = kFlagNonfinite;
     err |= __reduce_or_sync(0xFFFFFFFFu, nonfinite);
   }
-  __syncwarp();
 
   if (err) {
     for (int j = lane; j <= Dm; j += 32) ot[j] = -1;
@@ -180,8 +179,9 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
       a.out_al[b] = -1;
       if (a.out_flags) a.out_flags[b] = err;
       atomicOr(a.status, err);
-      a.rdesc[b].kind = kRaceNone;
+      rd->kind = kRaceNone;
     }
+    __syncwarp();
     return kRaceNone;
   }
 
@@ -241,36 +241,31 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, RowRes* rows) {
   if (lane == 0) {
     a.out_al[b] = n + 1;
     if (a.out_flags) a.out_flags[b] = flags;
-    RaceDesc rd;
-    rd.kind = kind;
-    rd.n = n;
-    rd.g = g;
-    rd.flags = flags;
-    rd.T = Td;
-    rd.lse_t = rows[n].lse;
-    rd.k2 = log2e_over_T(rp.T);
-    rd.l2_t = (float)(rows[n].lse * 1.4426950408889634);
-    rd.l2_q = 0.0f;
-    rd.kmin = INFINITY;
-    rd.lse_q = 0.0;
-    rd.ln_c = log(c);
-    rd.ln_Z = 0.0;
-    rd.ntop = 0;
+    rd->kind = kind;
+    rd->n = n;
+    rd->g = g;
+    rd->flags = flags;
+    rd->T = Td;
+    rd->lse_t = rows[n].lse;
+    rd->k2 = log2e_over_T(rp.T);
+    rd->K0 = -INFINITY;
+    rd->cup = INFINITY;
+    rd->lse_q = 0.0;
+    rd->ln_c = log(c);
+    rd->ln_Z = 0.0;
+    rd->ntop = 0;
+    rd->ref_seg = rows[n].mseg;
     if (kind == kRaceResidual) {
       const RowRes& rq = rows[Dm + 1 + n];
-      rd.lse_q = rq.lse;
-      double shift = rq.lse;
+      rd->lse_q = rq.lse;
       if (saguaro) {
-        rd.ln_Z = rq.lnZ;
-        rd.ntop = rq.ntop;
-        for (int i = 0; i < rq.ntop; ++i) rd.top[i] = rq.top[i];
-        shift = rq.lse + rq.lnZ;
-        if (rq.ntop > 0) rd.kmin = rq.topv[rq.ntop - 1];
+        rd->ln_Z = rq.lnZ;
+        rd->ntop = rq.ntop;
+        for (int i = 0; i < rq.ntop; ++i) rd->top[i] = rq.top[i];
       }
-      rd.l2_q = (float)(shift * 1.4426950408889634);
     }
-    a.rdesc[b] = rd;
   }
+  __syncwarp();
   return kind;
 }
 

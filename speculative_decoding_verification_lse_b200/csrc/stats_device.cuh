@@ -242,21 +242,6 @@ __device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* r
   stats_reduce<DT, LSE, ARGMAX, TOP>(raw, seg, k2, topk, out, tout);
 }
 
-// The same from a copy of the segment in shared memory (vector i of the
-// segment at smem[i], nv vectors valid; the rest of the buffer is stale and
-// reads as -inf).
-template <int DT, bool LSE, bool ARGMAX, bool TOP>
-__device__ __forceinline__ void stats_segment_smem(const uint4* smem, int nv, int seg, float k2,
-                                                   int topk, PartStat* out, TopPart* tout) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t fill = DT == kF32 ? kNegInfF32 : kNegInfBf2;
-  uint4 raw[kLaneVecs];
-#pragma unroll
-  for (int j = 0; j < kLaneVecs; ++j)
-    raw[j] = lane + 32 * j < nv ? smem[lane + 32 * j] : make_uint4(fill, fill, fill, fill);
-  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, seg, k2, topk, out, tout);
-}
-
 // Whether row `slot` of a request with parameters rp is read by the rule.
 __device__ __forceinline__ bool row_needed(const VerifyArgs& a, int slot, const ReqParams& rp) {
   if (rp.err) return false;
@@ -285,41 +270,6 @@ __device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot,
   } else {
     stats_segment<DT, true, false, false>(a, row, seg, k2, 0, out, nullptr);
   }
-}
-
-// Statistics of segment `seg` of row `slot` of request b from its copy in
-// shared memory (one full warp).
-template <int DT>
-__device__ __forceinline__ void stats_item_smem(const VerifyArgs& a, const uint4* smem, int nv,
-                                                int b, int slot, int seg, const ReqParams& rp) {
-  const bool is_target = slot <= a.D_max;
-  PartStat* out = a.pstat + ((size_t)b * a.slots + slot) * a.nseg + seg;
-  const float k2 = rp.mode == kGreedy ? 0.0f : log2e_over_T(rp.T);
-  if (is_target) {
-    if (rp.mode == kGreedy)
-      stats_segment_smem<DT, false, true, false>(smem, nv, seg, k2, 0, out, nullptr);
-    else
-      stats_segment_smem<DT, true, false, false>(smem, nv, seg, k2, 0, out, nullptr);
-  } else if (rp.mode == kSaguaro) {
-    TopPart* tout = a.tpart + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * a.nseg + seg;
-    stats_segment_smem<DT, true, false, true>(smem, nv, seg, k2, a.saguaro_k, out, tout);
-  } else {
-    stats_segment_smem<DT, true, false, false>(smem, nv, seg, k2, 0, out, nullptr);
-  }
-}
-
-// Bytes of segment `seg` of a row that one bulk copy can bring to shared
-// memory, or 0 when the segment must be read through registers (a row not
-// 16-byte aligned, or a last segment whose length is not a multiple of 16).
-template <int DT>
-__device__ __forceinline__ uint32_t bulk_bytes(const VerifyArgs& a, const char* row, int seg) {
-  if (((uintptr_t)row & 15u) != 0) return 0u;
-  const long long row_bytes = (long long)a.V * (DT == kF32 ? 4 : 2);
-  const long long off = (long long)seg * kSegVecs * 16;
-  long long n = row_bytes - off;
-  if (n > kSegVecs * 16) n = kSegVecs * 16;
-  if (n <= 0 || (n & 15)) return 0u;
-  return (uint32_t)n;
 }
 
 // (b, slot, seg) of work item `it` of the request-major item order, advanced
@@ -354,5 +304,22 @@ struct ItemWalker {
     b += d_b + carry;
   }
 };
+
+// The statistics pass: warp w0 of W walks the (request, row, segment) items
+// w0, w0 + W, w0 + 2W, ... in request-major order, so that at any moment the
+// device streams one contiguous stretch of the logits.  Rows the rule does not
+// read are skipped (parameter errors are reported by the scan).
+template <int DT>
+__device__ __forceinline__ void stats_pass(const VerifyArgs& a, unsigned w0, unsigned W) {
+  const unsigned total = (unsigned)a.B * (unsigned)a.slots * (unsigned)a.nseg;
+  if (w0 >= total) return;
+  ItemWalker it;
+  it.init(a, w0, W);
+  for (unsigned i = w0; i < total; i += W, it.advance(a)) {
+    const ReqParams rp = load_req(a, it.b);
+    if (!row_needed(a, it.slot, rp)) continue;
+    stats_item<DT>(a, it.b, it.slot, it.seg, rp);
+  }
+}
 
 }  // namespace sv

@@ -69,6 +69,7 @@ struct __align__(16) RowRes {
   int argmax;   // greedy target rows
   uint32_t bad;
   int ntop;
+  int mseg;     // the segment holding the row's largest logit (lowest such segment)
   int top[kMaxTopK];
   float topv[kMaxTopK];
 };
@@ -84,28 +85,12 @@ struct __align__(16) RaceDesc {
   double lse_q;      // natural-log LSE of draft row n (residual)
   double ln_c;       // saguaro: ln c
   double ln_Z;       // saguaro: ln Z of draft row n
+  double K0;         // the exact key of one real candidate of this race (-inf: none known)
   float k2;          // fl(log2(e) / T)
-  float l2_t;        // fl(lse_t * log2(e))
-  float l2_q;        // fl((lse_q + ln Z) * log2(e)): z*k2 - l2_q approximates log2 q'(x)
-                     // for every x outside K (ln Z = 0 unless saguaro)
-  float kmin;        // saguaro: the smallest logit in K (a token with a smaller draft
-                     // logit is not in K); +inf otherwise
+  float cup;         // the word filter's offset for K0 (race_device.cuh); +inf keeps every token
   int ntop;          // saguaro: size of K (0 otherwise)
   int top[kMaxTopK]; // saguaro: K of draft row n
-};
-
-// One race segment's result: the best and second-best exact keys and the winner.
-struct __align__(16) RacePart {
-  double best;
-  double second;
-  int idx;           // -1 if the segment had no candidate
-  int pad;
-};
-
-// Counters of the fused kernel (on its own 128-byte line).
-struct __align__(128) FusedState {
-  unsigned int next_ticket;   // next ticket
-  unsigned int pad0[31];
+  int ref_seg;       // the segment of target row n holding its largest logit
 };
 
 // Everything a kernel needs, passed by value.
@@ -123,14 +108,7 @@ struct VerifyArgs {
   unsigned int* status;    // the device status word
   PartStat* pstat;         // [B, slots, nseg]
   TopPart* tpart;          // [B, D_max, nseg] (saguaro draft rows)
-  RaceDesc* rdesc;         // [B]
-  RacePart* rpart;         // [B, nseg]
-  unsigned int* rcount;    // [B] race segments finished
-  RowRes* rowres;          // [B, slots] merged rows
-  FusedState* fstate;      // fused kernel: ticket counter
-  unsigned int* row_done;  // [B, slots] fused kernel: segments of the row finished
-  unsigned int* req_rows;  // [B] fused kernel: rows of the request merged
-  unsigned int* ready;     // [B] fused kernel: 0 running, 1 race published, 2 nothing to race
+  unsigned int* barrier;   // fused kernel: CTAs past the statistics pass (zero at launch)
   uint64_t seed;
   int B, D_max, V, dtype;
   int nvec, nseg, slots;
@@ -142,9 +120,9 @@ struct VerifyArgs {
 };
 
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
-// [zero, total) holds the counters that must read zero when a fused launch starts.
+// [zero, total) must read zero when a fused launch starts.
 struct WsLayout {
-  size_t pstat, tpart, rowres, rdesc, rpart, zero, fstate, rcount, row_done, req_rows, ready, total;
+  size_t pstat, tpart, zero, barrier, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -167,23 +145,9 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   off = align_up(off + (size_t)B * slots * nseg * sizeof(PartStat), 256);
   L.tpart = off;
   off = align_up(off + (saguaro ? (size_t)B * D_max * nseg * sizeof(TopPart) : 0), 256);
-  L.rowres = off;
-  off = align_up(off + (size_t)B * slots * sizeof(RowRes), 256);
-  L.rdesc = off;
-  off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
-  L.rpart = off;
-  off = align_up(off + (size_t)B * nseg * sizeof(RacePart), 256);
   L.zero = off;
-  L.fstate = off;
-  off = align_up(off + sizeof(FusedState), 256);
-  L.rcount = off;
-  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
-  L.row_done = off;
-  off = align_up(off + (size_t)B * slots * sizeof(unsigned int), 256);
-  L.req_rows = off;
-  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
-  L.ready = off;
-  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.barrier = off;
+  off = align_up(off + sizeof(unsigned int), 256);
   L.total = off;
   return L;
 }
@@ -209,54 +173,6 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
-}
-
-// ---- shared-memory barriers and bulk copies (the async proxy)
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
-               : "memory");
-}
-
-// Makes barrier initialisation visible to the async proxy.
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-// Orders this thread's earlier shared-memory accesses before later async-proxy ones.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16, 16-byte aligned both ends) from global to
-// this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
-                                              uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
 }
 
 // bf16 halves of a 32-bit word as floats (exact widening).
@@ -353,10 +269,7 @@ __device__ __forceinline__ float load_logit(const VerifyArgs& a, const char* row
 namespace sv {
 cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s, int grid);
 int row_stats_blocks_per_sm(int dtype);
-int row_stats_threads();
-cudaError_t launch_accept_scan(const VerifyArgs& a, cudaStream_t s);
-cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_tail(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
-size_t fused_smem_bytes(int D_max);
 int fused_blocks_per_sm(int dtype);
 }  // namespace sv
