@@ -327,7 +327,10 @@ def run_ours(args):
         step_bytes = w.algorithmic_bytes()
         used_variant = args.variant if args.variant != "auto" else "split"
         if used_variant == "fused":
-            kname, kbytes, ksrc = "fused_verify", step_bytes, ["speculative_decoding_verification_lse_b200/csrc/fused_verify.cu"]
+            kname, kbytes = "fused_verify", step_bytes
+            ksrc = ["speculative_decoding_verification_lse_b200/csrc/" + f
+                    for f in ("fused_verify.cu", "tail_device.cuh", "race_device.cuh", "scan_device.cuh",
+                              "stats_device.cuh", "sv_common.cuh", "philox.cuh")]
         else:
             # the statistics pass reads every needed logit row once
             rows_read = 0
@@ -335,6 +338,7 @@ def run_ours(args):
                 rows_read += (d + 1) + (0 if m == 1 else d)
             kname, kbytes = "row_stats", rows_read * w.V * (2 if w.dtype == 1 else 4)
             ksrc = ["speculative_decoding_verification_lse_b200/csrc/row_stats.cu",
+                    "speculative_decoding_verification_lse_b200/csrc/stats_device.cuh",
                     "speculative_decoding_verification_lse_b200/csrc/sv_common.cuh"]
         achieved = kbytes / (k_ms / 1e3) / 1e9
         tr = traffic_record(kname, ksrc)
@@ -377,7 +381,7 @@ def run_ours(args):
                 "launch_ms": k_ms,
             },
             "clocks": clocks.summary(),
-            "gpu_launches": (1 if used_variant == "fused" else 3) * args.steps,
+            "gpu_launches": (1 if used_variant == "fused" else 2) * args.steps,
             "e2e": e2e,
         }
         if args.cpu_baseline and world == 1:

@@ -172,9 +172,11 @@ __device__ __forceinline__ uint32_t word_filter(const uint4 (&raw)[32 / Lanes<DT
   constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC;
   const float2 kk = make_float2(k2, k2), cc = make_float2(cup, cup);
   const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  uint32_t drop = 0u;
+  // one flag accumulator per vector (independent chains), joined at the end
+  uint32_t acc[QV];
 #pragma unroll
   for (int jj = 0; jj < QV; ++jj) {
+    acc[jj] = 0u;
 #pragma unroll
     for (int h = 0; h < VEC / 4; ++h) {
       const uint32_t base = (uint32_t)((v0 + 32 * (j0 + jj)) * VEC + 4 * h);
@@ -186,11 +188,14 @@ __device__ __forceinline__ uint32_t word_filter(const uint4 (&raw)[32 / Lanes<DT
         const uint32_t oa = e == 0 ? o4.x : o4.z, ob = e == 0 ? o4.y : o4.w;
         const int ta = __float_as_int(F.x) - msb_index(oa) - 0x4B400000;
         const int tb = __float_as_int(F.y) - msb_index(ob) - 0x4B400000;
-        drop = __funnelshift_l((uint32_t)ta, drop, 1);
-        drop = __funnelshift_l((uint32_t)tb, drop, 1);
+        acc[jj] = __funnelshift_l((uint32_t)ta, acc[jj], 1);
+        acc[jj] = __funnelshift_l((uint32_t)tb, acc[jj], 1);
       }
     }
   }
+  uint32_t drop = 0u;
+#pragma unroll
+  for (int jj = 0; jj < QV; ++jj) drop = (drop << VEC) + acc[jj];
   return drop;
 }
 
