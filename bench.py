@@ -108,6 +108,14 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def tail_items(w, sms):
+    """Whether the library races a batch of this shape as items spread over the
+    GPU (three split launches) rather than one CTA per request (two)."""
+    seg_tokens = 4096 if w.dtype == 1 else 2048
+    nseg = -(-w.V // seg_tokens)
+    return w.B < sms and w.B * nseg > sms
+
+
 def traffic_record(kernel_name, sources):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source (else None)."""
@@ -381,7 +389,11 @@ def run_ours(args):
                 "launch_ms": k_ms,
             },
             "clocks": clocks.summary(),
-            "gpu_launches": (1 if used_variant == "fused" else 2) * args.steps,
+            # fused: one launch; split: statistics, then one kernel per request or
+            # the scan and the race items (the library's rule, in include/specverify.h)
+            "gpu_launches": (1 if used_variant == "fused" else
+                             3 if tail_items(w, torch.cuda.get_device_properties(dev).multi_processor_count)
+                             else 2) * args.steps,
             "e2e": e2e,
         }
         if args.cpu_baseline and world == 1:

@@ -88,8 +88,16 @@ enum { SV_STOCHASTIC = 0, SV_GREEDY = 1, SV_SAGUARO = 2 };
 /* return codes */
 enum { SV_OK = 0, SV_ERR_INVALID_ARG = -1, SV_ERR_UNSUPPORTED = -2, SV_ERR_CUDA = -3 };
 
-/* sv_params.variant */
+/* sv_params.variant: the launch structure (AUTO, SPLIT or FUSED), optionally OR-ed
+ * with one layout of the work after the statistics pass (both layouts give the
+ * same results; without one, the library takes ITEMS when B is below the device's
+ * multiprocessor count and B times the row's 8 KiB segments is above it, and
+ * PER_REQUEST otherwise):
+ *   SV_TAIL_PER_REQUEST: one CTA per request merges, scans and races it;
+ *   SV_TAIL_ITEMS: one CTA per request merges and scans, then one warp per
+ *     (request, segment of the sampled row) races. */
 enum { SV_VARIANT_AUTO = 0, SV_VARIANT_SPLIT = 1, SV_VARIANT_FUSED = 2 };
+enum { SV_TAIL_PER_REQUEST = 1 << 4, SV_TAIL_ITEMS = 1 << 5 };
 
 /* per-request flag bits (sv_params.out_flags) */
 enum {
@@ -125,7 +133,7 @@ typedef struct sv_params {
   const int8_t* mode_per_req;        /* [B] device; NULL: every request uses `mode` */
   int saguaro_k;                     /* size of K; <= 0 means 5; at most SV_MAX_SAGUARO_K */
   float saguaro_c;                   /* down-weighting factor in (0, 1]; <= 0 means 0.5 */
-  int variant;                       /* SV_VARIANT_*; AUTO picks per shape */
+  int variant;                       /* SV_VARIANT_* [| SV_TAIL_*]; AUTO picks per shape */
   uint32_t request_offset;           /* global index of request 0 (sharded batches) */
   float* out_row_lse;                /* [B, 2*D_max+1] device, optional: natural-log LSE of
                                         target rows (slots 0..D_max) and draft rows (slots

@@ -150,7 +150,10 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   const float c = prm.saguaro_c <= 0.0f ? 0.5f : prm.saguaro_c;
   if (!(c > 0.0f && c <= 1.0f))
     return fail(SV_ERR_INVALID_ARG, "saguaro_c must be in (0, 1] (got %g)", (double)c);
-  if (prm.variant < SV_VARIANT_AUTO || prm.variant > SV_VARIANT_FUSED)
+  const int tail_bits = prm.variant & (SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
+  const int base_variant = prm.variant & ~(SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
+  if (base_variant < SV_VARIANT_AUTO || base_variant > SV_VARIANT_FUSED ||
+      tail_bits == (SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS))
     return fail(SV_ERR_INVALID_ARG, "unknown variant %d", prm.variant);
   if (B == 0) return SV_OK;
   if (!target_logits || !out_tokens || !out_accept_len)
@@ -181,13 +184,14 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   (void)saguaro_possible;
   void* ws = prm.workspace;
   unsigned int* status = nullptr;
-  const bool fused = prm.variant == SV_VARIANT_FUSED;
-  int grid = 0;
+  const bool fused = base_variant == SV_VARIANT_FUSED;
+  int grid = 0, sms = 0;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     int rc = status_word(dev, &status);
     if (rc) return rc;
     if ((rc = persistent_grid(dev, dtype, fused, &grid))) return rc;
+    sms = device_cache(dev)->sms;
     if (ws) {
       if (prm.workspace_bytes < L.total)
         return fail(SV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes",
@@ -215,6 +219,11 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.status = status;
   a.pstat = (PartStat*)((char*)ws + L.pstat);
   a.tpart = (TopPart*)((char*)ws + L.tpart);
+  a.rdesc = (RaceDesc*)((char*)ws + L.rdesc);
+  a.rpart = (RacePart*)((char*)ws + L.rpart);
+  a.rcount = (unsigned int*)((char*)ws + L.rcount);
+  a.best_key = (unsigned long long*)((char*)ws + L.best_key);
+  a.rorder = (unsigned short*)((char*)ws + L.rorder);
   a.barrier = (unsigned int*)((char*)ws + L.barrier);
   a.seed = seed;
   a.B = B;
@@ -225,6 +234,10 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.nseg = nseg;
   a.slots = (int)slots;
   a.mode = mode;
+  // one CTA per request once every multiprocessor gets one, or when there are too few race
+  // segments to spread; else the scan, then race items over the whole GPU
+  const bool spread = B < sms && (long long)B * nseg > sms;
+  a.per_request = tail_bits == SV_TAIL_PER_REQUEST ? 1 : tail_bits == SV_TAIL_ITEMS ? 0 : (spread ? 0 : 1);
   a.temperature = temperature;
   a.saguaro_k = k;
   a.saguaro_c = c;
@@ -233,9 +246,9 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   cudaStream_t s = (cudaStream_t)prm.stream;
   cudaEvent_t* ev = (cudaEvent_t*)prm.timing_events;
   if (fused) {
-    // the fused kernel's grid barrier starts at zero
+    // the fused kernel's grid barriers start at zero
     if ((e = cudaMemsetAsync((char*)ws + L.zero, 0, L.total - L.zero, s)) != cudaSuccess)
-      return cuda_fail(e, "cudaMemsetAsync(barrier)");
+      return cuda_fail(e, "cudaMemsetAsync(barriers)");
     if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_fused(a, s, grid)) != cudaSuccess) return cuda_fail(e, "fused launch");
     if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -244,7 +257,12 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if ((e = launch_row_stats(a, s, grid)) != cudaSuccess) return cuda_fail(e, "row statistics launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  if ((e = launch_tail(a, s)) != cudaSuccess) return cuda_fail(e, "scan and race launch");
+  if (a.per_request) {
+    if ((e = launch_requests(a, s)) != cudaSuccess) return cuda_fail(e, "scan and race launch");
+    return SV_OK;
+  }
+  if ((e = launch_scan(a, s)) != cudaSuccess) return cuda_fail(e, "accept scan launch");
+  if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");
   return SV_OK;
 }
 

@@ -83,6 +83,17 @@ __device__ __forceinline__ Best warp_combine(Best v) {
   return v;
 }
 
+// Doubles as unsigned integers in the same order (-0 < +0 aside).
+__device__ __forceinline__ unsigned long long ordered_u64(double v) {
+  const unsigned long long b = (unsigned long long)__double_as_longlong(v);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ double from_ordered_u64(unsigned long long o) {
+  const unsigned long long b = (o >> 63) ? (o & 0x7FFFFFFFFFFFFFFFull) : ~o;
+  return __longlong_as_double((long long)b);
+}
+
 // The exact key ln r(x) - ln E_x in double precision, the plain definition's
 // formulas; -inf if x is no candidate.
 static __device__ __noinline__ double exact_key(float zt, float zq, int x, uint32_t o,
@@ -161,10 +172,10 @@ __device__ __forceinline__ int msb_index(uint32_t o) {
 // 32/VEC - 1 of the lane (vector j of the lane is vector v0 + 32 j of the row),
 // logits in raw.  Returns the drop word: bit 31 - t is set when token t of the
 // group (element t mod VEC of vector j0 + t / VEC) cannot reach K0 - delta.
-// A token is kept iff o < 2^(rint(L) + 1) (>= 2^(L + 1/2)); with o's top set
-// bit at position m (m = -1 for o = 0) that is  m + 1 <= rint(L) + 1, i.e.
-//   bits(L + 1.5 * 2^23) - m - bits(1.5 * 2^23) >= 0:
-// for |L| < 2^22 the float sum holds rint(L) in its low bits, and below or
+// A token is kept iff o < 2^ceil(L); with o's top set bit at position m
+// (m = -1 for o = 0) that is  m + 1 <= ceil(L), i.e.
+//   bits(L + 1.5 * 2^23, rounded up) - m - bits(1.5 * 2^23) - 1 >= 0:
+// for |L| < 2^22 the float sum holds ceil(L) in its low bits, and below or
 // above that range (-inf included) the comparison still comes out right.
 template <int DT>
 __device__ __forceinline__ uint32_t word_filter(const uint4 (&raw)[32 / Lanes<DT>::VEC], int j0,
@@ -184,10 +195,10 @@ __device__ __forceinline__ uint32_t word_filter(const uint4 (&raw)[32 / Lanes<DT
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
         const float2 z = make_float2(elem<DT>(raw[jj], 4 * h + e), elem<DT>(raw[jj], 4 * h + e + 1));
-        const float2 F = __fadd2_rn(__ffma2_rn(z, kk, cc), magic);
+        const float2 F = __fadd2_ru(__ffma2_ru(z, kk, cc), magic);
         const uint32_t oa = e == 0 ? o4.x : o4.z, ob = e == 0 ? o4.y : o4.w;
-        const int ta = __float_as_int(F.x) - msb_index(oa) - 0x4B400000;
-        const int tb = __float_as_int(F.y) - msb_index(ob) - 0x4B400000;
+        const int ta = __float_as_int(F.x) - msb_index(oa) - (0x4B400000 + 1);
+        const int tb = __float_as_int(F.y) - msb_index(ob) - (0x4B400000 + 1);
         acc[jj] = __funnelshift_l((uint32_t)ta, acc[jj], 1);
         acc[jj] = __funnelshift_l((uint32_t)tb, acc[jj], 1);
       }
@@ -215,6 +226,56 @@ __device__ __forceinline__ void load_part(const VerifyArgs& a, const char* row, 
 #pragma unroll
     for (int j = 0; j < NJ; ++j) raw[j] = load_vec_checked<DT>(row, v0 + 32 * j, a.V, a.nvec, nfull, aligned);
   }
+}
+
+// An upper bound, in log2 units, of token x's race key (key / ln 2), from
+// single-precision arithmetic with every rounding error covered; -inf when x
+// cannot be a candidate (masked, or q'(x) >= p(x) for certain in a residual
+// race).  It uses r <= p and E >= W like the word filter, but with the exact
+// word and, for a residual, the factor (1 - q'/p):
+//   key/ln2 <= log2 p(x) + log2(1 - 2^d) + 32 - log2(o + 1/2),
+//   d = log2 q'(x) - log2 p(x),
+// each term bounded with slack for its rounding: log2 p from one FMA on k2
+// (within 2^-23 of log2(e)/T), log2f and expm1f (1 ulp each), the conversions,
+// and the sums (all below the 2^-21 relative slack added to each term).
+static __device__ __noinline__ float key2_upper(const VerifyArgs& a, const RaceDesc& rd,
+                                                const char* trow, const char* qrow,
+                                                bool residual, int x) {
+  const bool f32 = a.dtype == kF32;
+  const float z = f32 ? logit_at<kF32>(trow, x) : logit_at<kBF16>(trow, x);
+  if (!(z > -INFINITY)) return -INFINITY;
+  const float k2 = rd.k2;
+  const float l2t = (float)(rd.lse_t * 1.4426950408889634);
+  float l2p = fmaf(z, k2, -l2t);
+  l2p += (fabsf(z) * k2 + fabsf(l2t) + fabsf(l2p)) * 0x1p-21f + 0x1p-40f;
+  float h = 0.0f;
+  if (residual) {
+    const float zq = f32 ? logit_at<kF32>(qrow, x) : logit_at<kBF16>(qrow, x);
+    if (zq > -INFINITY) {
+      const float l2qb = (float)((rd.lse_q + rd.ln_Z) * 1.4426950408889634);
+      float l2q = fmaf(zq, k2, -l2qb);
+      float lc = 0.0f;
+      if (rd.ntop > 0) {
+        bool in_k = false;
+        for (int i = 0; i < rd.ntop; ++i) in_k |= (rd.top[i] == x);
+        if (in_k) lc = (float)(rd.ln_c * 1.4426950408889634);
+      }
+      l2q += lc;
+      l2q -= (fabsf(zq) * k2 + fabsf(l2qb) + fabsf(lc) + fabsf(l2q)) * 0x1p-21f + 0x1p-40f;
+      const float d = __fsub_rd(l2q, l2p);  // a lower bound of d
+      if (!(d < 0.0f)) return -INFINITY;
+      // log2(1 - 2^d) falls as d rises, so d's lower bound gives an upper bound;
+      // d ln 2 is rounded down (more negative), 1 - 2^y = -expm1(y ln 2)
+      const float u = -expm1f(__fmul_rd(d, 0.6931471825f));
+      const float hl = log2f(u * (1.0f + 0x1p-21f));
+      h = hl + fabsf(hl) * 0x1p-21f + 0x1p-40f;
+    }
+  }
+  const uint32_t o = race_word(a.seed, rd.g, x);
+  const float lw = log2f((float)o + 0.5f);
+  const float nlw = 32.0f - lw + fabsf(lw) * 0x1p-21f + 0x1p-20f;
+  const float sum = l2p + h + nlw;
+  return sum + (fabsf(l2p) + fabsf(h) + fabsf(nlw)) * 0x1p-21f;
 }
 
 // The best exact key among the lanes' largest target logits of a segment (one
@@ -264,8 +325,13 @@ __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceD
                                                 double K0, float cup) {
   constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC, NG = kLaneVecs / QV;
   const int v0 = seg * kSegVecs + (threadIdx.x & 31);
-  if (!(K0 > -INFINITY))
-    cup = filter_offset(lane_max_key<DT>(a, rd, trow, qrow, residual, seg), rd.lse_t);
+  if (!(K0 > -INFINITY)) {
+    K0 = lane_max_key<DT>(a, rd, trow, qrow, residual, seg);
+    cup = filter_offset(K0, rd.lse_t);
+  }
+  // survivors whose single-precision bound falls below K0 - delta need no exact key
+  const float thr2 = K0 > -INFINITY ? __double2float_rd((K0 - kRaceBand) * 1.4426950408889634 - 1e-5)
+                                    : -INFINITY;
 
   Best B{-INFINITY, -INFINITY, -1};
   uint4 cur[QV], nxt[QV];
@@ -280,7 +346,8 @@ __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceD
         const int t = __clz((int)keep);
         keep &= ~(0x80000000u >> t);
         const int x = (v0 + 32 * (gi * QV + t / VEC)) * VEC + t % VEC;
-        if (x < a.V) offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
+        if (x < a.V && key2_upper(a, rd, trow, qrow, residual, x) >= thr2)
+          offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
       }
     }
     if (gi + 1 < NG) {

@@ -93,6 +93,14 @@ struct __align__(16) RaceDesc {
   int ref_seg;       // the segment of target row n holding its largest logit
 };
 
+// One race segment's result: the best and second-best exact keys and the winner.
+struct __align__(16) RacePart {
+  double best;
+  double second;
+  int idx;           // -1 if the segment had no survivor
+  int pad;
+};
+
 // Everything a kernel needs, passed by value.
 struct VerifyArgs {
   const void* target;
@@ -108,11 +116,17 @@ struct VerifyArgs {
   unsigned int* status;    // the device status word
   PartStat* pstat;         // [B, slots, nseg]
   TopPart* tpart;          // [B, D_max, nseg] (saguaro draft rows)
-  unsigned int* barrier;   // fused kernel: CTAs past the statistics pass (zero at launch)
+  RaceDesc* rdesc;         // [B] race descriptions (written by the scan)
+  RacePart* rpart;         // [B, nseg] race segment results
+  unsigned int* rcount;    // [B] race segments finished (zeroed by the scan)
+  unsigned long long* best_key;  // [B] best exact race key so far, ordered bits (set by the scan)
+  unsigned short* rorder;  // [B, nseg] race segments by descending largest logit (set by the scan)
+  unsigned int* barrier;   // fused kernel: two grid barriers' counters (zero at launch)
   uint64_t seed;
   int B, D_max, V, dtype;
   int nvec, nseg, slots;
   int mode;
+  int per_request;         // after the statistics: 1 = one CTA per request, 0 = scan then race items
   float temperature;
   int saguaro_k;
   float saguaro_c;
@@ -122,7 +136,7 @@ struct VerifyArgs {
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
 // [zero, total) must read zero when a fused launch starts.
 struct WsLayout {
-  size_t pstat, tpart, zero, barrier, total;
+  size_t pstat, tpart, rdesc, rpart, rcount, best_key, rorder, zero, barrier, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -145,9 +159,19 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   off = align_up(off + (size_t)B * slots * nseg * sizeof(PartStat), 256);
   L.tpart = off;
   off = align_up(off + (saguaro ? (size_t)B * D_max * nseg * sizeof(TopPart) : 0), 256);
+  L.rdesc = off;
+  off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
+  L.rpart = off;
+  off = align_up(off + (size_t)B * nseg * sizeof(RacePart), 256);
+  L.rcount = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.best_key = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned long long), 256);
+  L.rorder = off;
+  off = align_up(off + (size_t)B * nseg * sizeof(unsigned short), 256);
   L.zero = off;
   L.barrier = off;
-  off = align_up(off + sizeof(unsigned int), 256);
+  off = align_up(off + 2 * sizeof(unsigned int), 256);
   L.total = off;
   return L;
 }
@@ -269,7 +293,9 @@ __device__ __forceinline__ float load_logit(const VerifyArgs& a, const char* row
 namespace sv {
 cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s, int grid);
 int row_stats_blocks_per_sm(int dtype);
-cudaError_t launch_tail(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype);
 }  // namespace sv

@@ -1,49 +1,68 @@
-// tail_device.cuh -- everything after the statistics pass for one request, by
-// one CTA: merge the request's rows (scan_device.cuh), run the accept scan,
-// find a reference key for the race, then race the sampled row segment by
-// segment (race_device.cuh) and write the token.
-//
-// The CTA's warps share the best exact key found so far in shared memory, so a
-// warp's later segments are filtered against the best key of every segment
-// finished before them (a larger K0 leaves fewer survivors).  Nothing here
-// waits on another CTA.
+// tail_device.cuh -- everything after the statistics pass, in one of two
+// layouts (the launcher picks one per call):
+//   per request: one CTA per request merges the request's rows
+//     (scan_device.cuh), runs its accept scan, finds a reference key for the
+//     race's word filter and races the sampled row, its warps taking segments
+//     w, w + 8, ... and sharing the best key found so far in shared memory
+//     (tail_request).  Best when there are at least as many requests as
+//     multiprocessors.
+//   scan, then race items: one CTA per request does the merge, the scan and the
+//     reference key (scan_cta); then one warp per (request, segment) races the
+//     segment, and the warp that finishes a request's last segment (an atomic
+//     counter, no waiting) combines them and writes the token (race_item).
+//     The items are taken rank-major -- every request's segment with the
+//     largest logit first, then every request's second, ... -- so that by the
+//     later waves each request's best key so far (ordered bits in global
+//     memory, raised with an atomic maximum) is usually the row's best and the
+//     filter leaves almost no survivors.  Best for small batches, whose races
+//     it spreads over the whole GPU.
 #pragma once
 #include "race_device.cuh"
 #include "scan_device.cuh"
 
 namespace sv {
 
-constexpr int kTailWarps = 8;
-constexpr int kTailThreads = 32 * kTailWarps;
-
 struct TailShared {
   RowRes rows[2 * kMaxDraft + 1];
   RaceDesc rd;
-  double key[kTailWarps];
-  double best[kTailWarps], second[kTailWarps];
-  int idx[kTailWarps];
-  unsigned long long k0;  // the best exact key so far, as ordered bits
+  double key[kWarps];
+  double best[kWarps], second[kWarps];
+  int idx[kWarps];
+  unsigned long long k0;  // the best exact key so far (per-request layout), as ordered bits
 };
 
-// Doubles as unsigned integers in the same order (-0 < +0 aside).
-__device__ __forceinline__ unsigned long long ordered_u64(double v) {
-  const unsigned long long b = (unsigned long long)__double_as_longlong(v);
-  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+// The end of request b's race, by one warp: r is the combination of every
+// segment's result.  An empty residual ({p > q} empty through rounding) is
+// drawn from p on the same row instead; then the token and the flags are
+// written.
+template <int DT>
+__device__ __forceinline__ void finish_race(const VerifyArgs& a, int b, const RaceDesc& rd, Best r) {
+  const int lane = threadIdx.x & 31;
+  const bool residual = rd.kind == kRaceResidual;
+  uint32_t flags = rd.flags;
+  if (r.idx < 0 && residual) {
+    flags |= kFlagResidualEmpty;
+    const char* trow = row_base(a, b, rd.n);
+    Best Bb{-INFINITY, -INFINITY, -1};
+    for (int s = 0; s < a.nseg; ++s)
+      Bb = combine(Bb, race_segment<DT>(a, rd, trow, nullptr, false, s, -INFINITY, INFINITY));
+    r = Bb;
+  }
+  if (lane == 0) {
+    if (r.best - r.second < 1e-6) flags |= kFlagRaceNearTie;
+    a.out_tokens[(size_t)b * (a.D_max + 1) + rd.n] = r.idx;
+    if (a.out_flags) a.out_flags[b] = flags;
+    if (flags & kFlagResidualEmpty) atomicOr(a.status, kFlagResidualEmpty);
+  }
 }
 
-__device__ __forceinline__ double from_ordered_u64(unsigned long long o) {
-  const unsigned long long b = (o >> 63) ? (o & 0x7FFFFFFFFFFFFFFFull) : ~o;
-  return __longlong_as_double((long long)b);
-}
-
-// Request b, by the whole CTA (kTailThreads threads, S in shared memory).
-// Every thread returns at the same point.
+// Request b, everything after its statistics, by the whole CTA (kThreads
+// threads, S in shared memory); every thread returns at the same point.
 template <int DT>
 __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailShared& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int nw = kTailWarps;
   const ReqParams rp = load_req(a, b);
-  for (int slot = warp; slot < a.slots; slot += nw)
+  for (int slot = warp; slot < a.slots; slot += kWarps)
     if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
   __syncthreads();
   if (warp == 0) scan_request(a, b, S.rows, &S.rd);
@@ -55,23 +74,21 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
   }
 
   // the reference key, from the segment holding the sampled row's largest logit
-  const uint32_t g = a.request_offset + (uint32_t)b;
-  const RaceStream R = race_stream(a.seed, g);
-  const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, nw);
+  const RaceStream R = race_stream(a.seed, S.rd.g);
+  const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
   if (lane == 0) S.key[warp] = kw;
   if (threadIdx.x == 0) S.k0 = ordered_u64(-INFINITY);
   __syncthreads();
   double K0 = S.key[0];
 #pragma unroll
-  for (int w = 1; w < nw; ++w) K0 = fmax(K0, S.key[w]);
+  for (int w = 1; w < kWarps; ++w) K0 = fmax(K0, S.key[w]);
 
-  // the race, warp w taking segments w, w + nw, ...
+  // the race, warp w taking segments w, w + 8, ...
   const bool residual = kind == kRaceResidual;
-  const int n = S.rd.n;
-  const char* trow = row_base(a, b, n);
-  const char* qrow = residual ? row_base(a, b, a.D_max + 1 + n) : nullptr;
+  const char* trow = row_base(a, b, S.rd.n);
+  const char* qrow = residual ? row_base(a, b, a.D_max + 1 + S.rd.n) : nullptr;
   Best B{-INFINITY, -INFINITY, -1};
-  for (int seg = warp; seg < a.nseg; seg += nw) {
+  for (int seg = warp; seg < a.nseg; seg += kWarps) {
     const double K = fmax(K0, from_ordered_u64(*(volatile unsigned long long*)&S.k0));
     const Best sb = race_segment_in<DT>(a, S.rd, R, trow, qrow, residual, seg, K,
                                         filter_offset(K, S.rd.lse_t));
@@ -86,29 +103,120 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
   __syncthreads();
   if (warp == 0) {
     Best r{-INFINITY, -INFINITY, -1};
-    if (lane < nw) {
+    if (lane < kWarps) {
       r.best = S.best[lane];
       r.second = S.second[lane];
       r.idx = S.idx[lane];
     }
-    r = warp_combine(r);
-    uint32_t flags = S.rd.flags;
-    if (r.idx < 0 && residual) {
-      // {p > q} was empty through rounding: draw from p on the same row instead
-      flags |= kFlagResidualEmpty;
-      Best Bb{-INFINITY, -INFINITY, -1};
-      for (int s = 0; s < a.nseg; ++s)
-        Bb = combine(Bb, race_segment<DT>(a, S.rd, trow, nullptr, false, s, -INFINITY, INFINITY));
-      r = Bb;
-    }
-    if (lane == 0) {
-      if (r.best - r.second < 1e-6) flags |= kFlagRaceNearTie;
-      a.out_tokens[(size_t)b * (a.D_max + 1) + n] = r.idx;
-      if (a.out_flags) a.out_flags[b] = flags;
-      if (flags & kFlagResidualEmpty) atomicOr(a.status, kFlagResidualEmpty);
-    }
+    finish_race<DT>(a, b, S.rd, warp_combine(r));
   }
   __syncthreads();  // S is reused by the next request
+}
+
+// Request b, by the whole CTA (kThreads threads, S in shared memory); every
+// thread returns at the same point.  Writes the request's outputs (all of them
+// unless it races), and for a race a.rdesc[b] and the race counters.
+template <int DT>
+__device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared& S) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const ReqParams rp = load_req(a, b);
+  for (int slot = warp; slot < a.slots; slot += kWarps)
+    if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
+  __syncthreads();
+  if (warp == 0) scan_request(a, b, S.rows, &S.rd);
+  __syncthreads();
+  const int kind = S.rd.kind;
+  if (kind != kRaceNone) {
+    // the reference key: each warp ranks a share of the segment holding the
+    // sampled row's largest logit and takes the exact key of its best token
+    const RaceStream R = race_stream(a.seed, S.rd.g);
+    const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
+    if (lane == 0) S.key[warp] = kw;
+    // the race order: rank of each segment by its largest logit (ties: lower
+    // index first); rows of more than kThreads segments keep index order
+    for (int sg = threadIdx.x; sg < a.nseg; sg += kThreads) {
+      int rank = sg;
+      if (a.nseg <= kThreads) {
+        const PartStat* ps = a.pstat + ((size_t)b * a.slots + S.rd.n) * a.nseg;
+        const float m = __ldcg(&ps[sg].m);
+        rank = 0;
+        for (int j = 0; j < a.nseg; ++j) {
+          const float mj = __ldcg(&ps[j].m);
+          rank += (mj > m || (mj == m && j < sg)) ? 1 : 0;
+        }
+      }
+      a.rorder[(size_t)b * a.nseg + rank] = (unsigned short)sg;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      double K0 = lane < kWarps ? S.key[lane] : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) K0 = fmax(K0, __shfl_xor_sync(0xFFFFFFFFu, K0, o));
+      if (lane == 0) {
+        S.rd.K0 = K0;
+        S.rd.cup = filter_offset(K0, S.rd.lse_t);
+        a.rcount[b] = 0u;
+        a.best_key[b] = K0 > -INFINITY ? ordered_u64(K0) : 0ull;
+      }
+      __syncwarp();
+      constexpr int n16 = sizeof(RaceDesc) / 16;
+      static_assert(sizeof(RaceDesc) % 16 == 0, "RaceDesc is copied in 16-byte pieces");
+      if (lane < n16)
+        reinterpret_cast<uint4*>(a.rdesc + b)[lane] = reinterpret_cast<const uint4*>(&S.rd)[lane];
+    }
+  } else if (threadIdx.x == 0) {
+    a.rdesc[b].kind = kRaceNone;
+  }
+  __syncthreads();  // S is reused by the next request
+}
+
+// Race item `item` (rank-major: item = rank * B + b), by one warp; rd: the
+// warp's shared slot for the request's race description.
+template <int DT>
+__device__ __forceinline__ void race_item(const VerifyArgs& a, long long item, RaceDesc* rd) {
+  const int lane = threadIdx.x & 31;
+  const int b = (int)(item % a.B);
+  const int rank = (int)(item / a.B);
+  constexpr int n16 = sizeof(RaceDesc) / 16;
+  if (lane < n16)
+    reinterpret_cast<uint4*>(rd)[lane] = __ldcg(reinterpret_cast<const uint4*>(a.rdesc + b) + lane);
+  __syncwarp();
+  if (rd->kind == kRaceNone) return;
+  const int seg = __ldcg(&a.rorder[(size_t)b * a.nseg + rank]);
+  const bool residual = rd->kind == kRaceResidual;
+  const char* trow = row_base(a, b, rd->n);
+  const char* qrow = residual ? row_base(a, b, a.D_max + 1 + rd->n) : nullptr;
+  const unsigned long long bk = *(volatile unsigned long long*)&a.best_key[b];
+  const double K = fmax(rd->K0, bk ? from_ordered_u64(bk) : -INFINITY);
+  const Best sb = race_segment_in<DT>(a, *rd, race_stream(a.seed, rd->g), trow, qrow, residual,
+                                      seg, K, filter_offset(K, rd->lse_t));
+  unsigned prev = 0;
+  if (lane == 0) {
+    if (sb.idx >= 0) atomicMax(&a.best_key[b], ordered_u64(sb.best));
+    RacePart p;
+    p.best = sb.best;
+    p.second = sb.second;
+    p.idx = sb.idx;
+    p.pad = 0;
+    a.rpart[(size_t)b * a.nseg + seg] = p;
+    __threadfence();
+    prev = atomicAdd(&a.rcount[b], 1u);
+  }
+  prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+  if (prev != (unsigned)(a.nseg - 1)) return;
+
+  // the request's last segment: combine every segment's result
+  __threadfence();
+  Best r{-INFINITY, -INFINITY, -1};
+  for (int s = lane; s < a.nseg; s += 32) {
+    const RacePart* pp = a.rpart + (size_t)b * a.nseg + s;
+    Best o;
+    o.best = __ldcg(&pp->best);
+    o.second = __ldcg(&pp->second);
+    o.idx = __ldcg(&pp->idx);
+    r = combine(r, o);
+  }
+  finish_race<DT>(a, b, *rd, warp_combine(r));
 }
 
 }  // namespace sv

@@ -1,8 +1,9 @@
 // Test helper: for every token of one target row (and draft row), the race's
 // word-filter decision for a given reference key K0, the token's Philox race
-// word and its exact double-precision key (exact_key_of), so that a test can
-// check that the filter keeps every token whose key reaches K0 - 1e-6 and
-// drops the rest up to its documented slack.
+// word, the single-precision upper bound of its key (key2_upper, log2 units)
+// and its exact double-precision key (exact_key_of), so that a test can check
+// that the filter keeps every token whose key reaches K0 - 1e-6 and drops the
+// rest up to its documented slack, and that the bound is one.
 #include "race_device.cuh"
 
 using namespace sv;
@@ -10,7 +11,8 @@ using namespace sv;
 template <int DT>
 __device__ void probe_segment(const VerifyArgs& a, const RaceDesc& rd, const char* trow,
                               const char* qrow, bool residual, int seg, float cup,
-                              unsigned char* keep_out, unsigned* words, double* exact) {
+                              unsigned char* keep_out, unsigned* words, double* exact,
+                              float* upper) {
   constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC, NG = kLaneVecs / QV;
   const int v0 = seg * kSegVecs + (threadIdx.x & 31);
   const RaceStream R = race_stream(a.seed, rd.g);
@@ -24,20 +26,21 @@ __device__ void probe_segment(const VerifyArgs& a, const RaceDesc& rd, const cha
       keep_out[x] = ((drop >> (31 - t)) & 1u) ? 0 : 1;
       words[x] = race_word(a.seed, rd.g, x);
       exact[x] = exact_key_of(a, rd, trow, qrow, residual, x);
+      upper[x] = key2_upper(a, rd, trow, qrow, residual, x);
     }
   }
 }
 
 __global__ void probe_kernel(VerifyArgs a, RaceDesc rd, const char* trow, const char* qrow,
                              int residual, float cup, unsigned char* keep, unsigned* words,
-                             double* exact) {
+                             double* exact, float* upper) {
   const int warp = threadIdx.x >> 5;
   const int seg = blockIdx.x * (blockDim.x >> 5) + warp;
   if (seg >= a.nseg) return;
   if (a.dtype == kF32)
-    probe_segment<kF32>(a, rd, trow, qrow, residual != 0, seg, cup, keep, words, exact);
+    probe_segment<kF32>(a, rd, trow, qrow, residual != 0, seg, cup, keep, words, exact, upper);
   else
-    probe_segment<kBF16>(a, rd, trow, qrow, residual != 0, seg, cup, keep, words, exact);
+    probe_segment<kBF16>(a, rd, trow, qrow, residual != 0, seg, cup, keep, words, exact, upper);
 }
 
 __global__ void offset_kernel(double K0, double lse_t, float T, float* out) {
@@ -51,7 +54,7 @@ extern "C" int race_filter_probe(const void* trow, const void* qrow, int V, int 
                                  double lse_t, double lse_q, int ntop, const int* top,
                                  double ln_c, double ln_Z, unsigned long long seed, unsigned g,
                                  int residual, double K0, unsigned char* keep, unsigned* words,
-                                 double* exact, float* cup_out) {
+                                 double* exact, float* upper, float* cup_out) {
   VerifyArgs a;
   memset(&a, 0, sizeof a);
   a.V = V;
@@ -80,6 +83,6 @@ extern "C" int race_filter_probe(const void* trow, const void* qrow, int V, int 
   rd.k2 = h[1];
   *cup_out = cup;
   probe_kernel<<<(a.nseg + 7) / 8, 256>>>(a, rd, (const char*)trow, (const char*)qrow, residual,
-                                          cup, keep, words, exact);
+                                          cup, keep, words, exact, upper);
   return cudaDeviceSynchronize() == cudaSuccess ? 0 : 1;
 }

@@ -15,8 +15,12 @@ from speculative_decoding_verification_lse_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED],
-                                   ids=["split", "fused"])
+# both launch structures, each with both layouts of the work after the statistics
+VARIANTS = pytest.mark.parametrize(
+    "variant",
+    [sv.SV_VARIANT_SPLIT | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
+     sv.SV_VARIANT_FUSED | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_FUSED | sv.SV_TAIL_ITEMS],
+    ids=["split-per-request", "split-items", "fused-per-request", "fused-items"])
 
 
 def make_random(B, D, V, dtype=sv.SV_BF16, seed=0, draft_sd=1.0, T=1.0, mode=0):

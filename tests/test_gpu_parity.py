@@ -16,8 +16,12 @@ from gpu_util import compare, gpu_run, oracle_on
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED],
-                                   ids=["split", "fused"])
+# both launch structures, each with both layouts of the work after the statistics
+VARIANTS = pytest.mark.parametrize(
+    "variant",
+    [sv.SV_VARIANT_SPLIT | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
+     sv.SV_VARIANT_FUSED | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_FUSED | sv.SV_TAIL_ITEMS],
+    ids=["split-per-request", "split-items", "fused-per-request", "fused-items"])
 
 
 @VARIANTS
@@ -69,15 +73,15 @@ def test_near_tie_rate_below_1e4_of_rows(sv, name, variant):
 
 
 def test_full_size_is_deterministic_and_variants_agree(sv):
+    # every launch structure and tail layout gives bit-identical outputs, run after run
     w = wl.make("b256", "cuda")
-    a = gpu_run(w, seed=3, variant=sv.SV_VARIANT_SPLIT)
-    b = gpu_run(w, seed=3, variant=sv.SV_VARIANT_SPLIT)
-    c = gpu_run(w, seed=3, variant=sv.SV_VARIANT_FUSED)
-    d = gpu_run(w, seed=3, variant=sv.SV_VARIANT_FUSED)
-    for k in a:
-        assert np.array_equal(a[k], b[k], equal_nan=True), k
-        assert np.array_equal(a[k], c[k], equal_nan=True), k
-        assert np.array_equal(c[k], d[k], equal_nan=True), k
+    runs = [gpu_run(w, seed=3, variant=v)
+            for v in (sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED,
+                      sv.SV_VARIANT_FUSED, sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
+                      sv.SV_VARIANT_FUSED | sv.SV_TAIL_ITEMS, sv.SV_VARIANT_AUTO)]
+    for r in runs[1:]:
+        for k in runs[0]:
+            assert np.array_equal(runs[0][k], r[k], equal_nan=True), k
 
 
 def test_accept_length_mean_is_plausible(sv):

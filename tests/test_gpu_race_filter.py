@@ -2,7 +2,9 @@
 token whose exact key reaches K0 - 1e-6 (the near-tie band) must survive the
 filter, and every survivor must satisfy the filter's inequality
     log2(o + 1/2) <= L(x) + 2,   L(x) = (z/T - lse_t - K0 + delta) log2(e) + 32,
-so that it keeps no more than its documented rounding slack allows.  Checked
+so that it keeps no more than its documented rounding slack allows.  The
+single-precision bound that screens survivors before their exact key must be
+at least the exact key (in log2 units) for every candidate, and close to it.  Checked
 on real rows for bonus and residual races, plain and saguaro, fp32 and bf16, T
 of 1 and 0.7, peaked rows, masked tokens and logits with a large offset, and
 for K0 at several depths of the key order."""
@@ -39,7 +41,7 @@ def probe(tmp_path_factory, sv):
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_float,
         ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
         ctypes.c_double, ctypes.c_double, ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_int,
-        ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.POINTER(ctypes.c_float)]
     return L
 
@@ -64,15 +66,16 @@ def _run(probe, zt, zq, T, kind, K0, V):
     keep = torch.full((V,), 7, dtype=torch.uint8, device="cuda")
     words = torch.zeros((V,), dtype=torch.int32, device="cuda")
     exact = torch.full((V,), float("nan"), dtype=torch.float64, device="cuda")
+    upper = torch.full((V,), float("nan"), dtype=torch.float32, device="cuda")
     cup = ctypes.c_float(0.0)
     rc = probe.race_filter_probe(zt.data_ptr(), zq.data_ptr(), V,
                                  0 if zt.dtype == torch.float32 else 1, T, lse_t, lse_q, ntop, top,
                                  ln_c, ln_Z, 12345, 3, 0 if kind == "bonus" else 1, K0,
                                  keep.data_ptr(), words.data_ptr(), exact.data_ptr(),
-                                 ctypes.byref(cup))
+                                 upper.data_ptr(), ctypes.byref(cup))
     assert rc == 0
     return (keep.cpu().numpy(), words.cpu().numpy().view(np.uint32).astype(np.float64),
-            exact.cpu().numpy(), lse_t, _as_f64(ht), cup.value)
+            exact.cpu().numpy(), lse_t, _as_f64(ht), cup.value, upper.cpu().numpy().astype(np.float64))
 
 
 def _rows(dtype, offset):
@@ -93,16 +96,27 @@ def test_word_filter_keeps_every_contender(probe, dtype, T, kind, offset):
     zt, zq, V = _rows(dtype, offset)
     T = float(np.float32(T))
     # K0 = -inf: every unmasked token survives, and the exact keys come back
-    keep, o, e, lse_t, z, cup = _run(probe, zt, zq, T, kind, float("-inf"), V)
+    keep, o, e, lse_t, z, cup, ub = _run(probe, zt, zq, T, kind, float("-inf"), V)
     assert cup == float("inf")
     live = np.isfinite(z)
     assert np.all(keep[live] == 1)
     assert np.all(keep <= 1)
+    # the survivor bound: never below the exact key; tight where the word is small
+    # (it bounds E by W, and E / W -> 1 as W -> 0: the filter's survivors) and the
+    # logits are of moderate size (its slack grows with |z|, and with a large offset
+    # and bf16 rounding p and q' nearly coincide, where log2(1 - q'/p) is steep)
+    cand = np.isfinite(e)
+    slack = ub[cand] - e[cand] * LOG2E
+    assert slack.min() >= 0.0, (slack.min(), int(np.flatnonzero(cand)[np.argmin(slack)]))
+    if offset == 0.0:
+        small = (o[cand] < 2.0 ** 24)
+        assert small.sum() > 0
+        assert np.median(slack[small]) < 0.01, np.median(slack[small])
     fin = np.sort(e[np.isfinite(e)])[::-1]
     assert fin.size >= 200  # bf16 with a large offset leaves few tokens with p > q
     for depth in (0, 1, 9, 99, fin.size // 2):
         K0 = float(fin[depth])
-        keep, o2, e2, _, _, cup = _run(probe, zt, zq, T, kind, K0, V)
+        keep, o2, e2, _, _, cup, _ = _run(probe, zt, zq, T, kind, K0, V)
         assert np.array_equal(o2, o) and np.array_equal(np.isnan(e2), np.isnan(e))
         assert math.isfinite(cup)
         # safe: every token within the near-tie band of K0 (or above it) is kept
