@@ -1,6 +1,8 @@
 // row_stats.cu -- the first kernel of the split path: the per-row statistics
 // pass (stats_device.cuh) on a persistent grid of warps, each item one warp's
-// 8 KiB segment of a row.
+// 8 KiB segment of a row.  Three CTAs of 8 warps per multiprocessor (at most 85
+// registers a thread): the 24 warps keep about 192 KiB of loads in flight per
+// multiprocessor, which the pass needs to stream at the HBM rate.
 #include "stats_device.cuh"
 
 namespace sv {
@@ -8,7 +10,7 @@ namespace sv {
 namespace {
 
 template <int DT>
-__global__ void __launch_bounds__(kThreads) row_stats_kernel(VerifyArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) row_stats_kernel(VerifyArgs a) {
   stats_pass<DT>(a, blockIdx.x * kWarps + (threadIdx.x >> 5), gridDim.x * kWarps);
 }
 
