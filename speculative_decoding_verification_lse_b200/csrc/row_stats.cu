@@ -12,6 +12,7 @@ namespace {
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 3) row_stats_kernel(VerifyArgs a) {
   stats_pass<DT>(a, blockIdx.x * kWarps + (threadIdx.x >> 5), gridDim.x * kWarps);
+  allow_next_kernel();
 }
 
 }  // namespace

@@ -199,6 +199,18 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   return v;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation waits here until the kernel before it on the stream has
+// completed and its writes are visible (it may be resident and set up before).
+__device__ __forceinline__ void wait_for_previous_kernel() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel on the stream (if launched for it) get resident now.
+__device__ __forceinline__ void allow_next_kernel() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // bf16 halves of a 32-bit word as floats (exact widening).
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

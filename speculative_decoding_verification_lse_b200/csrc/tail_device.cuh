@@ -74,7 +74,8 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
   }
 
   // the reference key, from the segment holding the sampled row's largest logit
-  const RaceStream R = race_stream(a.seed, S.rd.g);
+  // (the request's Philox stream from kernel arguments, the same on every thread)
+  const RaceStream R = race_stream(a.seed, a.request_offset + (uint32_t)b);
   const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
   if (lane == 0) S.key[warp] = kw;
   if (threadIdx.x == 0) S.k0 = ordered_u64(-INFINITY);

@@ -2,27 +2,35 @@
 // (tail_device.cuh): either one CTA per request for everything, or the accept
 // scan (one CTA per request) followed by the race (one warp per request and
 // segment of the sampled row).
+#include <cstring>
+
 #include "tail_device.cuh"
 
 namespace sv {
 
 namespace {
 
+// Each kernel starts by waiting for the kernel before it (they are launched
+// as programmatic dependents, so they can be resident while it drains).
 template <int DT>
 __global__ void __launch_bounds__(kThreads) scan_kernel(VerifyArgs a) {
   __shared__ TailShared S;
+  wait_for_previous_kernel();
   scan_cta<DT>(a, (int)blockIdx.x, S);
+  allow_next_kernel();
 }
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) request_kernel(VerifyArgs a) {
   __shared__ TailShared S;
+  wait_for_previous_kernel();
   tail_request<DT>(a, (int)blockIdx.x, S);
 }
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) race_kernel(VerifyArgs a) {
   __shared__ RaceDesc s_rd[kWarps];
+  wait_for_previous_kernel();
   const int warp = threadIdx.x >> 5;
   const long long item = (long long)blockIdx.x * kWarps + warp;
   if (item >= (long long)a.B * a.nseg) return;
@@ -31,33 +39,41 @@ __global__ void __launch_bounds__(kThreads, 2) race_kernel(VerifyArgs a) {
 
 }  // namespace
 
+// Launch as a programmatic dependent of the kernel before it on the stream.
+template <typename K>
+cudaError_t launch_dependent(K kernel, unsigned grid, cudaStream_t s, const VerifyArgs& a) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s) {
   if (a.B == 0) return cudaSuccess;
-  if (a.dtype == kF32)
-    scan_kernel<kF32><<<a.B, kThreads, 0, s>>>(a);
-  else
-    scan_kernel<kBF16><<<a.B, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return a.dtype == kF32 ? launch_dependent(scan_kernel<kF32>, a.B, s, a)
+                         : launch_dependent(scan_kernel<kBF16>, a.B, s, a);
 }
 
 cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s) {
   if (a.B == 0) return cudaSuccess;
-  if (a.dtype == kF32)
-    request_kernel<kF32><<<a.B, kThreads, 0, s>>>(a);
-  else
-    request_kernel<kBF16><<<a.B, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return a.dtype == kF32 ? launch_dependent(request_kernel<kF32>, a.B, s, a)
+                         : launch_dependent(request_kernel<kBF16>, a.B, s, a);
 }
 
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s) {
   const long long items = (long long)a.B * a.nseg;
   if (items == 0) return cudaSuccess;
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
-  if (a.dtype == kF32)
-    race_kernel<kF32><<<grid, kThreads, 0, s>>>(a);
-  else
-    race_kernel<kBF16><<<grid, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return a.dtype == kF32 ? launch_dependent(race_kernel<kF32>, grid, s, a)
+                         : launch_dependent(race_kernel<kBF16>, grid, s, a);
 }
 
 }  // namespace sv
