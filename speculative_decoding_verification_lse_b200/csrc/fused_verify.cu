@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_kernel(VerifyArgs a) {
   __shared__ TailShared S;
   __shared__ RaceDesc s_rd[kWarps];
   const int warp = threadIdx.x >> 5;
-  stats_pass<DT>(a, blockIdx.x * kWarps + warp, gridDim.x * kWarps);
+  stats_pass<DT, true>(a, blockIdx.x * kWarps + warp, gridDim.x * kWarps);
   if (!grid_barrier(a, 0)) return fail_requests(a);
   if (a.per_request) {
     for (int b = blockIdx.x; b < a.B; b += gridDim.x) tail_request<DT>(a, b, S);

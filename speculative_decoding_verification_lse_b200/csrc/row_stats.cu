@@ -9,9 +9,9 @@ namespace sv {
 
 namespace {
 
-template <int DT>
+template <int DT, bool WITH_TOP>
 __global__ void __launch_bounds__(kThreads, 3) row_stats_kernel(VerifyArgs a) {
-  stats_pass<DT>(a, blockIdx.x * kWarps + (threadIdx.x >> 5), gridDim.x * kWarps);
+  stats_pass<DT, WITH_TOP>(a, blockIdx.x * kWarps + (threadIdx.x >> 5), gridDim.x * kWarps);
   allow_next_kernel();
 }
 
@@ -19,21 +19,31 @@ __global__ void __launch_bounds__(kThreads, 3) row_stats_kernel(VerifyArgs a) {
 
 int row_stats_blocks_per_sm(int dtype) {
   int n = 0;
-  cudaError_t e =
-      dtype == kF32 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, row_stats_kernel<kF32>, kThreads, 0)
-                    : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, row_stats_kernel<kBF16>, kThreads, 0);
+  cudaError_t e = dtype == kF32 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                                      &n, row_stats_kernel<kF32, true>, kThreads, 0)
+                                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                                      &n, row_stats_kernel<kBF16, true>, kThreads, 0);
   return e == cudaSuccess ? n : 0;
 }
 
+// Saguaro requests (the batch's mode, or any per-request mode) need the top lists.
 cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s, int grid) {
   const long long items = (long long)a.B * a.slots * a.nseg;
   if (items == 0) return cudaSuccess;
   const long long need = (items + kWarps - 1) / kWarps;
   if (grid > need) grid = (int)need;
-  if (a.dtype == kF32)
-    row_stats_kernel<kF32><<<grid, kThreads, 0, s>>>(a);
-  else
-    row_stats_kernel<kBF16><<<grid, kThreads, 0, s>>>(a);
+  const bool top = a.mode == kSaguaro || a.mode_per_req != nullptr;
+  if (a.dtype == kF32) {
+    if (top)
+      row_stats_kernel<kF32, true><<<grid, kThreads, 0, s>>>(a);
+    else
+      row_stats_kernel<kF32, false><<<grid, kThreads, 0, s>>>(a);
+  } else {
+    if (top)
+      row_stats_kernel<kBF16, true><<<grid, kThreads, 0, s>>>(a);
+    else
+      row_stats_kernel<kBF16, false><<<grid, kThreads, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

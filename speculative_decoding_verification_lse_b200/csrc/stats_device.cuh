@@ -97,8 +97,9 @@ __device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* ro
 // Statistics of one segment whose lane vectors are raw[0..kLaneVecs-1] (the
 // vectors seg*kSegVecs + lane + 32 j of the row), by one full warp.
 template <int DT, bool LSE, bool ARGMAX, bool TOP>
-__device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], int seg, float k2,
-                                             int topk, PartStat* out, TopPart* tout) {
+__device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], const char* row,
+                                             int seg, float k2, int topk, PartStat* out,
+                                             TopPart* tout) {
   constexpr int VEC = DT == kF32 ? 4 : 8;
   const int lane = threadIdx.x & 31;
   const int v0 = seg * kSegVecs + lane;
@@ -171,8 +172,39 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], int 
     idx_w = warp_min_int(idx_t);
   }
 
-  // ---- the k largest logits (value desc, index asc), saguaro draft rows
+  // ---- the k largest logits (value desc, index asc), saguaro draft rows.
+  // The k largest lane maxima are k distinct elements, so every element of the
+  // segment's top k is at least T, the k-th largest lane maximum.  A branch-free
+  // pass marks the lane's elements >= T (and > -inf) in a bit set (a compare and
+  // a funnel shift each); a small rolled loop then inserts the marked ones (few,
+  // unless many values tie) into the lane's sorted list, re-reading each from
+  // the row, in index order so that ties keep the lower index.  An element of
+  // the segment's top k is in its own lane's top k, which the list keeps.
   if (TOP) {
+    float T = -INFINITY;
+    {
+      unsigned long long mine = value_index_key(m_t, lane);
+      for (int r = 0; r < topk; ++r) {
+        const unsigned long long win = warp_max_u64(mine);
+        T = key_value(win);
+        if (mine == win) mine = 0ull;  // each lane maximum counts once
+      }
+    }
+    constexpr int NW = kLaneVecs * VEC / 32;
+    uint32_t mark[NW];
+#pragma unroll
+    for (int w = 0; w < NW; ++w) mark[w] = 0u;
+#pragma unroll
+    for (int j = 0; j < kLaneVecs; ++j)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const int t = j * VEC + e;
+        // -inf is never kept, so padding past the row's end (-inf) is never marked
+        // and every marked element lies inside the row
+        const float z = elem<DT>(raw[j], e);
+        const uint32_t hit = (z >= T && z > -INFINITY) ? 0x80000000u : 0u;
+        mark[t >> 5] = __funnelshift_l(hit, mark[t >> 5], 1);
+      }
     float tv[kMaxTopK];
     int ti[kMaxTopK];
 #pragma unroll
@@ -180,16 +212,22 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], int 
       tv[s] = -INFINITY;
       ti[s] = INT_MAX;
     }
+#pragma unroll 1
+    for (int w = 0; w < NW; ++w) {
+      uint32_t m = mark[0];
 #pragma unroll
-    for (int j = 0; j < kLaneVecs; ++j)
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        const float z = elem<DT>(raw[j], e);
+      for (int u = 1; u < NW; ++u)
+        if (u == w) m = mark[u];
+      while (m) {
+        const int tb = __clz((int)m);  // bit 31 - tb: element 32 w + tb of the lane
+        m &= ~(0x80000000u >> tb);
+        const int t = 32 * w + tb;
+        const int x = (v0 + 32 * (t / VEC)) * VEC + t % VEC;
+        const float z = DT == kF32 ? ((const float*)row)[x]
+                                   : __uint_as_float((uint32_t)((const uint16_t*)row)[x] << 16);
         if (z > tv[kMaxTopK - 1]) {
-          // elements arrive in increasing index order, so an equal value stays
-          // below the earlier (lower-index) one: strict comparisons throughout
           tv[kMaxTopK - 1] = z;
-          ti[kMaxTopK - 1] = (v0 + 32 * j) * VEC + e;
+          ti[kMaxTopK - 1] = x;
 #pragma unroll
           for (int s = kMaxTopK - 1; s > 0; --s) {
             if (tv[s] > tv[s - 1]) {
@@ -203,6 +241,7 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], int 
           }
         }
       }
+    }
     int h = 0;
     for (int r = 0; r < topk; ++r) {
       float hv = -INFINITY;
@@ -239,7 +278,15 @@ __device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* r
                                               float k2, int topk, PartStat* out, TopPart* tout) {
   uint4 raw[kLaneVecs];
   load_segment<DT>(a, row, seg, raw);
-  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, seg, k2, topk, out, tout);
+  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, row, seg, k2, topk, out, tout);
+}
+
+// The statistics of a saguaro draft-row segment (with its top list), compiled
+// on its own so that the common path keeps its registers.
+template <int DT>
+__device__ __noinline__ void stats_segment_top(const VerifyArgs& a, const char* row, int seg,
+                                               float k2, int topk, PartStat* out, TopPart* tout) {
+  stats_segment<DT, true, false, true>(a, row, seg, k2, topk, out, tout);
 }
 
 // Whether row `slot` of a request with parameters rp is read by the rule.
@@ -251,7 +298,11 @@ __device__ __forceinline__ bool row_needed(const VerifyArgs& a, int slot, const 
 }
 
 // Statistics of segment `seg` of row `slot` of request b (one full warp).
-template <int DT>
+// WITH_TOP: the batch may hold saguaro requests (their draft rows need the top
+// list); the launcher compiles the pass both ways and picks by the batch, so
+// the common path carries no code for it.  A saguaro row met without it is a
+// launcher error, reported as a bad parameter.
+template <int DT, bool WITH_TOP>
 __device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot, int seg,
                                            const ReqParams& rp) {
   const bool is_target = slot <= a.D_max;
@@ -265,8 +316,12 @@ __device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot,
     else
       stats_segment<DT, true, false, false>(a, row, seg, k2, 0, out, nullptr);
   } else if (rp.mode == kSaguaro) {
-    TopPart* tout = a.tpart + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * a.nseg + seg;
-    stats_segment<DT, true, false, true>(a, row, seg, k2, a.saguaro_k, out, tout);
+    if (WITH_TOP) {
+      TopPart* tout = a.tpart + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * a.nseg + seg;
+      stats_segment_top<DT>(a, row, seg, k2, a.saguaro_k, out, tout);
+    } else if ((threadIdx.x & 31) == 0) {
+      atomicOr(a.status, kFlagBadParam);
+    }
   } else {
     stats_segment<DT, true, false, false>(a, row, seg, k2, 0, out, nullptr);
   }
@@ -309,7 +364,7 @@ struct ItemWalker {
 // w0, w0 + W, w0 + 2W, ... in request-major order, so that at any moment the
 // device streams one contiguous stretch of the logits.  Rows the rule does not
 // read are skipped (parameter errors are reported by the scan).
-template <int DT>
+template <int DT, bool WITH_TOP>
 __device__ __forceinline__ void stats_pass(const VerifyArgs& a, unsigned w0, unsigned W) {
   const unsigned total = (unsigned)a.B * (unsigned)a.slots * (unsigned)a.nseg;
   if (w0 >= total) return;
@@ -318,7 +373,7 @@ __device__ __forceinline__ void stats_pass(const VerifyArgs& a, unsigned w0, uns
   for (unsigned i = w0; i < total; i += W, it.advance(a)) {
     const ReqParams rp = load_req(a, it.b);
     if (!row_needed(a, it.slot, rp)) continue;
-    stats_item<DT>(a, it.b, it.slot, it.seg, rp);
+    stats_item<DT, WITH_TOP>(a, it.b, it.slot, it.seg, rp);
   }
 }
 

@@ -66,6 +66,24 @@ def test_row_D_with_zero_and_nan_padding(sv, variant):
     assert sv.sv_get_device_status() == 0
 
 
+@VARIANTS
+def test_saguaro_top_k_with_many_ties(sv, variant):
+    # draft logits on a coarse grid (many equal values in and across lanes and
+    # segments), plus copies of each row's maximum at spread-out positions, so
+    # the top-k selection must break ties by the lowest index exactly as the oracle
+    w = make_random(8, 4, 20000 + 37, seed=11, mode=2)
+    q = torch.round(w.draft.float() * 2.0) / 2.0
+    for b in range(w.B):
+        for d in range(w.D_max):
+            m = q[b, d].max()
+            for x in (5, 4096 + 31, 8191, 12000 + d, 19999):
+                q[b, d, x] = m
+    w.draft.copy_(q.to(w.draft.dtype))
+    got = gpu_run(w, variant=variant)
+    assert np.all((got["flags"] & sv.SV_FLAG_ERRORS) == 0)
+    compare(w, got, oracle_on(w))
+
+
 def test_identical_target_and_draft_accept_everything(sv):
     w = make_random(16, 6, 20000, seed=4)
     w.draft.copy_(w.target[:, :6])
