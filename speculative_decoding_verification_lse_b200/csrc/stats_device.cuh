@@ -98,7 +98,7 @@ __device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* ro
 // vectors seg*kSegVecs + lane + 32 j of the row), by one full warp.
 template <int DT, bool LSE, bool ARGMAX, bool TOP>
 __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], const char* row,
-                                             int seg, float k2, int topk, PartStat* out,
+                                             int V, int seg, float k2, int topk, PartStat* out,
                                              TopPart* tout) {
   constexpr int VEC = DT == kF32 ? 4 : 8;
   const int lane = threadIdx.x & 31;
@@ -175,11 +175,11 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
   // ---- the k largest logits (value desc, index asc), saguaro draft rows.
   // The k largest lane maxima are k distinct elements, so every element of the
   // segment's top k is at least T, the k-th largest lane maximum.  A branch-free
-  // pass marks the lane's elements >= T (and > -inf) in a bit set (a compare and
-  // a funnel shift each); a small rolled loop then inserts the marked ones (few,
-  // unless many values tie) into the lane's sorted list, re-reading each from
-  // the row, in index order so that ties keep the lower index.  An element of
-  // the segment's top k is in its own lane's top k, which the list keeps.
+  // pass marks the lane's 16-byte vectors whose largest element reaches T (and
+  // is above -inf); a small rolled loop then re-reads the marked vectors (few,
+  // unless many values tie) and inserts their elements >= T into the lane's
+  // sorted list, in index order so that ties keep the lower index.  An element
+  // of the segment's top k is in its own lane's top k, which the list keeps.
   if (TOP) {
     float T = -INFINITY;
     {
@@ -190,21 +190,22 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
         if (mine == win) mine = 0ull;  // each lane maximum counts once
       }
     }
-    constexpr int NW = kLaneVecs * VEC / 32;
-    uint32_t mark[NW];
+    uint32_t mark = 0u;  // bit 31 - j: vector j of the lane
 #pragma unroll
-    for (int w = 0; w < NW; ++w) mark[w] = 0u;
-#pragma unroll
-    for (int j = 0; j < kLaneVecs; ++j)
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        const int t = j * VEC + e;
-        // -inf is never kept, so padding past the row's end (-inf) is never marked
-        // and every marked element lies inside the row
-        const float z = elem<DT>(raw[j], e);
-        const uint32_t hit = (z >= T && z > -INFINITY) ? 0x80000000u : 0u;
-        mark[t >> 5] = __funnelshift_l(hit, mark[t >> 5], 1);
+    for (int j = 0; j < kLaneVecs; ++j) {
+      float vm;
+      if (DT == kBF16) {
+        const __nv_bfloat162 p = __hmax2(__hmax2(as_bf2(raw[j].x), as_bf2(raw[j].y)),
+                                         __hmax2(as_bf2(raw[j].z), as_bf2(raw[j].w)));
+        vm = fmaxf(__low2float(p), __high2float(p));
+      } else {
+        vm = fmaxf(fmaxf(elem<DT>(raw[j], 0), elem<DT>(raw[j], 1)),
+                   fmaxf(elem<DT>(raw[j], 2), elem<DT>(raw[j], 3)));
       }
+      const uint32_t hit = (vm >= T && vm > -INFINITY) ? 0x80000000u : 0u;
+      mark = __funnelshift_l(hit, mark, 1);
+    }
+    mark <<= (32 - kLaneVecs);
     float tv[kMaxTopK];
     int ti[kMaxTopK];
 #pragma unroll
@@ -212,20 +213,16 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
       tv[s] = -INFINITY;
       ti[s] = INT_MAX;
     }
+    while (mark) {
+      const int j = __clz((int)mark);
+      mark &= ~(0x80000000u >> j);
 #pragma unroll 1
-    for (int w = 0; w < NW; ++w) {
-      uint32_t m = mark[0];
-#pragma unroll
-      for (int u = 1; u < NW; ++u)
-        if (u == w) m = mark[u];
-      while (m) {
-        const int tb = __clz((int)m);  // bit 31 - tb: element 32 w + tb of the lane
-        m &= ~(0x80000000u >> tb);
-        const int t = 32 * w + tb;
-        const int x = (v0 + 32 * (t / VEC)) * VEC + t % VEC;
+      for (int e = 0; e < VEC; ++e) {
+        const int x = (v0 + 32 * j) * VEC + e;
+        if (x >= V) break;
         const float z = DT == kF32 ? ((const float*)row)[x]
                                    : __uint_as_float((uint32_t)((const uint16_t*)row)[x] << 16);
-        if (z > tv[kMaxTopK - 1]) {
+        if (z >= T && z > tv[kMaxTopK - 1]) {
           tv[kMaxTopK - 1] = z;
           ti[kMaxTopK - 1] = x;
 #pragma unroll
@@ -278,7 +275,7 @@ __device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* r
                                               float k2, int topk, PartStat* out, TopPart* tout) {
   uint4 raw[kLaneVecs];
   load_segment<DT>(a, row, seg, raw);
-  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, row, seg, k2, topk, out, tout);
+  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, row, a.V, seg, k2, topk, out, tout);
 }
 
 // The statistics of a saguaro draft-row segment (with its top list), compiled
