@@ -303,13 +303,23 @@ def run_ours(args):
         o_t = torch.empty(out["tokens"].shape, dtype=torch.int32, pin_memory=True)
         o_a = torch.empty(out["accept_len"].shape, dtype=torch.int32, pin_memory=True)
         d_t, d_q, d_x = torch.empty_like(w.target), torch.empty_like(w.draft), torch.empty_like(w.tokens)
+        # the per-request inputs (ragged draft lengths, modes, temperatures) travel too
+        small = {k: getattr(w, k) for k in ("row_D", "temperature_per_req", "mode_per_req")
+                 if getattr(w, k) is not None}
+        h_small = {k: v.cpu().pin_memory() for k, v in small.items()}
+        d_small = {k: torch.empty_like(v) for k, v in small.items()}
 
         def e2e_step(i):
             d_t.copy_(h_t, non_blocking=True)
             d_q.copy_(h_q, non_blocking=True)
             d_x.copy_(h_x, non_blocking=True)
-            sv.verify(d_t, d_q, d_x, None, temperature=w.temperature, mode=w.mode, seed=5000 + i,
-                      request_offset=offset, variant=variant, stream=stream, out=out)
+            for k in d_small:
+                d_small[k].copy_(h_small[k], non_blocking=True)
+            sv.verify(d_t, d_q, d_x, d_small.get("row_D"), temperature=w.temperature, mode=w.mode,
+                      seed=5000 + i, temperature_per_req=d_small.get("temperature_per_req"),
+                      mode_per_req=d_small.get("mode_per_req"), saguaro_k=w.saguaro_k,
+                      saguaro_c=w.saguaro_c, request_offset=offset, variant=variant, stream=stream,
+                      out=out)
             o_t.copy_(out["tokens"], non_blocking=True)
             o_a.copy_(out["accept_len"], non_blocking=True)
 
@@ -323,7 +333,8 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), dev)
-        h2d = h_t.numel() * h_t.element_size() + h_q.numel() * h_q.element_size() + h_x.numel() * 4
+        h2d = (h_t.numel() * h_t.element_size() + h_q.numel() * h_q.element_size() + h_x.numel() * 4
+               + sum(v.numel() * v.element_size() for v in h_small.values()))
         d2h = o_t.numel() * 4 + o_a.numel() * 4
         e2e = {"value": w.verified_rows() * args.e2e_steps * world / (ems / 1e3), "unit": "rows/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
