@@ -225,6 +225,7 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.best_key = (unsigned long long*)((char*)ws + L.best_key);
   a.rorder = (unsigned short*)((char*)ws + L.rorder);
   a.barrier = (unsigned int*)((char*)ws + L.barrier);
+  a.ticket = (unsigned int*)((char*)ws + L.ticket);
   a.seed = seed;
   a.B = B;
   a.D_max = D_max;
@@ -254,8 +255,12 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     return SV_OK;
   }
+  const bool tickets = row_stats_tickets(a, grid);
+  if (tickets && (e = cudaMemsetAsync(a.ticket, 0, 8 * 128, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync(ticket)");
   if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  if ((e = launch_row_stats(a, s, grid)) != cudaSuccess) return cuda_fail(e, "row statistics launch");
+  if ((e = launch_row_stats(a, s, grid, tickets)) != cudaSuccess)
+    return cuda_fail(e, "row statistics launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if (a.per_request) {
     if ((e = launch_requests(a, s)) != cudaSuccess) return cuda_fail(e, "scan and race launch");

@@ -122,6 +122,7 @@ struct VerifyArgs {
   unsigned long long* best_key;  // [B] best exact race key so far, ordered bits (set by the scan)
   unsigned short* rorder;  // [B, nseg] race segments by descending largest logit (set by the scan)
   unsigned int* barrier;   // fused kernel: two grid barriers' counters (zero at launch)
+  unsigned int* ticket;    // statistics kernel with tickets: 8 counters, 32 words apart (zero at launch)
   uint64_t seed;
   int B, D_max, V, dtype;
   int nvec, nseg, slots;
@@ -136,7 +137,7 @@ struct VerifyArgs {
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
 // [zero, total) must read zero when a fused launch starts.
 struct WsLayout {
-  size_t pstat, tpart, rdesc, rpart, rcount, best_key, rorder, zero, barrier, total;
+  size_t pstat, tpart, rdesc, rpart, rcount, best_key, rorder, zero, barrier, ticket, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -172,6 +173,8 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   L.zero = off;
   L.barrier = off;
   off = align_up(off + 2 * sizeof(unsigned int), 256);
+  L.ticket = off;
+  off = align_up(off + 8 * 128, 256);  // eight counters, one 128-byte line each
   L.total = off;
   return L;
 }
@@ -303,7 +306,8 @@ __device__ __forceinline__ float load_logit(const VerifyArgs& a, const char* row
 
 // Host-side launchers (one per kernel file), called from the C ABI.
 namespace sv {
-cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s, int grid);
+cudaError_t launch_row_stats(const VerifyArgs& a, cudaStream_t s, int grid, bool tickets);
+bool row_stats_tickets(const VerifyArgs& a, int grid);
 int row_stats_blocks_per_sm(int dtype);
 cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
