@@ -153,12 +153,10 @@ __device__ __forceinline__ float filter_offset(double K0, double lse_t) {
   return __double2float_ru(C + (64.0 + fabs(C)) * 0x1p-21 + 0x1p-20);
 }
 
-// Tokens per lane in a segment, and the 32-bit words of their flags.
+// Tokens per 16-byte vector.
 template <int DT>
 struct Lanes {
   static constexpr int VEC = DT == kF32 ? 4 : 8;
-  static constexpr int TOK = kLaneVecs * VEC;
-  static constexpr int WORDS = TOK / 32;
 };
 
 // The index of the most significant set bit of o, -1 for o = 0.
