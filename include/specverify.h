@@ -51,7 +51,10 @@
  *   - All array arguments are DEVICE pointers on the current CUDA device,
  *     row-major and contiguous; the caller owns every buffer.
  *   - Calls are asynchronous on the stream (sv_params.stream, default: the
- *     legacy default stream) and never synchronise.
+ *     legacy default stream) and never synchronise.  Calls without their own
+ *     workspace share the library's cached one on their device, so they must
+ *     not overlap on the GPU: run them on one stream, or pass each its own
+ *     workspace (sv_params.workspace).
  *   - Host-detectable argument errors return a negative code, launch nothing
  *     and leave the outputs untouched; sv_last_error() describes the error.
  *   - Errors found on the device (a draft token outside [0, V), row_D[b]

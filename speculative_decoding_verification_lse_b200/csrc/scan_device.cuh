@@ -137,26 +137,52 @@ __device__ inline void merge_row_into(const VerifyArgs& a, int b, int slot, cons
   if ((threadIdx.x & 31) == 0) *dst = rr;
 }
 
+// The scan's per-position inputs, which do not depend on the merged rows: lane
+// d < D_b holds draft token x_d and, for a sampling request, its target and
+// draft logits and its accept word.  Loaded by the scanning warp before it
+// merges rows, so that their latency overlaps the merge.
+struct ScanInputs {
+  int x;
+  float zt, zq;
+  uint32_t uw;
+  uint32_t err;
+};
+
+__device__ __forceinline__ ScanInputs scan_inputs(const VerifyArgs& a, int b, const ReqParams& rp) {
+  const int lane = threadIdx.x & 31;
+  ScanInputs in;
+  in.x = -1;
+  in.zt = in.zq = 0.0f;
+  in.uw = 0u;
+  in.err = rp.err;
+  if (!rp.err && lane < rp.Db) {
+    in.x = a.tokens[(size_t)b * a.D_max + lane];
+    if (in.x < 0 || in.x >= a.V) {
+      in.err |= kFlagBadToken;
+    } else if (rp.mode != kGreedy) {
+      in.zt = load_logit(a, row_base(a, b, lane), in.x);
+      in.zq = load_logit(a, row_base(a, b, a.D_max + 1 + lane), in.x);
+      in.uw = accept_word(a.seed, a.request_offset + (uint32_t)b, (uint32_t)lane);
+    }
+  }
+  return in;
+}
+
 // The accept scan of request b by one full warp, once every row it reads has
-// been merged into rows (2*D_max+1 entries of shared memory).  Writes the
+// been merged into rows (2*D_max+1 entries of shared memory); in: the warp's
+// scan_inputs.  Writes the
 // outputs (slot n too for greedy), the flags and the row LSEs, and lane 0
 // writes the race description to *rd; returns the race kind (same on all
 // lanes).
-__device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* rows, RaceDesc* rd) {
+__device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* rows, RaceDesc* rd,
+                                   const ScanInputs& in) {
   const int lane = threadIdx.x & 31;
   const int Dm = a.D_max;
   const ReqParams rp = load_req(a, b);
   const uint32_t g = a.request_offset + (uint32_t)b;
   int32_t* ot = a.out_tokens + (size_t)b * (Dm + 1);
-  uint32_t err = rp.err;
-
-  // draft tokens of the tested positions
-  int x = -1;
-  if (!err && lane < rp.Db) {
-    x = a.tokens[(size_t)b * Dm + lane];
-    if (x < 0 || x >= a.V) err |= kFlagBadToken;
-  }
-  err = __reduce_or_sync(0xFFFFFFFFu, err);
+  const int x = in.x;
+  uint32_t err = __reduce_or_sync(0xFFFFFFFFu, in.err);
 
   const bool greedy = rp.mode == kGreedy;
   const bool saguaro = rp.mode == kSaguaro;
@@ -191,11 +217,9 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* row
     if (greedy) {
       accept = (x == rows[lane].argmax);
     } else {
-      const char* trow = row_base(a, b, lane);
-      const char* qrow = row_base(a, b, Dm + 1 + lane);
       const RowRes& rq = rows[Dm + 1 + lane];
-      const double lp = (double)load_logit(a, trow, x) / Td - rows[lane].lse;
-      double lq = (double)load_logit(a, qrow, x) / Td - rq.lse;
+      const double lp = (double)in.zt / Td - rows[lane].lse;
+      double lq = (double)in.zq / Td - rq.lse;
       if (saguaro && lq != -INFINITY) {
         bool in_k = false;
         for (int i = 0; i < rq.ntop; ++i) in_k |= (rq.top[i] == x);
@@ -208,7 +232,7 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* row
         acc = 1.0;
       else
         acc = fmin(1.0, exp(lp - lq));
-      const double u = (double)(accept_word(a.seed, g, (uint32_t)lane) >> 8) * 0x1p-24;
+      const double u = (double)(in.uw >> 8) * 0x1p-24;
       accept = u < acc;
       near = fabs(u - acc) < 1e-5;
     }

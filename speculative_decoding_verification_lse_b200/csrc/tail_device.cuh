@@ -24,6 +24,7 @@ namespace sv {
 
 struct TailShared {
   RowRes rows[2 * kMaxDraft + 1];
+  ScanInputs in[32];
   RaceDesc rd;
   double key[kWarps];
   double best[kWarps], second[kWarps];
@@ -62,10 +63,12 @@ template <int DT>
 __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailShared& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const ReqParams rp = load_req(a, b);
+  // the scan's inputs by the last warp (the fewest rows to merge), during the merges
+  if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
   for (int slot = warp; slot < a.slots; slot += kWarps)
     if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
   __syncthreads();
-  if (warp == 0) scan_request(a, b, S.rows, &S.rd);
+  if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();
   const int kind = S.rd.kind;
   if (kind == kRaceNone) {
@@ -121,10 +124,12 @@ template <int DT>
 __device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const ReqParams rp = load_req(a, b);
+  // the scan's inputs by the last warp (the fewest rows to merge), during the merges
+  if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
   for (int slot = warp; slot < a.slots; slot += kWarps)
     if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
   __syncthreads();
-  if (warp == 0) scan_request(a, b, S.rows, &S.rd);
+  if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();
   const int kind = S.rd.kind;
   if (kind != kRaceNone) {
