@@ -356,6 +356,72 @@ __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceD
   return warp_combine(B);
 }
 
+// Segments seg0, seg0 + step, ... (below a.nseg) of the race, by one warp, as
+// one stream of 32-token groups: the next group loads while the current one is
+// filtered, across segment boundaries too.  At each boundary the warp raises
+// *shared (the request's best key so far, ordered bits, in shared memory) with
+// its own best and takes the largest of K0, its own best and *shared as the
+// reference key for the next segment.  Returns the combination of all the
+// segments' results (all lanes); otherwise as race_segment_in.
+template <int DT>
+__device__ __forceinline__ Best race_span_in(const VerifyArgs& a, const RaceDesc& rd,
+                                             const RaceStream& R, const char* trow,
+                                             const char* qrow, bool residual, int seg0, int step,
+                                             double K0, unsigned long long* shared) {
+  constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC, NG = kLaneVecs / QV;
+  const int lane = threadIdx.x & 31;
+  Best B{-INFINITY, -INFINITY, -1};
+  if (seg0 >= a.nseg) return B;
+  int seg = seg0;
+  double K = fmax(K0, from_ordered_u64(*(volatile unsigned long long*)shared));
+  if (!(K > -INFINITY)) K = lane_max_key<DT>(a, rd, trow, qrow, residual, seg);
+  float cup = filter_offset(K, rd.lse_t);
+  float thr2 = K > -INFINITY ? __double2float_rd((K - kRaceBand) * 1.4426950408889634 - 1e-5)
+                             : -INFINITY;
+  uint4 cur[QV], nxt[QV];
+  load_part<DT>(a, trow, seg, 0, cur);
+  int gi = 0;
+#pragma unroll 1
+  for (;;) {
+    const bool seg_end = gi + 1 == NG;
+    const int nseg_ = seg_end ? seg + step : seg;
+    const int ngi = seg_end ? 0 : gi + 1;
+    const bool more = nseg_ < a.nseg;
+    if (more) load_part<DT>(a, trow, nseg_, ngi * QV, nxt);
+    const int v0 = seg * kSegVecs + lane;
+    uint32_t keep = ~word_filter<DT>(cur, gi * QV, R, v0, rd.k2, cup);
+    // exact keys of the survivors, one token per lane at a time
+    while (__any_sync(0xFFFFFFFFu, keep != 0u)) {
+      if (keep) {
+        const int t = __clz((int)keep);
+        keep &= ~(0x80000000u >> t);
+        const int x = (v0 + 32 * (gi * QV + t / VEC)) * VEC + t % VEC;
+        if (x < a.V && key2_upper(a, rd, trow, qrow, residual, x) >= thr2)
+          offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
+      }
+    }
+    if (!more) break;
+    if (seg_end) {
+      // share the warp's best so far and refresh the reference key
+      double wb = B.best;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wb = fmax(wb, __shfl_xor_sync(0xFFFFFFFFu, wb, o));
+      if (lane == 0 && wb > -INFINITY) atomicMax(shared, ordered_u64(wb));
+      __syncwarp();
+      K = fmax(K, fmax(wb, from_ordered_u64(*(volatile unsigned long long*)shared)));
+      if (!(K > -INFINITY)) K = lane_max_key<DT>(a, rd, trow, qrow, residual, nseg_);
+      cup = filter_offset(K, rd.lse_t);
+      thr2 = K > -INFINITY ? __double2float_rd((K - kRaceBand) * 1.4426950408889634 - 1e-5)
+                           : -INFINITY;
+      seg = nseg_;
+    }
+    gi = ngi;
+#pragma unroll
+    for (int j = 0; j < QV; ++j) cur[j] = nxt[j];
+  }
+  return warp_combine(B);
+}
+
 template <int DT>
 __device__ __noinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
                                           const char* trow, const char* qrow, bool residual,

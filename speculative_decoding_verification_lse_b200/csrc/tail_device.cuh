@@ -87,18 +87,11 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
 #pragma unroll
   for (int w = 1; w < kWarps; ++w) K0 = fmax(K0, S.key[w]);
 
-  // the race, warp w taking segments w, w + 8, ...
+  // the race, warp w taking segments w, w + 8, ... as one stream
   const bool residual = kind == kRaceResidual;
   const char* trow = row_base(a, b, S.rd.n);
   const char* qrow = residual ? row_base(a, b, a.D_max + 1 + S.rd.n) : nullptr;
-  Best B{-INFINITY, -INFINITY, -1};
-  for (int seg = warp; seg < a.nseg; seg += kWarps) {
-    const double K = fmax(K0, from_ordered_u64(*(volatile unsigned long long*)&S.k0));
-    const Best sb = race_segment_in<DT>(a, S.rd, R, trow, qrow, residual, seg, K,
-                                        filter_offset(K, S.rd.lse_t));
-    if (lane == 0 && sb.idx >= 0) atomicMax(&S.k0, ordered_u64(sb.best));
-    B = combine(B, sb);
-  }
+  const Best B = race_span_in<DT>(a, S.rd, R, trow, qrow, residual, warp, kWarps, K0, &S.k0);
   if (lane == 0) {
     S.best[warp] = B.best;
     S.second[warp] = B.second;
