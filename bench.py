@@ -117,9 +117,10 @@ def tail_items(w, sms):
     return w.B < sms and w.B * nseg > sms
 
 
-def traffic_record(kernel_name, sources):
+def traffic_record(kernel_name, sources, alg_bytes):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel source and on a launch of the same algorithmic bytes (the
+    same workload), else None."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
@@ -132,7 +133,7 @@ def traffic_record(kernel_name, sources):
     with open(path) as f:
         for line in f:
             parts = line.split()
-            if len(parts) >= 4 and parts[0] == kernel_name:
+            if len(parts) >= 5 and parts[0] == kernel_name and int(parts[4]) == alg_bytes:
                 rec[parts[1]] = (float(parts[2]), int(parts[3]))  # sha -> (bytes per launch, units)
     return rec.get(sha)
 
@@ -363,7 +364,7 @@ def run_ours(args):
                     "speculative_decoding_verification_lse_b200/csrc/stats_device.cuh",
                     "speculative_decoding_verification_lse_b200/csrc/sv_common.cuh"]
         achieved = kbytes / (k_ms / 1e3) / 1e9
-        tr = traffic_record(kname, ksrc)
+        tr = traffic_record(kname, ksrc, kbytes)
         line = {
             "metric": METRIC,
             "value": value,
