@@ -25,6 +25,7 @@ namespace sv {
 struct TailShared {
   RowRes rows[2 * kMaxDraft + 1];
   ScanInputs in[32];
+  float segm[kThreads];  // the sampled row's segment maxima (race order)
   RaceDesc rd;
   double key[kWarps];
   double best[kWarps], second[kWarps];
@@ -129,24 +130,30 @@ __device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared&
     // the reference key: each warp ranks a share of the segment holding the
     // sampled row's largest logit and takes the exact key of its best token
     const RaceStream R = race_stream(a.seed, S.rd.g);
+    // the sampled row's segment maxima, for the race order, load while the
+    // reference key is searched
+    const bool ranked = a.nseg <= kThreads;
+    float m = 0.0f;
+    if (ranked && threadIdx.x < a.nseg)
+      m = __ldcg(&a.pstat[((size_t)b * a.slots + S.rd.n) * a.nseg + threadIdx.x].m);
     const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
     if (lane == 0) S.key[warp] = kw;
+    if (ranked && threadIdx.x < a.nseg) S.segm[threadIdx.x] = m;
+    __syncthreads();
     // the race order: rank of each segment by its largest logit (ties: lower
     // index first); rows of more than kThreads segments keep index order
     for (int sg = threadIdx.x; sg < a.nseg; sg += kThreads) {
       int rank = sg;
-      if (a.nseg <= kThreads) {
-        const PartStat* ps = a.pstat + ((size_t)b * a.slots + S.rd.n) * a.nseg;
-        const float m = __ldcg(&ps[sg].m);
+      if (ranked) {
+        const float ms = S.segm[sg];
         rank = 0;
         for (int j = 0; j < a.nseg; ++j) {
-          const float mj = __ldcg(&ps[j].m);
-          rank += (mj > m || (mj == m && j < sg)) ? 1 : 0;
+          const float mj = S.segm[j];
+          rank += (mj > ms || (mj == ms && j < sg)) ? 1 : 0;
         }
       }
       a.rorder[(size_t)b * a.nseg + rank] = (unsigned short)sg;
     }
-    __syncthreads();
     if (warp == 0) {
       double K0 = lane < kWarps ? S.key[lane] : -INFINITY;
 #pragma unroll
