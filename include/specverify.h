@@ -98,7 +98,8 @@ enum { SV_OK = 0, SV_ERR_INVALID_ARG = -1, SV_ERR_UNSUPPORTED = -2, SV_ERR_CUDA 
  * PER_REQUEST otherwise):
  *   SV_TAIL_PER_REQUEST: one CTA per request merges, scans and races it;
  *   SV_TAIL_ITEMS: one CTA per request merges and scans, then one warp per
- *     (request, segment of the sampled row) races. */
+ *     (request, segment of the sampled row) races -- per half segment while
+ *     those items fit in one wave of the device's resident warps. */
 enum { SV_VARIANT_AUTO = 0, SV_VARIANT_SPLIT = 1, SV_VARIANT_FUSED = 2 };
 enum { SV_TAIL_PER_REQUEST = 1 << 4, SV_TAIL_ITEMS = 1 << 5 };
 

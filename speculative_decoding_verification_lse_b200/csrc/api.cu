@@ -239,6 +239,8 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   // segments to spread; else the scan, then race items over the whole GPU
   const bool spread = B < sms && (long long)B * nseg > sms;
   a.per_request = tail_bits == SV_TAIL_PER_REQUEST ? 1 : tail_bits == SV_TAIL_ITEMS ? 0 : (spread ? 0 : 1);
+  // the fused kernel takes whole segments; the split path cuts them while one wave holds them
+  a.rsplit = fused || a.per_request ? 1 : race_split(B, nseg, dtype, sms);
   a.temperature = temperature;
   a.saguaro_k = k;
   a.saguaro_c = c;

@@ -5,8 +5,8 @@
 // barrier, and then does what the split path's later kernels do
 // (tail_device.cuh), in the same layout: either each CTA takes whole requests
 // (blockIdx.x, + gridDim.x, ...), or the CTAs take the accept scans, meet at a
-// second barrier, and the warps take the (request, segment) race items.  The
-// partial statistics are read back from L2.
+// second barrier, and the warps take the (request, segment) race items (whole
+// segments: a.rsplit is 1 here).  The partial statistics are read back from L2.
 //
 // The barriers are counters in the workspace, zero at launch.  Their waits are
 // bounded: a CTA that gives up sets SV_STATUS_TIMEOUT, writes -1 for its
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_kernel(VerifyArgs a) {
   }
   for (int b = blockIdx.x; b < a.B; b += gridDim.x) scan_cta<DT>(a, b, S);
   if (!grid_barrier(a, 1)) return fail_requests(a);
-  const long long items = (long long)a.B * a.nseg;
+  const long long items = (long long)a.B * a.nseg * a.rsplit;
   for (long long it = (long long)blockIdx.x * kWarps + warp; it < items; it += (long long)gridDim.x * kWarps)
     race_item<DT>(a, it, &s_rd[warp]);
 }

@@ -315,13 +315,16 @@ __device__ __noinline__ double lane_max_key(const VerifyArgs& a, const RaceDesc&
 // Philox stream.  The lane walks its part of the segment in groups of 32
 // tokens, loading the next group while it filters the current one, and takes
 // exact keys of a group's survivors (rare) right away, so the loop body stays
-// small enough for the instruction cache.
+// small enough for the instruction cache.  Only groups g0 .. g1 - 1 of the
+// lane's NG (g1 < 0: to the end) are raced, so that a segment can be split
+// into independent items.
 template <int DT>
 __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceDesc& rd,
                                                 const RaceStream& R, const char* trow,
                                                 const char* qrow, bool residual, int seg,
-                                                double K0, float cup) {
+                                                double K0, float cup, int g0 = 0, int g1 = -1) {
   constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC, NG = kLaneVecs / QV;
+  if (g1 < 0) g1 = NG;
   const int v0 = seg * kSegVecs + (threadIdx.x & 31);
   if (!(K0 > -INFINITY)) {
     K0 = lane_max_key<DT>(a, rd, trow, qrow, residual, seg);
@@ -333,10 +336,10 @@ __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceD
 
   Best B{-INFINITY, -INFINITY, -1};
   uint4 cur[QV], nxt[QV];
-  load_part<DT>(a, trow, seg, 0, cur);
+  load_part<DT>(a, trow, seg, g0 * QV, cur);
 #pragma unroll 1
-  for (int gi = 0; gi < NG; ++gi) {
-    if (gi + 1 < NG) load_part<DT>(a, trow, seg, (gi + 1) * QV, nxt);
+  for (int gi = g0; gi < g1; ++gi) {
+    if (gi + 1 < g1) load_part<DT>(a, trow, seg, (gi + 1) * QV, nxt);
     uint32_t keep = ~word_filter<DT>(cur, gi * QV, R, v0, rd.k2, cup);
     // exact keys of the survivors, one token per lane at a time
     while (__any_sync(0xFFFFFFFFu, keep != 0u)) {
@@ -348,7 +351,7 @@ __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceD
           offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
       }
     }
-    if (gi + 1 < NG) {
+    if (gi + 1 < g1) {
 #pragma unroll
       for (int j = 0; j < QV; ++j) cur[j] = nxt[j];
     }

@@ -24,6 +24,7 @@ constexpr int kLaneVecs = 16;        // 16-byte vectors per lane per segment
 constexpr int kSegVecs = 32 * kLaneVecs;  // 512 vectors = 8 KiB per segment
 constexpr int kMaxDraft = 32;
 constexpr int kMaxTopK = 8;
+constexpr int kMaxRaceSplit = 2;    // race items per segment, at most
 constexpr int kMaxSegs = 1024;       // segments per row (V up to 2^21 bf16 / 2^20 fp32)
 constexpr int kScanWarps = 4;        // requests per accept-scan CTA
 
@@ -117,7 +118,7 @@ struct VerifyArgs {
   PartStat* pstat;         // [B, slots, nseg]
   TopPart* tpart;          // [B, D_max, nseg] (saguaro draft rows)
   RaceDesc* rdesc;         // [B] race descriptions (written by the scan)
-  RacePart* rpart;         // [B, nseg] race segment results
+  RacePart* rpart;         // [B, nseg * rsplit] race item results
   unsigned int* rcount;    // [B] race segments finished (zeroed by the scan)
   unsigned long long* best_key;  // [B] best exact race key so far, ordered bits (set by the scan)
   unsigned short* rorder;  // [B, nseg] race segments by descending largest logit (set by the scan)
@@ -128,6 +129,7 @@ struct VerifyArgs {
   int nvec, nseg, slots;
   int mode;
   int per_request;         // after the statistics: 1 = one CTA per request, 0 = scan then race items
+  int rsplit;              // race items per segment (1 or kMaxRaceSplit) in the race-items layout
   float temperature;
   int saguaro_k;
   float saguaro_c;
@@ -163,7 +165,7 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   L.rdesc = off;
   off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
   L.rpart = off;
-  off = align_up(off + (size_t)B * nseg * sizeof(RacePart), 256);
+  off = align_up(off + (size_t)B * nseg * kMaxRaceSplit * sizeof(RacePart), 256);
   L.rcount = off;
   off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
   L.best_key = off;
@@ -311,6 +313,7 @@ bool row_stats_tickets(const VerifyArgs& a, int grid);
 int row_stats_blocks_per_sm(int dtype);
 cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
+int race_split(int B, int nseg, int dtype, int sms);
 cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype);

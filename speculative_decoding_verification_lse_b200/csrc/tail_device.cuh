@@ -8,7 +8,8 @@
 //     multiprocessors.
 //   scan, then race items: one CTA per request does the merge, the scan and the
 //     reference key (scan_cta); then one warp per (request, segment) races the
-//     segment, and the warp that finishes a request's last segment (an atomic
+//     segment -- or half of it, while the items fit in one wave of resident
+//     warps -- and the warp that finishes a request's last item (an atomic
 //     counter, no waiting) combines them and writes the token (race_item).
 //     The items are taken rank-major -- every request's segment with the
 //     largest logit first, then every request's second, ... -- so that by the
@@ -176,13 +177,18 @@ __device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared&
   __syncthreads();  // S is reused by the next request
 }
 
-// Race item `item` (rank-major: item = rank * B + b), by one warp; rd: the
-// warp's shared slot for the request's race description.
+// Race item `item`, by one warp; rd: the warp's shared slot for the request's
+// race description.  Each segment is cut into a.rsplit parts of whole 32-token
+// groups; the items are rank-major over the parts (item = (rank * rsplit + h)
+// * B + b: part h of request b's segment of rank `rank`).
 template <int DT>
 __device__ __forceinline__ void race_item(const VerifyArgs& a, long long item, RaceDesc* rd) {
+  constexpr int NG = kLaneVecs / (32 / Lanes<DT>::VEC);
   const int lane = threadIdx.x & 31;
   const int b = (int)(item % a.B);
-  const int rank = (int)(item / a.B);
+  const int pr = (int)(item / a.B);
+  const int rank = pr / a.rsplit, h = pr % a.rsplit;
+  const int nparts = a.nseg * a.rsplit;
   constexpr int n16 = sizeof(RaceDesc) / 16;
   if (lane < n16)
     reinterpret_cast<uint4*>(rd)[lane] = __ldcg(reinterpret_cast<const uint4*>(a.rdesc + b) + lane);
@@ -195,7 +201,8 @@ __device__ __forceinline__ void race_item(const VerifyArgs& a, long long item, R
   const unsigned long long bk = *(volatile unsigned long long*)&a.best_key[b];
   const double K = fmax(rd->K0, bk ? from_ordered_u64(bk) : -INFINITY);
   const Best sb = race_segment_in<DT>(a, *rd, race_stream(a.seed, rd->g), trow, qrow, residual,
-                                      seg, K, filter_offset(K, rd->lse_t));
+                                      seg, K, filter_offset(K, rd->lse_t), h * NG / a.rsplit,
+                                      (h + 1) * NG / a.rsplit);
   unsigned prev = 0;
   if (lane == 0) {
     if (sb.idx >= 0) atomicMax(&a.best_key[b], ordered_u64(sb.best));
@@ -204,18 +211,18 @@ __device__ __forceinline__ void race_item(const VerifyArgs& a, long long item, R
     p.second = sb.second;
     p.idx = sb.idx;
     p.pad = 0;
-    a.rpart[(size_t)b * a.nseg + seg] = p;
+    a.rpart[(size_t)b * nparts + seg * a.rsplit + h] = p;
     __threadfence();
     prev = atomicAdd(&a.rcount[b], 1u);
   }
   prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-  if (prev != (unsigned)(a.nseg - 1)) return;
+  if (prev != (unsigned)(nparts - 1)) return;
 
-  // the request's last segment: combine every segment's result
+  // the request's last part: combine every part's result
   __threadfence();
   Best r{-INFINITY, -INFINITY, -1};
-  for (int s = lane; s < a.nseg; s += 32) {
-    const RacePart* pp = a.rpart + (size_t)b * a.nseg + s;
+  for (int s = lane; s < nparts; s += 32) {
+    const RacePart* pp = a.rpart + (size_t)b * nparts + s;
     Best o;
     o.best = __ldcg(&pp->best);
     o.second = __ldcg(&pp->second);

@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(kThreads, 2) race_kernel(VerifyArgs a) {
   wait_for_previous_kernel();
   const int warp = threadIdx.x >> 5;
   const long long item = (long long)blockIdx.x * kWarps + warp;
-  if (item >= (long long)a.B * a.nseg) return;
+  if (item >= (long long)a.B * a.nseg * a.rsplit) return;
   race_item<DT>(a, item, &s_rd[warp]);
 }
 
@@ -68,8 +68,25 @@ cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s) {
                          : launch_dependent(request_kernel<kBF16>, a.B, s, a);
 }
 
+// Race items per segment: a race warp is bound by its own chain of Philox
+// rounds and loads, not by the SM's throughput, so while the items fit in one
+// wave of resident warps, cutting each segment in two halves the race's time.
+int race_split(int B, int nseg, int dtype, int sms) {
+  static int per_sm[2] = {-1, -1};
+  int& n = per_sm[dtype == kF32 ? 0 : 1];
+  if (n < 0) {
+    int m = 0;
+    const cudaError_t e =
+        dtype == kF32 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, race_kernel<kF32>, kThreads, 0)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, race_kernel<kBF16>, kThreads, 0);
+    n = e == cudaSuccess ? m : 0;
+  }
+  const long long resident = (long long)n * sms * kWarps;
+  return (long long)B * nseg * kMaxRaceSplit <= resident ? kMaxRaceSplit : 1;
+}
+
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s) {
-  const long long items = (long long)a.B * a.nseg;
+  const long long items = (long long)a.B * a.nseg * a.rsplit;
   if (items == 0) return cudaSuccess;
   const unsigned grid = (unsigned)((items + kWarps - 1) / kWarps);
   return a.dtype == kF32 ? launch_dependent(race_kernel<kF32>, grid, s, a)
