@@ -94,6 +94,22 @@ __device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* ro
   }
 }
 
+// "Largest value, then lowest index" keys in 32 bits for bf16 values and
+// indices below 2^16 (the top half of the value's order-preserving bits, then
+// the complemented index), so that one hardware warp reduction finds the
+// maximum; 0 is below every real key.
+__device__ __forceinline__ uint32_t value_index_key32(float v, int idx) {
+  return (ordered_bits(v) & 0xFFFF0000u) | (0xFFFFu - (uint32_t)idx);
+}
+
+__device__ __forceinline__ float key32_value(uint32_t k) {
+  const uint32_t o = k >> 16;
+  const uint32_t b = (o & 0x8000u) ? (o & 0x7FFFu) : (~o & 0xFFFFu);
+  return __uint_as_float(b << 16);
+}
+
+__device__ __forceinline__ int key32_index(uint32_t k) { return (int)(0xFFFFu - (k & 0xFFFFu)); }
+
 // Statistics of one segment whose lane vectors are raw[0..kLaneVecs-1] (the
 // vectors seg*kSegVecs + lane + 32 j of the row), by one full warp.
 template <int DT, bool LSE, bool ARGMAX, bool TOP>
@@ -182,7 +198,14 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
   // of the segment's top k is in its own lane's top k, which the list keeps.
   if (TOP) {
     float T = -INFINITY;
-    {
+    if constexpr (DT == kBF16) {
+      uint32_t mine = value_index_key32(m_t, lane);
+      for (int r = 0; r < topk; ++r) {
+        const uint32_t win = __reduce_max_sync(0xFFFFFFFFu, mine);
+        T = key32_value(win);
+        if (mine == win) mine = 0u;  // each lane maximum counts once
+      }
+    } else {
       unsigned long long mine = value_index_key(m_t, lane);
       for (int r = 0; r < topk; ++r) {
         const unsigned long long win = warp_max_u64(mine);
@@ -249,12 +272,24 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
           hv = tv[s];
           hi = ti[s];
         }
-      const unsigned long long key = hi == INT_MAX ? 0ull : value_index_key(hv, hi);
-      const unsigned long long win = warp_max_u64(key);
-      if (win != 0ull && key == win) ++h;
-      if (lane == 0) {
-        tout->v[r] = win ? key_value(win) : -INFINITY;
-        tout->i[r] = win ? key_index(win) : INT_MAX;
+      if constexpr (DT == kBF16) {
+        // indices relative to the segment's first token (below 4096)
+        const int base = seg * kSegVecs * VEC;
+        const uint32_t key = hi == INT_MAX ? 0u : value_index_key32(hv, hi - base);
+        const uint32_t win = __reduce_max_sync(0xFFFFFFFFu, key);
+        if (win != 0u && key == win) ++h;
+        if (lane == 0) {
+          tout->v[r] = win ? key32_value(win) : -INFINITY;
+          tout->i[r] = win ? base + key32_index(win) : INT_MAX;
+        }
+      } else {
+        const unsigned long long key = hi == INT_MAX ? 0ull : value_index_key(hv, hi);
+        const unsigned long long win = warp_max_u64(key);
+        if (win != 0ull && key == win) ++h;
+        if (lane == 0) {
+          tout->v[r] = win ? key_value(win) : -INFINITY;
+          tout->i[r] = win ? key_index(win) : INT_MAX;
+        }
       }
     }
   }
