@@ -115,13 +115,17 @@ enum {
 };
 
 /* device status word bits (sv_get_device_status): the union of the error
- * flags of every request since the word was last cleared */
+ * flags of every request since the word was last cleared, and
+ * SV_STATUS_TIMEOUT: a bounded wait of the fused kernel's grid barrier expired
+ * (the CTAs that gave up wrote -1 outputs and this bit as the flags of their
+ * requests); the context stays usable. */
 enum {
   SV_STATUS_BAD_TOKEN = SV_FLAG_BAD_TOKEN,
   SV_STATUS_BAD_ROW_D = SV_FLAG_BAD_ROW_D,
   SV_STATUS_NONFINITE = SV_FLAG_NONFINITE,
   SV_STATUS_BAD_PARAM = SV_FLAG_BAD_PARAM,
-  SV_STATUS_RESIDUAL_EMPTY = SV_FLAG_RESIDUAL_EMPTY
+  SV_STATUS_RESIDUAL_EMPTY = SV_FLAG_RESIDUAL_EMPTY,
+  SV_STATUS_TIMEOUT = 1u << 12
 };
 
 /* Limits checked on the host. */

@@ -25,7 +25,9 @@ SV_FLAG_BAD_ROW_D = 1 << 9
 SV_FLAG_NONFINITE = 1 << 10
 SV_FLAG_BAD_PARAM = 1 << 11
 SV_FLAG_NEAR_TIE = SV_FLAG_ACCEPT_NEAR_TIE | SV_FLAG_RACE_NEAR_TIE
-SV_FLAG_ERRORS = SV_FLAG_BAD_TOKEN | SV_FLAG_BAD_ROW_D | SV_FLAG_NONFINITE | SV_FLAG_BAD_PARAM
+SV_STATUS_TIMEOUT = 1 << 12
+SV_FLAG_ERRORS = (SV_FLAG_BAD_TOKEN | SV_FLAG_BAD_ROW_D | SV_FLAG_NONFINITE | SV_FLAG_BAD_PARAM
+                  | SV_STATUS_TIMEOUT)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspecverify.so")

@@ -12,39 +12,12 @@
 // bounded: a CTA that gives up sets SV_STATUS_TIMEOUT, writes -1 for its
 // requests and ends.  Since the launch is cooperative, no CTA ever waits for
 // one that is not running.
+#include "grid_barrier.cuh"
 #include "tail_device.cuh"
 
 namespace sv {
 
 namespace {
-
-constexpr int kBarrierPolls = 1 << 22;  // with a 64 ns sleep each: about a quarter second
-
-__device__ __forceinline__ unsigned load_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Every CTA of the grid at barrier `k`; false if the wait gave up.
-__device__ bool grid_barrier(const VerifyArgs& a, int k) {
-  __shared__ int s_ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();  // the CTA's writes before its arrival
-    atomicAdd(&a.barrier[k], 1u);
-    unsigned n = load_acquire(&a.barrier[k]);
-    for (int i = 0; n < gridDim.x && i < kBarrierPolls; ++i) {
-      __nanosleep(64);
-      n = load_acquire(&a.barrier[k]);
-    }
-    s_ok = n >= gridDim.x;
-    if (!s_ok) atomicOr(a.status, kStatusTimeout);
-    __threadfence();
-  }
-  __syncthreads();
-  return s_ok != 0;
-}
 
 // The CTA gave up at a barrier: -1 for its requests.
 __device__ void fail_requests(const VerifyArgs& a) {
@@ -64,13 +37,13 @@ __global__ void __launch_bounds__(kThreads, 2) fused_kernel(VerifyArgs a) {
   __shared__ RaceDesc s_rd[kWarps];
   const int warp = threadIdx.x >> 5;
   stats_pass<DT, true>(a, blockIdx.x * kWarps + warp, gridDim.x * kWarps);
-  if (!grid_barrier(a, 0)) return fail_requests(a);
+  if (!grid_barrier(&a.barrier[0], a.status)) return fail_requests(a);
   if (a.per_request) {
     for (int b = blockIdx.x; b < a.B; b += gridDim.x) tail_request<DT>(a, b, S);
     return;
   }
   for (int b = blockIdx.x; b < a.B; b += gridDim.x) scan_cta<DT>(a, b, S);
-  if (!grid_barrier(a, 1)) return fail_requests(a);
+  if (!grid_barrier(&a.barrier[1], a.status)) return fail_requests(a);
   const long long items = (long long)a.B * a.nseg * a.rsplit;
   for (long long it = (long long)blockIdx.x * kWarps + warp; it < items; it += (long long)gridDim.x * kWarps)
     race_item<DT>(a, it, &s_rd[warp]);

@@ -1,5 +1,6 @@
 """The CUDA helpers that the GPU tests compile on the fly (the cuRAND Philox
-probe and the race word-filter probe, which includes the library's device headers)
+probe, the race word-filter probe and the grid-barrier probe, which include the
+library's device headers)
 must keep compiling for sm_100a; nvcc works without a GPU, so this runs here."""
 import os
 import subprocess
@@ -12,7 +13,8 @@ CSRC = os.path.join(ROOT, "speculative_decoding_verification_lse_b200", "csrc")
 INC = os.path.join(ROOT, "include")
 
 
-@pytest.mark.parametrize("src", ["curand_philox_probe.cu", "race_filter_probe.cu"])
+@pytest.mark.parametrize("src", ["curand_philox_probe.cu", "race_filter_probe.cu",
+                                 "barrier_probe.cu"])
 def test_gpu_test_helper_compiles(tmp_path, src):
     subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
                     "-shared", "-Xcompiler", "-fPIC", "-I", CSRC, "-I", INC,
