@@ -29,8 +29,9 @@
 // logit (race_ref_key_warp), and grows as segments finish; where none is known
 // (K0 = -inf) a segment first takes the best exact key of its 32 lane-wise
 // largest logits, and if that is -inf too every token survives the filter.
-// One warp handles an 8 KiB segment (race_segment_in); the CTA that owns the
-// request combines the segments (tail_device.cuh).
+// One warp handles an 8 KiB segment, or a run of them (race_segment_in,
+// race_span_in); the segments' results are combined by the CTA that owns the
+// request or by the warp that finishes its last segment (tail_device.cuh).
 #pragma once
 #include "philox.cuh"
 #include "stats_device.cuh"

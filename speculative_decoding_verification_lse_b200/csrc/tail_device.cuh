@@ -2,7 +2,7 @@
 // layouts (the launcher picks one per call):
 //   per request: one CTA per request merges the request's rows
 //     (scan_device.cuh), runs its accept scan, finds a reference key for the
-//     race's word filter and races the sampled row, its warps taking segments
+//     race's word filter and races the sampled row, warp w streaming segments
 //     w, w + 8, ... and sharing the best key found so far in shared memory
 //     (tail_request).  Best when there are at least as many requests as
 //     multiprocessors.
