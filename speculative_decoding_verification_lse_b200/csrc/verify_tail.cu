@@ -2,6 +2,7 @@
 // (tail_device.cuh): either one CTA per request for everything, or the accept
 // scan (one CTA per request) followed by the race (one warp per request and
 // segment of the sampled row).
+#include <atomic>
 #include <cstring>
 
 #include "tail_device.cuh"
@@ -72,14 +73,18 @@ cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s) {
 // rounds and loads, not by the SM's throughput, so while the items fit in one
 // wave of resident warps, cutting each segment in two halves the race's time.
 int race_split(int B, int nseg, int dtype, int sms) {
-  static int per_sm[2] = {-1, -1};
-  int& n = per_sm[dtype == kF32 ? 0 : 1];
+  // resident race CTAs per SM, by dtype (host threads may race to fill it in;
+  // they all store the same value)
+  static std::atomic<int> per_sm[2] = {{-1}, {-1}};
+  std::atomic<int>& slot = per_sm[dtype == kF32 ? 0 : 1];
+  int n = slot.load(std::memory_order_relaxed);
   if (n < 0) {
     int m = 0;
     const cudaError_t e =
         dtype == kF32 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, race_kernel<kF32>, kThreads, 0)
                       : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, race_kernel<kBF16>, kThreads, 0);
     n = e == cudaSuccess ? m : 0;
+    slot.store(n, std::memory_order_relaxed);
   }
   const long long resident = (long long)n * sms * kWarps;
   return (long long)B * nseg * kMaxRaceSplit <= resident ? kMaxRaceSplit : 1;
