@@ -121,6 +121,15 @@ def tail_items(w, sms):
     return w.B < sms and w.B * nseg > sms
 
 
+def input_copies(in_bytes):
+    """How many copies of a step's inputs the timed loop rotates over: enough
+    that together they are at least twice the L2 (at most MAX_INPUT_COPIES),
+    or 1 when the inputs alone are that large."""
+    if in_bytes >= L2_ROTATE_BYTES:
+        return 1
+    return min(MAX_INPUT_COPIES, -(-L2_ROTATE_BYTES // max(1, in_bytes)))
+
+
 def traffic_record(kernel_name, sources, alg_bytes):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source and on a launch of the same algorithmic bytes (the
@@ -257,7 +266,7 @@ def run_ours(args):
     # inputs that fit in L2 rotate over copies whose total is at least twice the
     # L2, so that every timed step reads its logits from HBM
     in_bytes = sum(t.numel() * t.element_size() for t in (w.target, w.draft, w.tokens))
-    ncopies = min(MAX_INPUT_COPIES, -(-L2_ROTATE_BYTES // in_bytes)) if in_bytes < L2_ROTATE_BYTES else 1
+    ncopies = input_copies(in_bytes)
     copies = [w]
     if ncopies > 1:
         big = [t.unsqueeze(0).repeat((ncopies,) + (1,) * t.dim()) for t in (w.target, w.draft, w.tokens)]
