@@ -25,6 +25,11 @@ SV_FLAG_BAD_ROW_D = 1 << 9
 SV_FLAG_NONFINITE = 1 << 10
 SV_FLAG_BAD_PARAM = 1 << 11
 SV_FLAG_NEAR_TIE = SV_FLAG_ACCEPT_NEAR_TIE | SV_FLAG_RACE_NEAR_TIE
+SV_STATUS_BAD_TOKEN = SV_FLAG_BAD_TOKEN
+SV_STATUS_BAD_ROW_D = SV_FLAG_BAD_ROW_D
+SV_STATUS_NONFINITE = SV_FLAG_NONFINITE
+SV_STATUS_BAD_PARAM = SV_FLAG_BAD_PARAM
+SV_STATUS_RESIDUAL_EMPTY = SV_FLAG_RESIDUAL_EMPTY
 SV_STATUS_TIMEOUT = 1 << 12
 SV_FLAG_ERRORS = (SV_FLAG_BAD_TOKEN | SV_FLAG_BAD_ROW_D | SV_FLAG_NONFINITE | SV_FLAG_BAD_PARAM
                   | SV_STATUS_TIMEOUT)

@@ -52,6 +52,30 @@ def test_only_the_abi_is_exported():
     assert ours == set(declared_functions())
 
 
+def header_constants():
+    """Every `SV_NAME = value` of the header's enums, values evaluated (1u << n,
+    plain integers, and references to earlier names)."""
+    text = open(os.path.join(ROOT, "include", "specverify.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    vals = {}
+    for body in re.findall(r"enum\s*\{(.*?)\}", text, flags=re.S):
+        for item in body.split(","):
+            m = re.match(r"\s*(SV_\w+)\s*=\s*(.+?)\s*$", item, flags=re.S)
+            if not m:
+                continue
+            expr = re.sub(r"(\d+)u\b", r"\1", m.group(2))
+            vals[m.group(1)] = eval(expr, {}, dict(vals))
+    return vals
+
+
+def test_binding_constants_equal_the_header():
+    vals = header_constants()
+    assert len(vals) >= 20
+    for name, v in vals.items():
+        assert hasattr(sv, name), name
+        assert getattr(sv, name) == v, (name, getattr(sv, name), v)
+
+
 def test_version_and_workspace_sizes(lib):
     assert sv.sv_version() == 10000
     a = sv.sv_workspace_bytes(256, 7, 128256, sv.SV_BF16)
