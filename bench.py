@@ -151,26 +151,83 @@ def traffic_record(kernel_name, sources, alg_bytes):
     return rec.get(sha)
 
 
-def cpu_baseline(w, target_seconds=10.0):
+def cpu_baseline(w, target_seconds=10.0, single_seconds=5.0):
     """The oracle, as it stands, on the host cores over the same host copy of the
-    inputs; the whole batch is repeated until about `target_seconds` pass."""
+    inputs: the whole batch repeated on all cores (OpenMP over requests) until
+    about `target_seconds` pass, and the plain single-threaded loop on the first
+    requests of the batch for about `single_seconds`."""
     import oracle
     h = w.host_arrays()
     cores = os.cpu_count() or 1
+
+    def run(sl, nthreads):
+        oracle.verify(h["target"][sl], h["draft"][sl], h["tokens"][sl],
+                      None if h["row_D"] is None else h["row_D"][sl], temperature=w.temperature,
+                      mode=w.mode, seed=w.seed,
+                      temperature_per_req=None if h["temperature_per_req"] is None
+                      else h["temperature_per_req"][sl],
+                      mode_per_req=None if h["mode_per_req"] is None else h["mode_per_req"][sl],
+                      saguaro_k=w.saguaro_k, saguaro_c=w.saguaro_c, nthreads=nthreads,
+                      request_offset=sl.start)
+
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.verify(h["target"], h["draft"], h["tokens"], h["row_D"], temperature=w.temperature,
-                      mode=w.mode, seed=w.seed, temperature_per_req=h["temperature_per_req"],
-                      mode_per_req=h["mode_per_req"], saguaro_k=w.saguaro_k,
-                      saguaro_c=w.saguaro_c, nthreads=cores)
+        run(slice(0, w.B), cores)
         reps += 1
         el = time.perf_counter() - t0
         if el >= target_seconds or reps >= 50:
             break
     rows = reps * w.verified_rows()
+    D = w.row_D_list()
+    # single core: requests one at a time until the budget is spent
+    n1, t1 = 0, time.perf_counter()
+    while n1 < w.B:
+        run(slice(n1, n1 + 1), 1)
+        n1 += 1
+        if time.perf_counter() - t1 >= single_seconds:
+            break
+    el1 = time.perf_counter() - t1
+    rows1 = sum(d + 1 for d in D[:n1])
     return {"value": rows / el, "unit": "rows/s", "cores": cores, "kind": "oracle",
             "sample": f"the whole {w.name} batch ({w.B} requests, {w.verified_rows()} verified rows) "
-                      f"x {reps} repetitions, {el:.1f} s, OpenMP over requests"}
+                      f"x {reps} repetitions, {el:.1f} s, OpenMP over requests on {cores} threads",
+            "single_core": {"value": rows1 / el1, "unit": "rows/s", "cores": 1,
+                            "sample": f"the first {n1} requests ({rows1} verified rows), "
+                                      f"{el1:.1f} s, the plain single-threaded loop"}}
+
+
+def acceptance_stats(sv, w, variant, nseeds, stream):
+    """Mean accepted length and the AL histogram (AL = 1 .. D_max+1) of the
+    workload's stochastic requests over `nseeds` verifier seeds, from the
+    library's own outputs; for requests that rejected a draft, the share whose
+    correction token is among the draft row's k largest logits (what saguaro
+    concentrates the residual on)."""
+    import torch
+    stoch = torch.tensor([m != sv.SV_GREEDY for m in w.modes()], device=w.target.device)
+    hist = torch.zeros(w.D_max + 2, dtype=torch.int64, device=w.target.device)
+    in_top = rejected = 0
+    k = min(w.saguaro_k, w.V)
+    Db = torch.tensor(w.row_D_list(), device=w.target.device)
+    out = None
+    for seed in range(nseeds):
+        out = sv.verify_workload(w, seed=7000 + seed, variant=variant, stream=stream, out=out)
+        al = out["accept_len"].long()
+        hist += torch.bincount(al[stoch], minlength=w.D_max + 2)
+        n = al - 1
+        rej = stoch & (n < Db)
+        if bool(rej.any()):
+            b = torch.nonzero(rej).flatten()
+            rows = w.draft[b, n[b]].float()
+            top = torch.topk(rows, k, dim=-1).indices
+            tok = out["tokens"][b, n[b]].long()
+            in_top += int((top == tok[:, None]).any(dim=1).sum())
+            rejected += int(b.numel())
+    hist = hist.cpu().tolist()
+    total = sum(hist)
+    return {"mean_al": sum(i * c for i, c in enumerate(hist)) / max(1, total),
+            "al_hist": hist[1:], "requests": total,
+            "rejections": rejected,
+            f"correction_in_draft_top{k}": in_top / max(1, rejected)}
 
 
 def run_reference(args):
@@ -277,12 +334,26 @@ def run_ours(args):
         sv.verify_workload(copies[i % ncopies], seed=1000 + i, request_offset=offset,
                            variant=variant, stream=stream, out=out, timing_events=ev)
 
+    # clocks are sampled from the start of the warm-up to the end of a window of
+    # untimed steps after the timed region, every step the same call, so that a
+    # short timed region still has samples around it
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    clocks.active = True
+    t_window = time.perf_counter()
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
     status = sv.sv_get_device_status(stream)
     if status & sv.SV_FLAG_ERRORS:
         raise RuntimeError(f"device status {status:#x} during warm-up")
+    extra = 0
+    while time.perf_counter() - t_window < args.clock_window / 2:  # untimed, before
+        for _ in range(16):
+            step(args.warmup + args.steps + extra)
+            extra += 1
+        torch.cuda.synchronize()
 
     # dominant-kernel timing events on every KEV_EVERY-th step of the timed region
     # (a pair on every step would add its own recording cost to the step time)
@@ -294,25 +365,43 @@ def run_ours(args):
         b_ev.record(stream)
     torch.cuda.synchronize()
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    clocks.active = True
     t_start.record(stream)
     for i in range(args.steps):
         step(args.warmup + i, kev[i // KEV_EVERY] if i % KEV_EVERY == 0 else None)
     t_stop.record(stream)
     torch.cuda.synchronize()
+    t_after = time.perf_counter()
+    while time.perf_counter() - t_after < args.clock_window / 2:  # untimed, after
+        for _ in range(16):
+            step(args.warmup + args.steps + extra)
+            extra += 1
+        torch.cuda.synchronize()
     clocks.active = False
+    window_s = time.perf_counter() - t_window
     barrier()
     clocks.stop()
     ms = max_over_ranks(t_start.elapsed_time(t_stop), dev)
-    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    k_list = [a.elapsed_time(b) for a, b in kev]
+    k_ms = statistics.mean(k_list)
+    k_med = statistics.median(k_list)
     ms_per_step = ms / args.steps
     rows_total = w.verified_rows() * args.steps * world
     value = rows_total / (ms / 1e3)
+
+    # acceptance: mean AL and its histogram (for saguaro next to the plain rule
+    # on the same logits, its draft tokens drawn from q instead of q')
+    acceptance = None
+    if args.al_seeds > 0:
+        acceptance = acceptance_stats(sv, w, variant, args.al_seeds, stream)
+        if w.mode == sv.SV_SAGUARO:
+            wp = workloads.make(args.workload, dev, mode=sv.SV_STOCHASTIC,
+                                seed=workloads.CONFIGS[args.workload]["seed"] + 97 * rank)
+            acceptance = {"saguaro": acceptance,
+                          "plain_rule_same_logits": acceptance_stats(sv, wp, variant, args.al_seeds,
+                                                                     stream)}
+            del wp
 
     # end to end through the same call with host buffers: pinned H2D of the
     # step's inputs, the call, D2H of the step's outputs, all in the timed region
@@ -428,14 +517,19 @@ def run_ours(args):
                 "traffic": None if tr is None else tr[0],
                 "algorithmic_bytes_per_launch": kbytes,
                 "launch_ms": k_ms,
+                "launch_ms_median": k_med,
+                "launches_timed": len(k_list),
             },
-            "clocks": clocks.summary(),
+            "clocks": dict(clocks.summary(), window=(
+                f"{window_s:.2f} s from the first warm-up step to {args.clock_window / 2:.2f} s of "
+                f"untimed steps after the timed region, every step the same call")),
             # fused: one launch; split: statistics, then one kernel per request or
             # the scan and the race items (the library's rule, in include/specverify.h)
             "gpu_launches": (1 if used_variant == "fused" else
                              3 if tail_items(w, torch.cuda.get_device_properties(dev).multi_processor_count)
                              else 2) * args.steps,
             "e2e": e2e,
+            "acceptance": acceptance,
         }
         if args.cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
@@ -458,6 +552,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
+    ap.add_argument("--clock-window", type=float, default=0.8,
+                    help="seconds of same-call steps around the timed region while clocks are sampled")
+    ap.add_argument("--al-seeds", type=int, default=40,
+                    help="verifier seeds for the acceptance statistics (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

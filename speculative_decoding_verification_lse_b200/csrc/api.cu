@@ -106,32 +106,11 @@ int cached_workspace(int dev, size_t bytes, void** out) {
 
 }  // namespace
 
-int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
-
-}  // namespace sv
-
-using namespace sv;
-
-extern "C" {
-
-int sv_version(void) { return 10000; }
-
-const char* sv_last_error(void) { return g_last_error.c_str(); }
-
-size_t sv_workspace_bytes(int B, int D_max, int V, int dtype) {
-  if (B < 0 || D_max < 0 || V < 1 || (dtype != SV_F32 && dtype != SV_BF16)) return 0;
-  return ws_layout(B, D_max, V, dtype, true).total;
-}
-
-int sv_verify_ex(const void* target_logits, const void* draft_logits,
-                 const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max, int V,
-                 int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
-                 int32_t* out_accept_len, const sv_params* p) {
-  sv_params prm;
-  memset(&prm, 0, sizeof prm);
-  if (p) prm = *p;
-  g_last_error.clear();
-
+// Every host-side argument check of sv_verify_ex (B == 0 passes them all);
+// also run by sv_verify_static before its size test.
+int check_args(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
+               int B, int D_max, int V, int dtype, float temperature, int mode,
+               const int32_t* out_tokens, const int32_t* out_accept_len, const sv_params& prm) {
   if (B < 0) return fail(SV_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
   if (D_max < 0 || D_max > SV_MAX_DRAFT)
     return fail(SV_ERR_INVALID_ARG, "D_max must be in [0, %d] (got %d)", SV_MAX_DRAFT, D_max);
@@ -170,18 +149,57 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   if (nseg > kMaxSegs)
     return fail(SV_ERR_UNSUPPORTED, "V larger than %d is not supported for this dtype",
                 kMaxSegs * kSegVecs * vec_elems(dtype));
-  const long long slots = 2LL * D_max + 1;
-  if ((long long)B * (slots + 1) * nseg > 0x7FFFFFFFLL)
+  if ((long long)B * (2LL * D_max + 2) * nseg > 0x7FFFFFFFLL)
     return fail(SV_ERR_UNSUPPORTED, "B * (2*D_max+2) * segments exceeds 2^31");
-  const bool saguaro_possible = mode == SV_SAGUARO || prm.mode_per_req != nullptr;
+  return SV_OK;
+}
 
+int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
+}  // namespace sv
+
+using namespace sv;
+
+extern "C" {
+
+int sv_version(void) { return 10000; }
+
+const char* sv_last_error(void) { return g_last_error.c_str(); }
+
+size_t sv_workspace_bytes(int B, int D_max, int V, int dtype) {
+  if (B < 0 || D_max < 0 || V < 1 || (dtype != SV_F32 && dtype != SV_BF16)) return 0;
+  return ws_layout(B, D_max, V, dtype, true).total;
+}
+
+int sv_verify_ex(const void* target_logits, const void* draft_logits,
+                 const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max, int V,
+                 int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
+                 int32_t* out_accept_len, const sv_params* p) {
+  sv_params prm;
+  memset(&prm, 0, sizeof prm);
+  if (p) prm = *p;
+  g_last_error.clear();
+
+  {
+    const int rc = check_args(target_logits, draft_logits, draft_tokens, B, D_max, V, dtype,
+                              temperature, mode, out_tokens, out_accept_len, prm);
+    if (rc != SV_OK) return rc;
+  }
+  if (B == 0) return SV_OK;
+  int k = prm.saguaro_k <= 0 ? 5 : prm.saguaro_k;
+  if (k > V) k = V;
+  const float c = prm.saguaro_c <= 0.0f ? 0.5f : prm.saguaro_c;
+  const int tail_bits = prm.variant & (SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
+  const int base_variant = prm.variant & ~(SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
+  int nvec, nseg;
+  row_geometry(V, dtype, &nvec, &nseg);
+  const long long slots = 2LL * D_max + 1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
 
   // the same layout sv_workspace_bytes reports, whatever the modes
   const WsLayout L = ws_layout(B, D_max, V, dtype, true);
-  (void)saguaro_possible;
   void* ws = prm.workspace;
   unsigned int* status = nullptr;
   const bool fused = base_variant == SV_VARIANT_FUSED;

@@ -19,6 +19,10 @@ namespace sv {
 
 // Sets the message sv_last_error returns and passes the code through (api.cu).
 int set_last_error(int code, const char* msg);
+// sv_verify_ex's host-side argument checks (api.cu).
+int check_args(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
+               int B, int D_max, int V, int dtype, float temperature, int mode,
+               const int32_t* out_tokens, const int32_t* out_accept_len, const sv_params& prm);
 
 namespace {
 
@@ -60,7 +64,15 @@ extern "C" int sv_verify_static(const void* target_logits, const void* draft_log
                                 uint64_t seed, int32_t* out_tokens, int32_t* out_accept_len,
                                 const sv_params* p) {
   using namespace sv;
-  // the same argument checks as sv_verify_ex run first, inside it; here only the size
+  sv_params q;
+  memset(&q, 0, sizeof q);
+  if (p) q = *p;
+  // sv_verify_ex's argument checks first, so that invalid calls get its error codes
+  {
+    const int rc = check_args(target_logits, draft_logits, draft_tokens, B, D_max, V, dtype,
+                              temperature, mode, out_tokens, out_accept_len, q);
+    if (rc != SV_OK) return rc;
+  }
   const size_t need = sv_workspace_bytes(B, D_max, V, dtype);
   if (need > kStaticBytes) {
     char buf[256];
@@ -76,9 +88,6 @@ extern "C" int sv_verify_static(const void* target_logits, const void* draft_log
   void* ws = nullptr;
   const int rc = static_address(dev, &ws);
   if (rc != SV_OK) return rc;
-  sv_params q;
-  memset(&q, 0, sizeof q);
-  if (p) q = *p;
   q.workspace = ws;
   q.workspace_bytes = kStaticBytes;
   return sv_verify_ex(target_logits, draft_logits, draft_tokens, row_D, B, D_max, V, dtype,

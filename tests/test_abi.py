@@ -152,3 +152,19 @@ def test_product_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "svo_" not in text and "svo.h" not in text, f
+
+
+def test_static_entry_point_checks_arguments_before_its_size(lib):
+    # the ordinary argument checks come first, so an invalid call of any size
+    # gets sv_verify_ex's code, and a valid call too large for the fixed array
+    # gets SV_ERR_UNSUPPORTED; neither reaches a CUDA call
+    fake = 1 << 20
+    rc = sv.sv_verify_static(fake, fake, fake, None, 4096, 33, 128256, sv.SV_BF16, 1.0,
+                             sv.SV_STOCHASTIC, 0, fake, fake, None)
+    assert rc == sv.SV_ERR_INVALID_ARG and "D_max" in sv.sv_last_error()
+    rc = sv.sv_verify_static(fake, fake, fake, None, 4096, 7, 128256, sv.SV_BF16, 0.0,
+                             sv.SV_STOCHASTIC, 0, fake, fake, None)
+    assert rc == sv.SV_ERR_INVALID_ARG and "temperature" in sv.sv_last_error()
+    rc = sv.sv_verify_static(fake, fake, fake, None, 4096, 7, 128256, sv.SV_BF16, 1.0,
+                             sv.SV_STOCHASTIC, 0, fake, fake, None)
+    assert rc == sv.SV_ERR_UNSUPPORTED and "sv_verify_static" in sv.sv_last_error()

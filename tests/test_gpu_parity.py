@@ -60,16 +60,39 @@ def test_full_size_workloads(sv, name, sample, variant):
     print(name, s)
 
 
+# (workload, seeds): about 2e5 stochastic requests in all, so that the bound
+# 1e-4 allows about 20 of them
+NEAR_TIE_POOL = [("b256", 400), ("saguaro", 400), ("b32", 800), ("ragged", 800)]
+_POOL_CACHE = {}
+
+
 @VARIANTS
-@pytest.mark.parametrize("name", ["b32", "b256", "ragged", "saguaro"])
-def test_near_tie_rate_below_1e4_of_rows(sv, name, variant):
-    w = wl.make(name, "cuda")
-    flagged = rows = 0
-    for seed in range(8):
-        got = gpu_run(w, seed=seed, variant=variant)
-        flagged += int(np.count_nonzero(got["flags"] & sv.SV_FLAG_NEAR_TIE))
-        rows += w.verified_rows()
-    assert flagged <= max(1, 1e-4 * rows), (flagged, rows)
+def test_near_tie_rate_below_1e4(sv, variant):
+    """Near-tie flags, counted per request against the stochastic requests
+    verified (the strictest unit: a flagged request holds at least one near-tie
+    row, so flagged rows / verified rows is lower still), pooled over four
+    full-size workloads and many seeds; the bound is 0.01%."""
+    flagged = total = 0
+    for name, nseeds in NEAR_TIE_POOL:
+        if name not in _POOL_CACHE:
+            _POOL_CACHE.clear()
+            _POOL_CACHE[name] = wl.make(name, "cuda")
+        w = _POOL_CACHE[name]
+        stoch = torch.tensor([m != sv.SV_GREEDY for m in w.modes()], device="cuda")
+        acc = torch.zeros((), dtype=torch.int64, device="cuda")
+        errs = torch.zeros((), dtype=torch.int64, device="cuda")
+        out = None
+        for seed in range(nseeds):
+            out = sv.verify_workload(w, seed=seed, variant=variant, out=out)
+            acc += (((out["flags"] & sv.SV_FLAG_NEAR_TIE) != 0) & stoch).sum()
+            errs += ((out["flags"] & sv.SV_FLAG_ERRORS) != 0).sum()
+        torch.cuda.synchronize()
+        assert int(errs) == 0, name
+        flagged += int(acc)
+        total += int(stoch.sum()) * nseeds
+    print(f"near-tie requests: {flagged} of {total} stochastic requests")
+    assert total >= 200_000
+    assert flagged <= 1e-4 * total, (flagged, total)
 
 
 def test_full_size_is_deterministic_and_variants_agree(sv):

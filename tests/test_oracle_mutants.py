@@ -39,6 +39,15 @@ MUTANTS = {
     "philox_drops_key": ("uint32_t n0 = hi1 ^ c1 ^ k0;", "uint32_t n0 = hi1 ^ c1;"),
     "philox_two_rounds": ("for (int round = 0; round < 10; ++round)",
                           "for (int round = 0; round < 2; ++round)"),
+    "philox_multipliers_swapped": (
+        "    uint64_t prod0 = (uint64_t)0xD2511F53u * (uint64_t)c0;\n"
+        "    uint64_t prod1 = (uint64_t)0xCD9E8D57u * (uint64_t)c2;",
+        "    uint64_t prod0 = (uint64_t)0xCD9E8D57u * (uint64_t)c0;\n"
+        "    uint64_t prod1 = (uint64_t)0xD2511F53u * (uint64_t)c2;"),
+    "philox_words_permuted": ("  out[0] = c0;\n  out[1] = c1;\n  out[2] = c2;\n  out[3] = c3;",
+                              "  out[0] = c2;\n  out[1] = c1;\n  out[2] = c0;\n  out[3] = c3;"),
+    "philox_weyl_swapped": ("    k0 += 0x9E3779B9u;\n    k1 += 0xBB67AE85u;",
+                            "    k0 += 0xBB67AE85u;\n    k1 += 0x9E3779B9u;"),
     "greedy_wrong_row": ("int am = svo_row_argmax(row_ptr(a->target, trow0 + d, V, dt), V, dt);",
                          "int am = svo_row_argmax(row_ptr(a->target, trow0 + d + 1, V, dt), V, dt);"),
     "argmax_last_tie": ("    if (z > bz) {\n      bz = z;\n      best = x;",
@@ -91,6 +100,47 @@ def check_avalanche(svo, L):
             d.append(sum(bin(x ^ y).count("1") for x, y in zip(a, b)))
     d = np.array(d, float)
     return abs(d.mean() - 64) < 4 * 5.66 / math.sqrt(len(d)) and d.min() > 30
+
+
+def check_kat(svo, L):
+    # the published known answer (C++26 philox4x32, tests/golden/philox4x32_10_kat.txt)
+    from test_oracle_philox_kat import read_kat
+    return all(svo.philox4x32_10([c0, c1, c2, c3], [k0, k1], L=L)[w] == v
+               for c0, c1, c2, c3, k0, k1, w, v in read_kat())
+
+
+_ENGINE_WORDS = {}
+
+
+def check_engines(svo, L):
+    # every word against the independent host implementations (when they build here)
+    if not _ENGINE_WORDS:
+        import test_oracle_philox_kat as kat
+        std_dir, torch_dir = kat._include_dirs()
+        if torch_dir is None and std_dir is None:
+            _ENGINE_WORDS["none"] = None
+        else:
+            with tempfile.TemporaryDirectory() as tmp:
+                exe = os.path.join(tmp, "engines")
+                cmd = ["g++", "-std=c++17", "-O1", kat.PROBE, "-o", exe]
+                kinds = []
+                if std_dir:
+                    cmd[1:1] = ["-DWITH_STD_ENGINE", "-I", std_dir]
+                    kinds.append("std")
+                if torch_dir:
+                    cmd[1:1] = ["-DWITH_TORCH_ENGINE", "-I", torch_dir]
+                    kinds.append("torch")
+                subprocess.run(cmd, check=True, capture_output=True)
+                pairs = kat.pairs_to_check()[:300]
+                _ENGINE_WORDS["pairs"] = pairs
+                _ENGINE_WORDS["words"] = kat.run_engines((exe, kinds), pairs)
+    if "none" in _ENGINE_WORDS:
+        return True
+    for words in _ENGINE_WORDS["words"].values():
+        for (c, k), w in zip(_ENGINE_WORDS["pairs"], words):
+            if svo.philox4x32_10(c, k, L=L) != w:
+                return False
+    return True
 
 
 def check_uniform(svo, L):
@@ -217,7 +267,7 @@ def check_greedy(svo, L):
     return int(out["accept_len"][0]) == D + 1 and list(out["tokens"][0]) == ref[:D + 1]
 
 
-CHECKS = [check_lse, check_argmax, check_avalanche, check_uniform, check_p_eq_q, check_al_law,
+CHECKS = [check_lse, check_argmax, check_kat, check_engines, check_avalanche, check_uniform, check_p_eq_q, check_al_law,
           check_residual_law, check_bonus_law, lambda s, L: check_marginal(s, L, 0),
           lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy]
 

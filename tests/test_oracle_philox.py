@@ -1,10 +1,11 @@
-"""Pins for the oracle's counter-based generator.
+"""Statistical pins for the oracle's counter-based generator.
 
-The pages name Philox but print no known-answer vector, and none ships in this
-image, so the exact words are pinned on the GPU against cuRAND's
-Philox4_32_10 (test_gpu_philox_curand.py).  Here, on the CPU, the generator is
-pinned by properties any correct 10-round Philox has and a broken one loses:
-uniform words, uniform accept draws, unit-exponential race draws, full
+The exact words are pinned on the CPU by test_oracle_philox_kat.py (the C++26
+standard's known answer for philox4x32 and two independent host
+implementations of the same published generator) and on the GPU against
+cuRAND's Philox4_32_10 (test_gpu_philox_curand.py).  Here the generator is
+also pinned by properties any correct 10-round Philox has and a broken one
+loses: uniform words, uniform accept draws, unit-exponential race draws, full
 avalanche on every input bit, and independence of neighbouring counters."""
 import math
 

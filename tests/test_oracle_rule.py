@@ -11,12 +11,15 @@ oracle.  Per-cell bounds are 4 sigma next to a chi^2 test (many cells are
 checked, so 3 sigma would fail a correct sampler by chance); the 10^6-draw
 marginal test keeps the 3 sigma bound it is specified with."""
 import math
+import os
 
 import numpy as np
 import pytest
 
 from svtest_util import (bf16_bits, chi2_pvalue, sample_categorical, sample_rows, softmax,
                          within_sigma)
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 NT = 8  # host threads for the large statistical runs (same code path as 1)
 
@@ -266,28 +269,46 @@ def test_saguaro_topk_and_downweighting(svo):
     same = svo.verify(zt, zq, tok, seed=41, mode=svo.SVO_SAGUARO, saguaro_c=1.0)
     for k in ("tokens", "accept_len"):
         np.testing.assert_array_equal(plain[k], same[k])
-    # a deterministic two-token case: V=6, draft logits tie; top-5 = tokens 0..4
-    zq1 = np.zeros((1, 1, 6), np.float32)
-    zt1 = np.zeros((1, 2, 6), np.float32)
-    # q = 1/6 each; q'(5) = (1/6) / Z with Z = 1 - 0.5 * 5/6 = 7/12 -> q'(5) = 2/7
-    # p(5) = 2/7 exactly at logit ln(2/7) - ln((5/7)/5): accept prob = 1 for any u
-    zt1[0, 0, :] = math.log((5 / 7) / 5)
-    zt1[0, 0, 5] = math.log(2 / 7) + 1e-6
-    out = svo.verify(zt1, zq1, np.array([[5]], np.int32), mode=svo.SVO_SAGUARO, seed=0)
-    assert out["accept_len"][0] == 2
-    # tied draft logits put tokens 0..4 (the lowest indices) in K, so
-    # q'(0) = (1/12)/(7/12) = 1/7: with p(0) just above 1/7 it is always accepted
-    zt2 = np.zeros((1, 2, 6), np.float32)
-    zt2[0, 0, :] = math.log(1 / 7) + 1e-6
-    zt2[0, 0, 5] = math.log(2 / 7)
-    for s in range(50):
-        out = svo.verify(zt2, zq1, np.array([[0]], np.int32), mode=svo.SVO_SAGUARO, seed=s)
-        assert out["accept_len"][0] == 2
-    # with p(0) = 0 token 0 is never accepted nor emitted
-    zt1[0, 0, 0] = -np.inf
-    for s in range(50):
-        out = svo.verify(zt1, zq1, np.array([[0]], np.int32), mode=svo.SVO_SAGUARO, seed=s)
-        assert out["accept_len"][0] == 1 and out["tokens"][0, 0] != 0
+
+
+def read_saguaro_golden():
+    vals = {}
+    with open(os.path.join(GOLDEN, "saguaro_tied_draft.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, *v = line.split()
+                vals[k] = [float(x) for x in v]
+    return int(vals["V"][0]), vals["c"][0], vals["Z"][0], np.array(vals["qprime"])
+
+
+def test_saguaro_tied_draft_matches_the_hand_computed_case(svo):
+    """tests/golden/saguaro_tied_draft.txt: every draft logit 0 at V=6, so K is
+    tokens 0..4 (lowest indices on ties) and q' is known by hand.  The oracle
+    must accept token x with probability min(1, p(x)/q'(x)): always when p(x)
+    is just above q'(x), with probability 1/2 when p(x) = q'(x)/2, never when
+    p(x) = 0."""
+    V, c, Z, qp = read_saguaro_golden()
+    zq = np.zeros((1, 1, V), np.float32)
+    N = 4000
+    for x in (0, 5):
+        for scale, rate in ((1.0 + 1e-5, 1.0), (0.5, 0.5), (0.0, 0.0)):
+            px = qp[x] * scale
+            p = np.full(V, (1.0 - px) / (V - 1))
+            p[x] = px
+            zt = np.zeros((1, 2, V), np.float32)
+            with np.errstate(divide="ignore"):
+                zt[0, 0] = np.log(p).astype(np.float32)  # p(x) = 0 -> -inf, a masked token
+            out = svo.verify(np.repeat(zt, N, 0), np.repeat(zq, N, 0), np.full((N, 1), x, np.int32),
+                             mode=svo.SVO_SAGUARO, saguaro_c=c, seed=3)
+            acc = float(np.mean(out["accept_len"] == 2))
+            if rate in (0.0, 1.0):
+                assert acc == rate, (x, scale, acc)
+            else:
+                assert abs(acc - rate) < 4 * math.sqrt(rate * (1 - rate) / N), (x, scale, acc)
+            # an emitted correction is never the rejected draft when p(x) <= q'(x)
+            rej = out["accept_len"] == 1
+            assert np.all(out["tokens"][rej, 0] != x)
+    assert abs(Z - (1 - (1 - c) * 5 / V)) < 1e-15 and abs(qp.sum() - 1) < 1e-12
 
 
 def test_accept_near_tie_is_flagged(svo):
