@@ -62,6 +62,10 @@ def _declare(L):
         ctypes.c_int,
     ]
     L.svo_verify.restype = ctypes.c_int
+    L.svo_epilogue.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                               ctypes.c_void_p, ctypes.c_void_p]
+    L.svo_epilogue.restype = ctypes.c_int
     L.svo_has_openmp.argtypes = []
     L.svo_has_openmp.restype = ctypes.c_int
     return L
@@ -164,3 +168,25 @@ def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SVO_STOCH
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
     return dict(tokens=out_tokens, accept_len=out_al, flags=out_flags, row_lse=out_lse)
+
+
+def epilogue(window, out_tokens, accept_len, seq=None, seq_len=None, *, next_window=True,
+             L=None):
+    """The host epilogue (svo_epilogue).  window, out_tokens [B, D_max+1] int32,
+    accept_len [B]; seq [B, cap] and seq_len [B] are updated in copies.
+    Returns dict(next_window or None, seq, seq_len, full [B] bool)."""
+    out_tokens = np.ascontiguousarray(out_tokens, dtype=np.int32)
+    B, W = out_tokens.shape
+    accept_len = np.ascontiguousarray(accept_len, dtype=np.int32).reshape(B)
+    win = None if window is None else np.ascontiguousarray(window, dtype=np.int32).reshape(B, W)
+    nw = np.empty((B, W), np.int32) if next_window else None
+    sq = None if seq is None else np.array(seq, dtype=np.int32, copy=True, order="C")
+    sl = None if seq_len is None else np.array(seq_len, dtype=np.int32, copy=True).reshape(B)
+    full = np.zeros(((B + 31) // 32,), np.uint32)
+    cap = 0 if sq is None else sq.shape[1]
+    rc = (L or lib()).svo_epilogue(_ptr(win), _ptr(out_tokens), _ptr(accept_len), B, W - 1,
+                                   _ptr(nw), _ptr(sq), cap, _ptr(sl), _ptr(full))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (rc={rc})")
+    bits = np.array([(full[b // 32] >> (b % 32)) & 1 for b in range(B)], bool)
+    return dict(next_window=nw, seq=sq, seq_len=sl, full=bits)

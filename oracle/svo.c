@@ -446,6 +446,53 @@ int svo_verify(const void* target, const void* draft, const int32_t* tokens,
   return 0;
 }
 
+/* ---------------------------------------------------------------- epilogue */
+
+/* "Accélérer Sonar par la Spéculation", section "Calendrier MTP pour un jeton
+ * unique": after verification the target's input tokens are shifted by one and
+ * the next target token is inserted at its slot; the accepted length decides
+ * the next sequence length.  Reading: the verification window of request b is
+ * its last committed token followed by its D_max draft slots, so the shifted
+ * window starts with the drafts, and the token the verifier emitted at slot n
+ * (the correction or the bonus) goes to slot n of the shifted window; the slots
+ * after n keep the shifted drafts (the page's "redundant work on tokens that
+ * were not accepted") and the last slot, which nothing shifts into, is -1.  The
+ * AL emitted tokens are appended to the request's sequence at its current
+ * length. */
+int svo_epilogue(const int32_t* window, const int32_t* out_tokens, const int32_t* accept_len,
+                 int B, int D_max, int32_t* next_window, int32_t* seq, int seq_cap,
+                 int32_t* seq_len, uint32_t* full) {
+  if (B < 0 || D_max < 0) return -1;
+  if (B > 0 && (!out_tokens || !accept_len)) return -1;
+  if (next_window && !window) return -1;
+  if (seq && (!seq_len || seq_cap < 0)) return -1;
+  const size_t W = (size_t)D_max + 1;
+  for (int b = 0; b < B; ++b) {
+    /* an accepted length outside [1, D_max + 1] is an error the verification flagged */
+    const int32_t AL = accept_len[b] >= 1 && (size_t)accept_len[b] <= W ? accept_len[b] : 0;
+    const int32_t* ot = out_tokens + (size_t)b * W;
+    if (next_window) {
+      /* read the whole row first: next_window may be window itself */
+      int32_t row[W];
+      for (size_t j = 0; j < W; ++j) row[j] = -1;
+      if (AL >= 1) {
+        for (size_t j = 0; j + 1 < W; ++j) row[j] = window[(size_t)b * W + j + 1];
+        row[AL - 1] = ot[AL - 1];
+      }
+      for (size_t j = 0; j < W; ++j) next_window[(size_t)b * W + j] = row[j];
+    }
+    if (seq && AL >= 1) {
+      if ((long long)seq_len[b] + AL > seq_cap || seq_len[b] < 0) {
+        if (full) full[b / 32] |= 1u << (b % 32);
+      } else {
+        for (int j = 0; j < AL; ++j) seq[(size_t)b * (size_t)seq_cap + seq_len[b] + j] = ot[j];
+        seq_len[b] += AL;
+      }
+    }
+  }
+  return 0;
+}
+
 int svo_has_openmp(void) {
 #ifdef _OPENMP
   return 1;

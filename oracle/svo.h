@@ -91,6 +91,28 @@ int svo_verify(const void* target, const void* draft, const int32_t* tokens,
                int32_t* out_tokens, int32_t* out_accept_len, uint32_t* out_flags,
                double* out_row_lse, int nthreads);
 
+/*
+ * The step after verification, on the host ("Accélérer Sonar par la
+ * Spéculation", section "Calendrier MTP pour un jeton unique": the target's
+ * input tokens are shifted and the next target token is inserted at its slot,
+ * so the next run needs no CPU sync; the accepted length sets the next
+ * sequence length).  For request b with AL = accept_len[b] and n = AL - 1:
+ *   next_window[b][j] = window[b][j + 1] for j < D_max, next_window[b][D_max] = -1,
+ *   then next_window[b][n] = out_tokens[b][n]          (when next_window != NULL)
+ *   seq[b][seq_len[b] + j] = out_tokens[b][j] for j < AL, seq_len[b] += AL
+ *                                                      (when seq != NULL)
+ * A request with AL outside [1, D_max + 1] (an error flagged by the
+ * verification) gets a next-window row of -1 and no append; one whose append would pass seq_cap
+ * gets its next-window row but no append, and its bit in *full (when full is
+ * not NULL) is set: full[b / 32] |= 1 << (b % 32).
+ * Arrays: window, next_window [B, D_max+1]; out_tokens [B, D_max+1];
+ * accept_len, seq_len [B]; seq [B, seq_cap].  Returns 0, or -1 for invalid
+ * arguments.
+ */
+int svo_epilogue(const int32_t* window, const int32_t* out_tokens, const int32_t* accept_len,
+                 int B, int D_max, int32_t* next_window, int32_t* seq, int seq_cap,
+                 int32_t* seq_len, uint32_t* full);
+
 /* 1 when built with OpenMP, else 0. */
 int svo_has_openmp(void);
 

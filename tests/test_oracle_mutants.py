@@ -55,6 +55,9 @@ MUTANTS = {
     "saguaro_no_renormalise": ("return lq + (in_k ? q->ln_c : 0.0) - q->ln_Z;",
                                "return lq + (in_k ? q->ln_c : 0.0);"),
     "saguaro_topk_last_tie": ("if (best < 0 || z > bz) {", "if (best < 0 || z >= bz) {"),
+    "epilogue_insert_one_late": ("row[AL - 1] = ot[AL - 1];", "if (AL < (int32_t)W) row[AL] = ot[AL - 1];"),
+    "epilogue_no_shift": ("row[j] = window[(size_t)b * W + j + 1];", "row[j] = window[(size_t)b * W + j];"),
+    "epilogue_append_drops_last": ("for (int j = 0; j < AL; ++j) seq", "for (int j = 0; j + 1 < AL; ++j) seq"),
 }
 
 
@@ -267,9 +270,31 @@ def check_greedy(svo, L):
     return int(out["accept_len"][0]) == D + 1 and list(out["tokens"][0]) == ref[:D + 1]
 
 
+def check_epilogue(svo, L):
+    # the hand-written example and the greedy chain of test_oracle_epilogue.py
+    import test_oracle_epilogue as te
+
+    class Shim:
+        SVO_GREEDY = svo.SVO_GREEDY
+
+        @staticmethod
+        def epilogue(*a, **k):
+            return svo.epilogue(*a, L=L, **k)
+
+        @staticmethod
+        def verify(*a, **k):
+            return svo.verify(*a, L=L, **k)
+    try:
+        te.test_worked_example(Shim)
+        te.test_greedy_chain_with_epilogue_reproduces_argmax_decoding(Shim)
+    except AssertionError:
+        return False
+    return True
+
+
 CHECKS = [check_lse, check_argmax, check_kat, check_engines, check_avalanche, check_uniform, check_p_eq_q, check_al_law,
           check_residual_law, check_bonus_law, lambda s, L: check_marginal(s, L, 0),
-          lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy]
+          lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy, check_epilogue]
 
 
 def _build_variant(tmp, text):
