@@ -111,26 +111,41 @@ enum {
   SV_FLAG_BAD_TOKEN = 1u << 8,
   SV_FLAG_BAD_ROW_D = 1u << 9,
   SV_FLAG_NONFINITE = 1u << 10,
-  SV_FLAG_BAD_PARAM = 1u << 11
+  SV_FLAG_BAD_PARAM = 1u << 11,
+  SV_FLAG_SEQ_FULL = 1u << 13        /* sv_epilogue: the append would pass seq_cap (skipped) */
 };
 
 /* device status word bits (sv_get_device_status): the union of the error
  * flags of every request since the word was last cleared, and
- * SV_STATUS_TIMEOUT: a bounded wait of the fused kernel's grid barrier expired
- * (the CTAs that gave up wrote -1 outputs and this bit as the flags of their
- * requests); the context stays usable. */
+ * SV_STATUS_TIMEOUT: a bounded wait of the fused kernel expired (about two
+ * seconds; the warps that gave up left, and that call's outputs are
+ * undefined); the context stays usable. */
 enum {
   SV_STATUS_BAD_TOKEN = SV_FLAG_BAD_TOKEN,
   SV_STATUS_BAD_ROW_D = SV_FLAG_BAD_ROW_D,
   SV_STATUS_NONFINITE = SV_FLAG_NONFINITE,
   SV_STATUS_BAD_PARAM = SV_FLAG_BAD_PARAM,
   SV_STATUS_RESIDUAL_EMPTY = SV_FLAG_RESIDUAL_EMPTY,
-  SV_STATUS_TIMEOUT = 1u << 12
+  SV_STATUS_TIMEOUT = 1u << 12,
+  SV_STATUS_SEQ_FULL = SV_FLAG_SEQ_FULL
 };
 
 /* Limits checked on the host. */
 #define SV_MAX_DRAFT 32  /* D_max <= 32 */
 #define SV_MAX_SAGUARO_K 8
+
+/* The step after verification, run on the device by sv_epilogue or by
+ * sv_verify_ex when sv_params.epilogue is set (see sv_epilogue). */
+typedef struct sv_epilogue_args {
+  const int32_t* window;   /* [B, D_max+1] device: the verified input window of each request
+                              (its last committed token, then its draft slots); may be NULL
+                              when next_window is NULL */
+  int32_t* next_window;    /* [B, D_max+1] device, optional: the shifted window with the
+                              emitted target token inserted; may be `window` itself */
+  int32_t* seq;            /* [B, seq_cap] device, optional: each request's token sequence */
+  int seq_cap;             /* tokens per row of seq */
+  int32_t* seq_len;        /* [B] device, in/out: each request's sequence length (with seq) */
+} sv_epilogue_args;
 
 /*
  * Optional parameters.  Zero-initialise, then set what you need.
@@ -155,6 +170,10 @@ typedef struct sv_params {
   void* timing_events;               /* optional cudaEvent_t[2]: recorded on the stream
                                         immediately before and after the row-statistics
                                         kernel (split) or the fused kernel (fused) */
+  const sv_epilogue_args* epilogue;  /* optional: after the verification, on the same stream,
+                                        the step sv_epilogue describes, on this call's
+                                        out_tokens / out_accept_len (and out_flags, which get
+                                        SV_FLAG_SEQ_FULL); host struct, read during the call */
 } sv_params;
 
 /*
@@ -217,6 +236,33 @@ SV_API int sv_verify_static(const void* target_logits, const void* draft_logits,
                             const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max,
                             int V, int dtype, float temperature, int mode, uint64_t seed,
                             int32_t* out_tokens, int32_t* out_accept_len, const sv_params* p);
+
+/*
+ * sv_epilogue: the step after verification, on the device, so that the next
+ * decoding step needs no GPU-to-CPU sync ("Accélérer Sonar par la
+ * Spéculation", section "Calendrier MTP pour un jeton unique": the target's
+ * input tokens are shifted and a kernel inserts the next target tokens at
+ * their slots; section "Inférence avec décodage spéculatif": the accepted
+ * length sets the next sequence length).  Per request b with
+ * AL = out_accept_len[b] and n = AL - 1:
+ *   next_window[b][j] = window[b][j + 1] for j < D_max; next_window[b][D_max] = -1;
+ *   then next_window[b][n] = out_tokens[b][n] (the correction or bonus token).
+ *   So next_window[b][0..n] are the AL emitted tokens, and the slots after n
+ *   keep the drafts that were not accepted (the draft model may re-run on the
+ *   whole window; their results are simply not used).
+ *   seq[b][seq_len[b] + j] = out_tokens[b][j] for j < AL; seq_len[b] += AL.
+ * A request whose AL lies outside [1, D_max + 1] (the verification flagged an
+ * error for it) gets a next-window row of -1 and no append.  An append that
+ * would pass seq_cap (or a negative seq_len) is skipped and sets
+ * SV_FLAG_SEQ_FULL in flags[b] (when flags is not NULL) and in the device
+ * status word.  All arrays are device arrays the caller owns; next_window and
+ * seq may each be NULL (that part is skipped).  Asynchronous on `stream`
+ * (cudaStream_t, NULL = legacy default); host-detectable errors return a
+ * negative code and launch nothing.
+ */
+SV_API int sv_epilogue(const int32_t* window, const int32_t* out_tokens,
+                       const int32_t* out_accept_len, int B, int D_max, int32_t* next_window,
+                       int32_t* seq, int seq_cap, int32_t* seq_len, uint32_t* flags, void* stream);
 
 /* Bytes of scratch one call with these sizes needs (for sv_params.workspace). */
 SV_API size_t sv_workspace_bytes(int B, int D_max, int V, int dtype);

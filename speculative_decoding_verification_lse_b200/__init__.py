@@ -24,6 +24,7 @@ SV_FLAG_BAD_TOKEN = 1 << 8
 SV_FLAG_BAD_ROW_D = 1 << 9
 SV_FLAG_NONFINITE = 1 << 10
 SV_FLAG_BAD_PARAM = 1 << 11
+SV_FLAG_SEQ_FULL = 1 << 13
 SV_FLAG_NEAR_TIE = SV_FLAG_ACCEPT_NEAR_TIE | SV_FLAG_RACE_NEAR_TIE
 SV_STATUS_BAD_TOKEN = SV_FLAG_BAD_TOKEN
 SV_STATUS_BAD_ROW_D = SV_FLAG_BAD_ROW_D
@@ -31,11 +32,23 @@ SV_STATUS_NONFINITE = SV_FLAG_NONFINITE
 SV_STATUS_BAD_PARAM = SV_FLAG_BAD_PARAM
 SV_STATUS_RESIDUAL_EMPTY = SV_FLAG_RESIDUAL_EMPTY
 SV_STATUS_TIMEOUT = 1 << 12
+SV_STATUS_SEQ_FULL = SV_FLAG_SEQ_FULL
 SV_FLAG_ERRORS = (SV_FLAG_BAD_TOKEN | SV_FLAG_BAD_ROW_D | SV_FLAG_NONFINITE | SV_FLAG_BAD_PARAM
                   | SV_STATUS_TIMEOUT)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspecverify.so")
+
+
+class SvEpilogueArgs(ctypes.Structure):
+    """Mirror of sv_epilogue_args."""
+    _fields_ = [
+        ("window", ctypes.c_void_p),
+        ("next_window", ctypes.c_void_p),
+        ("seq", ctypes.c_void_p),
+        ("seq_cap", ctypes.c_int),
+        ("seq_len", ctypes.c_void_p),
+    ]
 
 
 class SvParams(ctypes.Structure):
@@ -53,6 +66,7 @@ class SvParams(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
         ("timing_events", ctypes.c_void_p),
+        ("epilogue", ctypes.POINTER(SvEpilogueArgs)),
     ]
 
 
@@ -90,6 +104,10 @@ def load(build_if_needed=True):
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_void_p, ctypes.c_void_p]
     L.sv_verify_greedy.restype = ctypes.c_int
+    L.sv_epilogue.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                              ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    L.sv_epilogue.restype = ctypes.c_int
     L.sv_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.sv_workspace_bytes.restype = ctypes.c_size_t
     L.sv_get_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
@@ -154,6 +172,13 @@ def sv_verify_static(target_logits, draft_logits, draft_tokens, row_D, B, D_max,
 SV_STATIC_WORKSPACE_BYTES = 8 << 20
 
 
+def sv_epilogue(window, out_tokens, out_accept_len, B, D_max, next_window, seq, seq_cap, seq_len,
+                flags=None, stream=None):
+    return load().sv_epilogue(_p(window), _p(out_tokens), _p(out_accept_len), B, D_max,
+                              _p(next_window), _p(seq), int(seq_cap), _p(seq_len), _p(flags),
+                              _stream_ptr(stream))
+
+
 def sv_workspace_bytes(B, D_max, V, dtype):
     return load().sv_workspace_bytes(B, D_max, V, dtype)
 
@@ -198,9 +223,12 @@ def _dtype_code(t):
 def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHASTIC, seed=0,
            temperature_per_req=None, mode_per_req=None, saguaro_k=5, saguaro_c=0.5,
            request_offset=0, variant=SV_VARIANT_AUTO, stream=None, row_lse=False,
-           out=None, workspace=None, timing_events=None):
+           out=None, workspace=None, timing_events=None, epilogue=None):
     """Verify a batch held in CUDA tensors; returns dict(tokens, accept_len, flags
-    [, row_lse]) as CUDA tensors, enqueued on `stream` (not synchronised)."""
+    [, row_lse]) as CUDA tensors, enqueued on `stream` (not synchronised).
+    epilogue: optional dict(window, next_window, seq, seq_len) of int32 CUDA
+    tensors (any may be None) for the on-device step after verification
+    (sv_epilogue), run on the same stream."""
     import torch
     if not target.is_cuda:
         raise ValueError("target logits must be a CUDA tensor (there is no CPU path)")
@@ -245,6 +273,16 @@ def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHA
             raise ValueError("timing events must have been recorded once before use")
         arr = (ctypes.c_void_p * 2)(timing_events[0].cuda_event, timing_events[1].cuda_event)
         prm.timing_events = ctypes.cast(arr, ctypes.c_void_p)
+    ep = None
+    if epilogue is not None:
+        ep = SvEpilogueArgs()
+        ep.window = _p(epilogue.get("window"))
+        ep.next_window = _p(epilogue.get("next_window"))
+        sq = epilogue.get("seq")
+        ep.seq = _p(sq)
+        ep.seq_cap = 0 if sq is None else int(sq.shape[-1])
+        ep.seq_len = _p(epilogue.get("seq_len"))
+        prm.epilogue = ctypes.pointer(ep)
     with torch.cuda.device(dev):
         _check(sv_verify_ex(target, draft, tokens, row_D, B, D, V, dt, float(temperature),
                             int(mode), int(seed), out["tokens"], out["accept_len"], prm))

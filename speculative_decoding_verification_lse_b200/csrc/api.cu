@@ -42,7 +42,7 @@ struct DeviceCache {
   size_t ws_bytes = 0;
   unsigned int* status = nullptr;  // device address of g_status_word
   int sms = 0;                     // multiprocessor count
-  int fused_per_sm[2] = {0, 0};    // resident fused CTAs per SM, by dtype
+  int fused_per_sm[2][2 * SV_MAX_DRAFT + 2] = {};  // resident fused CTAs per SM, by dtype and slots
   int stats_per_sm[2] = {0, 0};    // resident statistics CTAs per SM, by dtype
 };
 
@@ -68,15 +68,15 @@ int status_word(int dev, unsigned int** out) {
 }
 
 // Resident grids of the persistent kernels on the current device.
-int persistent_grid(int dev, int dtype, bool fused, int* grid) {
+int persistent_grid(int dev, int dtype, bool fused, int slots, int* grid) {
   DeviceCache* c = device_cache(dev);
   if (!c->sms) {
     cudaError_t e = cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   }
-  int* per_sm = fused ? &c->fused_per_sm[dtype] : &c->stats_per_sm[dtype];
+  int* per_sm = fused ? &c->fused_per_sm[dtype][slots] : &c->stats_per_sm[dtype];
   if (!*per_sm) {
-    *per_sm = fused ? fused_blocks_per_sm(dtype) : row_stats_blocks_per_sm(dtype);
+    *per_sm = fused ? fused_blocks_per_sm(dtype, slots) : row_stats_blocks_per_sm(dtype);
     if (*per_sm < 1) return fail(SV_ERR_CUDA, "kernel cannot be resident on this device");
   }
   *grid = c->sms * *per_sm;
@@ -102,6 +102,17 @@ int cached_workspace(int dev, size_t bytes, void** out) {
   }
   *out = c->ws;
   return SV_OK;
+}
+
+// The epilogue sv_params asks for, after the verification on stream s.
+int run_epilogue(const sv_params& prm, const int32_t* out_tokens, const int32_t* out_accept_len,
+                 int B, int D_max, unsigned int* status, cudaStream_t s) {
+  if (!prm.epilogue) return SV_OK;
+  const sv_epilogue_args& ep = *prm.epilogue;
+  const cudaError_t e = launch_epilogue(ep.window, out_tokens, out_accept_len, B, D_max,
+                                        ep.next_window, ep.seq, ep.seq_cap, ep.seq_len,
+                                        prm.out_flags, status, s);
+  return e == cudaSuccess ? SV_OK : cuda_fail(e, "epilogue launch");
 }
 
 }  // namespace
@@ -208,7 +219,7 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     std::lock_guard<std::mutex> lock(g_mu);
     int rc = status_word(dev, &status);
     if (rc) return rc;
-    if ((rc = persistent_grid(dev, dtype, fused, &grid))) return rc;
+    if ((rc = persistent_grid(dev, dtype, fused, (int)slots, &grid))) return rc;
     sms = device_cache(dev)->sms;
     if (ws) {
       if (prm.workspace_bytes < L.total)
@@ -242,8 +253,12 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.rcount = (unsigned int*)((char*)ws + L.rcount);
   a.best_key = (unsigned long long*)((char*)ws + L.best_key);
   a.rorder = (unsigned short*)((char*)ws + L.rorder);
-  a.barrier = (unsigned int*)((char*)ws + L.barrier);
   a.ticket = (unsigned int*)((char*)ws + L.ticket);
+  a.rowres = (RowRes*)((char*)ws + L.rowres);
+  a.rowcnt = (unsigned int*)((char*)ws + L.rowcnt);
+  a.reqcnt = (unsigned int*)((char*)ws + L.reqcnt);
+  a.pubq = (unsigned int*)((char*)ws + L.pubq);
+  a.ctl = (unsigned int*)((char*)ws + L.ctl);
   a.seed = seed;
   a.B = B;
   a.D_max = D_max;
@@ -257,8 +272,9 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   // segments to spread; else the scan, then race items over the whole GPU
   const bool spread = B < sms && (long long)B * nseg > sms;
   a.per_request = tail_bits == SV_TAIL_PER_REQUEST ? 1 : tail_bits == SV_TAIL_ITEMS ? 0 : (spread ? 0 : 1);
-  // the fused kernel takes whole segments; the split path cuts them while one wave holds them
-  a.rsplit = fused || a.per_request ? 1 : race_split(B, nseg, dtype, sms);
+  // the fused kernel races half segments; the split path cuts them while one wave holds them
+  a.rsplit = fused ? kMaxRaceSplit : a.per_request ? 1 : race_split(B, nseg, dtype, sms);
+  a.race_sm_every = fused ? fused_race_sm_every(a, grid) : 0;
   a.temperature = temperature;
   a.saguaro_k = k;
   a.saguaro_c = c;
@@ -266,14 +282,21 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
 
   cudaStream_t s = (cudaStream_t)prm.stream;
   cudaEvent_t* ev = (cudaEvent_t*)prm.timing_events;
+  if (prm.epilogue) {
+    const sv_epilogue_args& ep = *prm.epilogue;
+    const char* why = nullptr;
+    if (epilogue_check(ep.window, out_tokens, out_accept_len, B, D_max, ep.next_window, ep.seq,
+                       ep.seq_cap, ep.seq_len, &why) != SV_OK)
+      return fail(SV_ERR_INVALID_ARG, "sv_params.epilogue: %s", why);
+  }
   if (fused) {
-    // the fused kernel's grid barriers start at zero
+    // the fused kernel's counters, queue and tickets start at zero
     if ((e = cudaMemsetAsync((char*)ws + L.zero, 0, L.total - L.zero, s)) != cudaSuccess)
-      return cuda_fail(e, "cudaMemsetAsync(barriers)");
+      return cuda_fail(e, "cudaMemsetAsync(fused bookkeeping)");
     if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_fused(a, s, grid)) != cudaSuccess) return cuda_fail(e, "fused launch");
     if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    return SV_OK;
+    return run_epilogue(prm, out_tokens, out_accept_len, B, D_max, status, s);
   }
   const bool tickets = row_stats_tickets(a, grid);
   if (tickets && (e = cudaMemsetAsync(a.ticket, 0, 8 * 128, s)) != cudaSuccess)
@@ -284,11 +307,11 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if (a.per_request) {
     if ((e = launch_requests(a, s)) != cudaSuccess) return cuda_fail(e, "scan and race launch");
-    return SV_OK;
+  } else {
+    if ((e = launch_scan(a, s)) != cudaSuccess) return cuda_fail(e, "accept scan launch");
+    if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");
   }
-  if ((e = launch_scan(a, s)) != cudaSuccess) return cuda_fail(e, "accept scan launch");
-  if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");
-  return SV_OK;
+  return run_epilogue(prm, out_tokens, out_accept_len, B, D_max, status, s);
 }
 
 int sv_verify(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
@@ -303,6 +326,29 @@ int sv_verify_greedy(const void* target_logits, const int32_t* draft_tokens,
                      int32_t* out_tokens, int32_t* out_accept_len) {
   return sv_verify_ex(target_logits, nullptr, draft_tokens, row_D, B, D_max, V, dtype, 1.0f,
                       SV_GREEDY, 0, out_tokens, out_accept_len, nullptr);
+}
+
+int sv_epilogue(const int32_t* window, const int32_t* out_tokens, const int32_t* out_accept_len,
+                int B, int D_max, int32_t* next_window, int32_t* seq, int seq_cap,
+                int32_t* seq_len, uint32_t* flags, void* stream) {
+  g_last_error.clear();
+  const char* why = nullptr;
+  if (epilogue_check(window, out_tokens, out_accept_len, B, D_max, next_window, seq, seq_cap,
+                     seq_len, &why) != SV_OK)
+    return fail(SV_ERR_INVALID_ARG, "sv_epilogue: %s", why);
+  if (B == 0) return SV_OK;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  unsigned int* status = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    const int rc = status_word(dev, &status);
+    if (rc) return rc;
+  }
+  e = launch_epilogue(window, out_tokens, out_accept_len, B, D_max, next_window, seq, seq_cap,
+                      seq_len, flags, status, (cudaStream_t)stream);
+  return e == cudaSuccess ? SV_OK : cuda_fail(e, "epilogue launch");
 }
 
 int sv_get_device_status(void* stream, uint32_t* status_bits) {

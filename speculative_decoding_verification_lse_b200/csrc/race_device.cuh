@@ -209,6 +209,50 @@ __device__ __forceinline__ uint32_t word_filter(const uint4 (&raw)[32 / Lanes<DT
   return drop;
 }
 
+// word_filter with Philox's ten rounds in a loop (the round keys advanced in
+// place) over the group's eight counters at once: the same drop word from a
+// body a fraction of the unrolled one's size, for code that shares the
+// instruction cache with the statistics pass.
+template <int DT>
+__device__ __forceinline__ uint32_t word_filter_compact(const uint4 (&raw)[32 / Lanes<DT>::VEC],
+                                                        int j0, uint64_t seed, uint32_t g, int v0,
+                                                        float k2, float cup) {
+  constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC, NC = 8;  // eight blocks of four tokens
+  uint4 c[NC];
+#pragma unroll
+  for (int n = 0; n < NC; ++n) {
+    const int jj = n / (VEC / 4), h = n % (VEC / 4);
+    c[n] = make_uint4((uint32_t)((v0 + 32 * (j0 + jj)) * VEC + 4 * h) >> 2, g, 1u, 0u);
+  }
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+#pragma unroll 1
+  for (int r = 0; r < 10; ++r) {
+#pragma unroll
+    for (int n = 0; n < NC; ++n) philox_round(c[n], k0, k1);
+    k0 += kWeylA;
+    k1 += kWeylB;
+  }
+  const float2 kk = make_float2(k2, k2), cc = make_float2(cup, cup);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  uint32_t drop = 0u;
+#pragma unroll
+  for (int n = 0; n < NC; ++n) {
+    const int jj = n / (VEC / 4), h = n % (VEC / 4);
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const float2 z = make_float2(elem<DT>(raw[jj], 4 * h + e), elem<DT>(raw[jj], 4 * h + e + 1));
+      const float2 F = __fadd2_ru(__ffma2_ru(z, kk, cc), magic);
+      const uint32_t oa = e == 0 ? c[n].x : c[n].z, ob = e == 0 ? c[n].y : c[n].w;
+      const int ta = __float_as_int(F.x) - msb_index(oa) - (0x4B400000 + 1);
+      const int tb = __float_as_int(F.y) - msb_index(ob) - (0x4B400000 + 1);
+      drop = __funnelshift_l((uint32_t)ta, drop, 1);
+      drop = __funnelshift_l((uint32_t)tb, drop, 1);
+    }
+  }
+  (void)QV;
+  return drop;
+}
+
 // Vectors j0 .. j0 + NJ - 1 of one lane's part of segment `seg` (-inf past the
 // end of the row).
 template <int DT, int NJ>
@@ -422,6 +466,75 @@ __device__ __forceinline__ Best race_span_in(const VerifyArgs& a, const RaceDesc
     gi = ngi;
 #pragma unroll
     for (int j = 0; j < QV; ++j) cur[j] = nxt[j];
+  }
+  return warp_combine(B);
+}
+
+// Lane groups g0 .. g1 - 1 of segment `seg` of a race, by one warp, with a
+// small register budget (the fused kernel runs it beside the statistics pass
+// at three CTAs per multiprocessor): one 32-token group per lane in registers
+// at a time, no reference-key search beforehand.  The reference key K starts
+// at *best (the best exact key any finished part of the request published,
+// ordered bits; 0 = none) and, while it is unknown, is taken from the group
+// itself -- the best exact key among the lanes' largest logits of the group;
+// after each group it rises to the warp's best so far and *best.  Returns the
+// part's exact best and runner-up among the tokens that can reach K - delta
+// (all lanes), as race_segment_in does.
+template <int DT>
+__device__ __forceinline__ Best race_part(const VerifyArgs& a, const RaceDesc& rd,
+                                          const char* trow, const char* qrow, bool residual,
+                                          int seg, int g0, int g1,
+                                          const unsigned long long* best) {
+  constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC;
+  const int lane = threadIdx.x & 31;
+  const int v0 = seg * kSegVecs + lane;
+  unsigned long long bk = *(const volatile unsigned long long*)best;
+  double K = bk ? from_ordered_u64(bk) : -INFINITY;
+  Best B{-INFINITY, -INFINITY, -1};
+#pragma unroll 1
+  for (int gi = g0; gi < g1; ++gi) {
+    uint4 cur[QV];
+    load_part<DT>(a, trow, seg, gi * QV, cur);
+    if (!(K > -INFINITY)) {
+      float mv = -INFINITY;
+      int xi = -1;
+#pragma unroll
+      for (int j = 0; j < QV; ++j)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const float z = elem<DT>(cur[j], e);
+          if (z > mv) {
+            mv = z;
+            xi = (v0 + 32 * (gi * QV + j)) * VEC + e;
+          }
+        }
+      double k = -INFINITY;
+      if (xi >= 0 && xi < a.V) k = exact_key_of(a, rd, trow, qrow, residual, xi);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) k = fmax(k, __shfl_xor_sync(0xFFFFFFFFu, k, o));
+      K = k;
+    }
+    const float cup = filter_offset(K, rd.lse_t);
+    const float thr2 = K > -INFINITY ? __double2float_rd((K - kRaceBand) * 1.4426950408889634 - 1e-5)
+                                     : -INFINITY;
+    uint32_t keep = ~word_filter_compact<DT>(cur, gi * QV, a.seed, rd.g, v0, rd.k2, cup);
+    // exact keys of the survivors, one token per lane at a time
+    while (__any_sync(0xFFFFFFFFu, keep != 0u)) {
+      if (keep) {
+        const int t = __clz((int)keep);
+        keep &= ~(0x80000000u >> t);
+        const int x = (v0 + 32 * (gi * QV + t / VEC)) * VEC + t % VEC;
+        if (x < a.V && key2_upper(a, rd, trow, qrow, residual, x) >= thr2)
+          offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
+      }
+    }
+    if (gi + 1 < g1) {
+      double wb = B.best;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wb = fmax(wb, __shfl_xor_sync(0xFFFFFFFFu, wb, o));
+      bk = *(const volatile unsigned long long*)best;
+      K = fmax(K, fmax(wb, bk ? from_ordered_u64(bk) : -INFINITY));
+    }
   }
   return warp_combine(B);
 }

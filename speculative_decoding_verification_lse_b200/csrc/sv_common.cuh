@@ -41,7 +41,8 @@ enum : uint32_t {
   kFlagNonfinite = 1u << 10,
   kFlagBadParam = 1u << 11,
   kFlagErrors = kFlagBadToken | kFlagBadRowD | kFlagNonfinite | kFlagBadParam,
-  kStatusTimeout = 1u << 12   // a bounded wait of the fused kernel expired
+  kStatusTimeout = 1u << 12,  // a bounded wait of the fused kernel expired
+  kFlagSeqFull = 1u << 13     // the epilogue's append would pass the sequence capacity
 };
 
 // Partial statistics of one segment of one row (16 bytes).
@@ -122,14 +123,21 @@ struct VerifyArgs {
   unsigned int* rcount;    // [B] race segments finished (zeroed by the scan)
   unsigned long long* best_key;  // [B] best exact race key so far, ordered bits (set by the scan)
   unsigned short* rorder;  // [B, nseg] race segments by descending largest logit (set by the scan)
-  unsigned int* barrier;   // fused kernel: two grid barriers' counters (zero at launch)
-  unsigned int* ticket;    // statistics kernel with tickets: 8 counters, 32 words apart (zero at launch)
+  unsigned int* ticket;    // statistics tickets: 8 counters, 32 words apart (zero at launch)
+  // the fused kernel's bookkeeping (zero at launch, except rowres)
+  RowRes* rowres;          // [B, slots] merged rows
+  unsigned int* rowcnt;    // [B, slots] statistics items finished per row
+  unsigned int* reqcnt;    // [B] rows finished per request
+  unsigned int* pubq;      // [B] published races in order, as request index + 1
+  unsigned int* ctl;       // control words, one per 128-byte line (fused_verify.cu)
   uint64_t seed;
   int B, D_max, V, dtype;
   int nvec, nseg, slots;
   int mode;
   int per_request;         // after the statistics: 1 = one CTA per request, 0 = scan then race items
   int rsplit;              // race items per segment (1 or kMaxRaceSplit) in the race-items layout
+  int race_sm_every;       // fused kernel: while statistics remain, only multiprocessors whose
+                           // index is a multiple of this take race parts (0: every one)
   float temperature;
   int saguaro_k;
   float saguaro_c;
@@ -139,10 +147,13 @@ struct VerifyArgs {
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
 // [zero, total) must read zero when a fused launch starts.
 struct WsLayout {
-  size_t pstat, tpart, rdesc, rpart, rcount, best_key, rorder, zero, barrier, ticket, total;
+  size_t pstat, tpart, rdesc, rpart, rorder, rowres, zero, rcount, best_key, rowcnt, reqcnt, pubq,
+      ctl, ticket, total;
 };
 
-inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+constexpr int kCtlWords = 8 * 32;  // the fused kernel's control words, 32 words (128 B) apart
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline int vec_elems(int dtype) { return dtype == kF32 ? 4 : 8; }
 
@@ -166,15 +177,24 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
   L.rpart = off;
   off = align_up(off + (size_t)B * nseg * kMaxRaceSplit * sizeof(RacePart), 256);
+  L.rorder = off;
+  off = align_up(off + (size_t)B * nseg * sizeof(unsigned short), 256);
+  L.rowres = off;
+  off = align_up(off + (size_t)B * slots * sizeof(RowRes), 256);
+  // everything from here on reads zero when a fused launch starts
+  L.zero = off;
   L.rcount = off;
   off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
   L.best_key = off;
   off = align_up(off + (size_t)B * sizeof(unsigned long long), 256);
-  L.rorder = off;
-  off = align_up(off + (size_t)B * nseg * sizeof(unsigned short), 256);
-  L.zero = off;
-  L.barrier = off;
-  off = align_up(off + 2 * sizeof(unsigned int), 256);
+  L.rowcnt = off;
+  off = align_up(off + (size_t)B * slots * sizeof(unsigned int), 256);
+  L.reqcnt = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.pubq = off;
+  off = align_up(off + (size_t)B * sizeof(unsigned int), 256);
+  L.ctl = off;
+  off = align_up(off + kCtlWords * sizeof(unsigned int), 256);
   L.ticket = off;
   off = align_up(off + 8 * 128, 256);  // eight counters, one 128-byte line each
   L.total = off;
@@ -316,5 +336,13 @@ cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
 int race_split(int B, int nseg, int dtype, int sms);
 cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
-int fused_blocks_per_sm(int dtype);
+int fused_blocks_per_sm(int dtype, int slots);
+int fused_race_sm_every(const VerifyArgs& a, int grid);
+int epilogue_check(const int32_t* window, const int32_t* out_tokens, const int32_t* out_accept_len,
+                   int B, int D_max, const int32_t* next_window, const int32_t* seq, int seq_cap,
+                   const int32_t* seq_len, const char** why);
+cudaError_t launch_epilogue(const int32_t* window, const int32_t* out_tokens,
+                            const int32_t* out_accept_len, int B, int D_max, int32_t* next_window,
+                            int32_t* seq, int seq_cap, int32_t* seq_len, uint32_t* flags,
+                            unsigned* status, cudaStream_t s);
 }  // namespace sv

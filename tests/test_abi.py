@@ -168,3 +168,31 @@ def test_static_entry_point_checks_arguments_before_its_size(lib):
     rc = sv.sv_verify_static(fake, fake, fake, None, 4096, 7, 128256, sv.SV_BF16, 1.0,
                              sv.SV_STOCHASTIC, 0, fake, fake, None)
     assert rc == sv.SV_ERR_UNSUPPORTED and "sv_verify_static" in sv.sv_last_error()
+
+
+def test_epilogue_rejects_invalid_arguments_on_the_host(lib):
+    fake = 1 << 20  # never dereferenced: each call is rejected before any launch
+    cases = [
+        (dict(B=-1), "B must"),
+        (dict(D_max=33), "D_max"),
+        (dict(out_tokens=None), "non-NULL"),
+        (dict(window=None), "next_window needs window"),
+        (dict(seq_len=None), "seq needs seq_len"),
+        (dict(seq_cap=-1), "seq needs seq_len"),
+    ]
+    for kw, needle in cases:
+        a = dict(window=fake, out_tokens=fake, al=fake, B=4, D_max=3, next_window=fake, seq=fake,
+                 seq_cap=16, seq_len=fake)
+        a.update(kw)
+        rc = sv.sv_epilogue(a["window"], a["out_tokens"], a["al"], a["B"], a["D_max"],
+                            a["next_window"], a["seq"], a["seq_cap"], a["seq_len"])
+        assert rc == sv.SV_ERR_INVALID_ARG and needle in sv.sv_last_error(), kw
+    assert sv.sv_epilogue(None, None, None, 0, 3, None, None, 0, None) == sv.SV_OK
+    # the verification's own epilogue option is checked the same way, before any launch
+    p = sv.SvParams()
+    ep = sv.SvEpilogueArgs()
+    ep.next_window = fake
+    p.epilogue = ctypes.pointer(ep)
+    rc = sv.sv_verify_ex(fake, fake, fake, None, 2, 3, 100, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC, 0,
+                         fake, fake, p)
+    assert rc in (sv.SV_ERR_INVALID_ARG, sv.SV_ERR_CUDA)

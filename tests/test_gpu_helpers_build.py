@@ -1,5 +1,5 @@
 """The CUDA helpers that the GPU tests compile on the fly (the cuRAND Philox
-probe, the race word-filter probe and the grid-barrier probe, which include the
+probe, the race word-filter probe and the work-queue wait probe, which include the
 library's device headers)
 must keep compiling for sm_100a; nvcc works without a GPU, so this runs here."""
 import os
@@ -14,7 +14,7 @@ INC = os.path.join(ROOT, "include")
 
 
 @pytest.mark.parametrize("src", ["curand_philox_probe.cu", "race_filter_probe.cu",
-                                 "barrier_probe.cu"])
+                                 "queue_probe.cu"])
 def test_gpu_test_helper_compiles(tmp_path, src):
     subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
                     "-shared", "-Xcompiler", "-fPIC", "-I", CSRC, "-I", INC,
