@@ -306,7 +306,9 @@ def run_ours(args):
                                 device_id=dev)
     sv.load()
     variant = {"auto": sv.SV_VARIANT_AUTO, "split": sv.SV_VARIANT_SPLIT,
-               "fused": sv.SV_VARIANT_FUSED}[args.variant]
+               "split-items": sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
+               "split-per-request": sv.SV_VARIANT_SPLIT | sv.SV_TAIL_PER_REQUEST,
+               "fused": sv.SV_VARIANT_FUSED, "cluster": sv.SV_VARIANT_CLUSTER}[args.variant]
 
     # every rank verifies its own batch (its own seed and request range)
     w = workloads.make(args.workload, dev, seed=workloads.CONFIGS[args.workload]["seed"] + 97 * rank)
@@ -461,10 +463,11 @@ def run_ours(args):
         peak, peak_kind = measured_peak()
         step_bytes = w.algorithmic_bytes()
         used_variant = args.variant if args.variant != "auto" else "split"
-        if used_variant == "fused":
-            kname, kbytes = "fused_verify", step_bytes
+        if used_variant in ("fused", "cluster"):
+            main = "fused_verify.cu" if used_variant == "fused" else "cluster_verify.cu"
+            kname, kbytes = main[:-3], step_bytes
             ksrc = ["speculative_decoding_verification_lse_b200/csrc/" + f
-                    for f in ("fused_verify.cu", "tail_device.cuh", "race_device.cuh", "scan_device.cuh",
+                    for f in (main, "tail_device.cuh", "race_device.cuh", "scan_device.cuh",
                               "stats_device.cuh", "sv_common.cuh", "philox.cuh")]
         else:
             # the statistics pass reads every needed logit row once
@@ -525,8 +528,9 @@ def run_ours(args):
                 f"untimed steps after the timed region, every step the same call")),
             # fused: one launch; split: statistics, then one kernel per request or
             # the scan and the race items (the library's rule, in include/specverify.h)
-            "gpu_launches": (1 if used_variant == "fused" else
-                             3 if tail_items(w, torch.cuda.get_device_properties(dev).multi_processor_count)
+            "gpu_launches": (1 if used_variant in ("fused", "cluster") else
+                             3 if (used_variant == "split-items" or (used_variant == "split" and tail_items(
+                                 w, torch.cuda.get_device_properties(dev).multi_processor_count)))
                              else 2) * args.steps,
             "e2e": e2e,
             "acceptance": acceptance,
@@ -547,7 +551,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="b256")
-    ap.add_argument("--variant", choices=["auto", "split", "fused"], default="auto")
+    ap.add_argument("--variant", choices=["auto", "split", "split-items", "split-per-request",
+                                          "fused", "cluster"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

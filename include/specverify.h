@@ -91,7 +91,7 @@ enum { SV_STOCHASTIC = 0, SV_GREEDY = 1, SV_SAGUARO = 2 };
 /* return codes */
 enum { SV_OK = 0, SV_ERR_INVALID_ARG = -1, SV_ERR_UNSUPPORTED = -2, SV_ERR_CUDA = -3 };
 
-/* sv_params.variant: the launch structure (AUTO, SPLIT or FUSED), optionally OR-ed
+/* sv_params.variant: the launch structure, optionally OR-ed
  * with one layout of the work after the statistics pass (both layouts give the
  * same results; without one, the library takes ITEMS when B is below the device's
  * multiprocessor count and B times the row's 8 KiB segments is above it, and
@@ -99,8 +99,16 @@ enum { SV_OK = 0, SV_ERR_INVALID_ARG = -1, SV_ERR_UNSUPPORTED = -2, SV_ERR_CUDA 
  *   SV_TAIL_PER_REQUEST: one CTA per request merges, scans and races it;
  *   SV_TAIL_ITEMS: one CTA per request merges and scans, then one warp per
  *     (request, segment of the sampled row) races -- per half segment while
- *     those items fit in one wave of the device's resident warps. */
-enum { SV_VARIANT_AUTO = 0, SV_VARIANT_SPLIT = 1, SV_VARIANT_FUSED = 2 };
+ *     those items fit in one wave of the device's resident warps.
+ * The structures (all give the same results):
+ *   SV_VARIANT_SPLIT: a persistent statistics kernel, then the layout above;
+ *   SV_VARIANT_FUSED: one persistent launch in which each request's merge,
+ *     scan and race run beside the statistics of later requests;
+ *   SV_VARIANT_CLUSTER: one launch, one thread-block cluster (up to 8 CTAs) per
+ *     request doing its statistics, merges, scan and race between cluster
+ *     barriers;
+ *   SV_VARIANT_AUTO: the library's choice for the shape. */
+enum { SV_VARIANT_AUTO = 0, SV_VARIANT_SPLIT = 1, SV_VARIANT_FUSED = 2, SV_VARIANT_CLUSTER = 3 };
 enum { SV_TAIL_PER_REQUEST = 1 << 4, SV_TAIL_ITEMS = 1 << 5 };
 
 /* per-request flag bits (sv_params.out_flags) */

@@ -142,7 +142,7 @@ int check_args(const void* target_logits, const void* draft_logits, const int32_
     return fail(SV_ERR_INVALID_ARG, "saguaro_c must be in (0, 1] (got %g)", (double)c);
   const int tail_bits = prm.variant & (SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
   const int base_variant = prm.variant & ~(SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
-  if (base_variant < SV_VARIANT_AUTO || base_variant > SV_VARIANT_FUSED ||
+  if (base_variant < SV_VARIANT_AUTO || base_variant > SV_VARIANT_CLUSTER ||
       tail_bits == (SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS))
     return fail(SV_ERR_INVALID_ARG, "unknown variant %d", prm.variant);
   if (B == 0) return SV_OK;
@@ -288,6 +288,12 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     if (epilogue_check(ep.window, out_tokens, out_accept_len, B, D_max, ep.next_window, ep.seq,
                        ep.seq_cap, ep.seq_len, &why) != SV_OK)
       return fail(SV_ERR_INVALID_ARG, "sv_params.epilogue: %s", why);
+  }
+  if (base_variant == SV_VARIANT_CLUSTER) {
+    if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = launch_cluster(a, s)) != cudaSuccess) return cuda_fail(e, "cluster launch");
+    if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    return run_epilogue(prm, out_tokens, out_accept_len, B, D_max, status, s);
   }
   if (fused) {
     // the fused kernel's counters, queue and tickets start at zero

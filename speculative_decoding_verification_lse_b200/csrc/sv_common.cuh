@@ -27,6 +27,8 @@ constexpr int kMaxTopK = 8;
 constexpr int kMaxRaceSplit = 2;    // race items per segment, at most
 constexpr int kMaxSegs = 1024;       // segments per row (V up to 2^21 bf16 / 2^20 fp32)
 constexpr int kScanWarps = 4;        // requests per accept-scan CTA
+constexpr int kClusterMax = 8;       // CTAs per request in the cluster variant (portable limit)
+constexpr int kClusterParts = kClusterMax * kThreads / 32;  // race results per request there
 
 enum : int { kF32 = 0, kBF16 = 1 };
 enum : int { kStochastic = 0, kGreedy = 1, kSaguaro = 2 };
@@ -176,7 +178,9 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   L.rdesc = off;
   off = align_up(off + (size_t)B * sizeof(RaceDesc), 256);
   L.rpart = off;
-  off = align_up(off + (size_t)B * nseg * kMaxRaceSplit * sizeof(RacePart), 256);
+  const size_t parts = (size_t)nseg * kMaxRaceSplit > (size_t)kClusterParts
+                           ? (size_t)nseg * kMaxRaceSplit : (size_t)kClusterParts;
+  off = align_up(off + (size_t)B * parts * sizeof(RacePart), 256);
   L.rorder = off;
   off = align_up(off + (size_t)B * nseg * sizeof(unsigned short), 256);
   L.rowres = off;
@@ -338,6 +342,8 @@ cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);
+cudaError_t launch_cluster(const VerifyArgs& a, cudaStream_t s);
+int cluster_size(const VerifyArgs& a);
 int epilogue_check(const int32_t* window, const int32_t* out_tokens, const int32_t* out_accept_len,
                    int B, int D_max, const int32_t* next_window, const int32_t* seq, int seq_cap,
                    const int32_t* seq_len, const char** why);

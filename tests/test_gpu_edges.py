@@ -15,12 +15,12 @@ from speculative_decoding_verification_lse_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
 
-# both launch structures, each with both layouts of the work after the statistics
+# every launch structure, the split one with each layout of the work after the statistics
 VARIANTS = pytest.mark.parametrize(
     "variant",
     [sv.SV_VARIANT_SPLIT | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
-     sv.SV_VARIANT_FUSED | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_FUSED | sv.SV_TAIL_ITEMS],
-    ids=["split-per-request", "split-items", "fused-per-request", "fused-items"])
+     sv.SV_VARIANT_FUSED, sv.SV_VARIANT_CLUSTER],
+    ids=["split-per-request", "split-items", "fused", "cluster"])
 
 
 def make_random(B, D, V, dtype=sv.SV_BF16, seed=0, draft_sd=1.0, T=1.0, mode=0):

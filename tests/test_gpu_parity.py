@@ -16,12 +16,12 @@ from gpu_util import compare, gpu_run, oracle_on
 
 pytestmark = pytest.mark.gpu
 
-# both launch structures, each with both layouts of the work after the statistics
+# every launch structure, the split one with each layout of the work after the statistics
 VARIANTS = pytest.mark.parametrize(
     "variant",
     [sv.SV_VARIANT_SPLIT | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
-     sv.SV_VARIANT_FUSED | sv.SV_TAIL_PER_REQUEST, sv.SV_VARIANT_FUSED | sv.SV_TAIL_ITEMS],
-    ids=["split-per-request", "split-items", "fused-per-request", "fused-items"])
+     sv.SV_VARIANT_FUSED, sv.SV_VARIANT_CLUSTER],
+    ids=["split-per-request", "split-items", "fused", "cluster"])
 
 
 @VARIANTS
@@ -101,7 +101,7 @@ def test_full_size_is_deterministic_and_variants_agree(sv):
     runs = [gpu_run(w, seed=3, variant=v)
             for v in (sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED,
                       sv.SV_VARIANT_FUSED, sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
-                      sv.SV_VARIANT_FUSED | sv.SV_TAIL_ITEMS, sv.SV_VARIANT_AUTO)]
+                      sv.SV_VARIANT_CLUSTER, sv.SV_VARIANT_CLUSTER, sv.SV_VARIANT_AUTO)]
     for r in runs[1:]:
         for k in runs[0]:
             assert np.array_equal(runs[0][k], r[k], equal_nan=True), k

@@ -7,7 +7,7 @@ kernels with a fixed scratch array that lives in the library's own device
 memory.  Here it is called through the C ABI and checked against the ordinary
 entry point, sv_verify_ex with its own workspace, on two calls in a row (the
 array keeps the previous call's contents, so the second call shows that every
-call clears what it needs), in both kernel variants.  This file is collected
+call clears what it needs), in every launch structure.  This file is collected
 last so that a run stopping at its first failure has run every other test."""
 import ctypes
 
@@ -42,7 +42,8 @@ def _call(fn, w, seed, variant):
     return {k: v.cpu().numpy() for k, v in out.items()}
 
 
-@pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED], ids=["split", "fused"])
+@pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED, sv.SV_VARIANT_CLUSTER],
+                         ids=["split", "fused", "cluster"])
 @pytest.mark.parametrize("name", ["b256", "ragged", "saguaro", "tiny"])
 def test_static_entry_point_matches_the_ordinary_one(variant, name):
     sv.load()
