@@ -66,6 +66,13 @@ def _declare(L):
                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                ctypes.c_void_p, ctypes.c_void_p]
     L.svo_epilogue.restype = ctypes.c_int
+    L.svo_row_topk.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_void_p]
+    L.svo_row_topk.restype = None
+    L.svo_ssd_lookup.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    L.svo_ssd_lookup.restype = ctypes.c_int
     L.svo_has_openmp.argtypes = []
     L.svo_has_openmp.restype = ctypes.c_int
     return L
@@ -190,3 +197,34 @@ def epilogue(window, out_tokens, accept_len, seq=None, seq_len=None, *, next_win
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
     bits = np.array([(full[b // 32] >> (b % 32)) & 1 for b in range(B)], bool)
     return dict(next_window=nw, seq=sq, seq_len=sl, full=bits)
+
+
+def row_topk(row, k, L=None):
+    """Indices of the k largest logits of a row (logit desc, index asc)."""
+    row = np.ascontiguousarray(row)
+    idx = np.empty(k, np.int32)
+    (L or lib()).svo_row_topk(_ptr(row), row.shape[-1], _dtype_code(row), int(k), _ptr(idx))
+    return idx
+
+
+def ssd_lookup(out_tokens, accept_len, keys_al, keys_token, spec=None, L=None):
+    """The outcome lookup (svo_ssd_lookup).  out_tokens [B, D_max+1], accept_len [B],
+    keys_al / keys_token [B, K], spec [B, K, S] or None.
+    Returns dict(hit [B], spec [B, S] or None)."""
+    out_tokens = np.ascontiguousarray(out_tokens, dtype=np.int32)
+    B, W = out_tokens.shape
+    accept_len = np.ascontiguousarray(accept_len, dtype=np.int32).reshape(B)
+    keys_al = np.ascontiguousarray(keys_al, dtype=np.int32).reshape(B, -1)
+    keys_token = np.ascontiguousarray(keys_token, dtype=np.int32).reshape(B, -1)
+    K = keys_al.shape[1]
+    S = 0
+    if spec is not None:
+        spec = np.ascontiguousarray(spec, dtype=np.int32).reshape(B, K, -1)
+        S = spec.shape[2]
+    hit = np.empty(B, np.int32)
+    osp = np.empty((B, S), np.int32) if spec is not None else None
+    rc = (L or lib()).svo_ssd_lookup(_ptr(out_tokens), _ptr(accept_len), B, W - 1, _ptr(keys_al),
+                                     _ptr(keys_token), K, _ptr(spec), S, _ptr(hit), _ptr(osp))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (rc={rc})")
+    return dict(hit=hit, spec=osp)

@@ -493,6 +493,41 @@ int svo_epilogue(const int32_t* window, const int32_t* out_tokens, const int32_t
   return 0;
 }
 
+/* ---------------------------------------------------------------- SSD lookup */
+
+void svo_row_topk(const void* row, int V, int dtype, int k, int* idx) {
+  row_topk(row, V, dtype, k, idx);
+}
+
+/* "Speculative Speculative Decoding – асинхронизируй это.": the speculations
+ * prepared during verification are keyed by the verification outcome; a hit
+ * returns the prepared speculation, a miss returns nothing (the page's
+ * fallbacks -- a random token, n-grams -- are left to the caller).  Reading:
+ * the outcome is the accepted length with the token the verifier emitted
+ * after the accepted drafts; the first matching key wins. */
+int svo_ssd_lookup(const int32_t* out_tokens, const int32_t* accept_len, int B, int D_max,
+                   const int32_t* keys_al, const int32_t* keys_token, int K, const int32_t* spec,
+                   int S, int32_t* out_hit, int32_t* out_spec) {
+  if (B < 0 || D_max < 0 || K < 0 || S < 0) return -1;
+  if (B > 0 && (!out_tokens || !accept_len || !out_hit)) return -1;
+  if (B > 0 && K > 0 && (!keys_al || !keys_token)) return -1;
+  if (out_spec && S > 0 && !spec) return -1;
+  for (int b = 0; b < B; ++b) {
+    const int32_t AL = accept_len[b];
+    int hit = -1;
+    if (AL >= 1 && AL <= D_max + 1) {
+      const int32_t tok = out_tokens[(size_t)b * (size_t)(D_max + 1) + (size_t)(AL - 1)];
+      for (int k = 0; k < K && hit < 0; ++k)
+        if (keys_al[(size_t)b * K + k] == AL && keys_token[(size_t)b * K + k] == tok) hit = k;
+    }
+    out_hit[b] = hit;
+    if (out_spec)
+      for (int j = 0; j < S; ++j)
+        out_spec[(size_t)b * S + j] = hit >= 0 ? spec[((size_t)b * K + hit) * S + j] : -1;
+  }
+  return 0;
+}
+
 int svo_has_openmp(void) {
 #ifdef _OPENMP
   return 1;

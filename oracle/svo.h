@@ -113,6 +113,31 @@ int svo_epilogue(const int32_t* window, const int32_t* out_tokens, const int32_t
                  int B, int D_max, int32_t* next_window, int32_t* seq, int seq_cap,
                  int32_t* seq_len, uint32_t* full);
 
+/*
+ * The k largest logits of a row, by (logit descending, index ascending):
+ * idx[0..k-1].  ("Speculative Speculative Decoding – асинхронизируй это.",
+ * saguaro recipe item 1: the draft's most likely tokens.)  k <= V.
+ */
+void svo_row_topk(const void* row, int V, int dtype, int k, int* idx);
+
+/*
+ * Outcome lookup of speculative speculative decoding ("Speculative Speculative
+ * Decoding – асинхронизируй это.": while the target verifies, the draft
+ * predicts likely verification outcomes and prepares speculations for them; if
+ * the actual outcome is in the prepared set, its speculation is returned at
+ * once -- the cache hit of the page's restaurant analogy -- else it is a miss).
+ * The outcome of request b is (AL, token) = (accept_len[b], out_tokens[b][AL-1]);
+ * the prepared set is keys_al[b][0..K-1], keys_token[b][0..K-1].
+ *   out_hit[b] = the lowest k with keys_al[b][k] == AL and keys_token[b][k] ==
+ *                token, else -1 (also -1 when AL lies outside [1, D_max + 1]);
+ *   out_spec[b][0..S-1] = spec[b][out_hit[b]][0..S-1] on a hit, else -1
+ *                (when out_spec and spec are not NULL).
+ * Returns 0, or -1 for invalid arguments.
+ */
+int svo_ssd_lookup(const int32_t* out_tokens, const int32_t* accept_len, int B, int D_max,
+                   const int32_t* keys_al, const int32_t* keys_token, int K, const int32_t* spec,
+                   int S, int32_t* out_hit, int32_t* out_spec);
+
 /* 1 when built with OpenMP, else 0. */
 int svo_has_openmp(void);
 

@@ -57,6 +57,9 @@ MUTANTS = {
     "saguaro_topk_last_tie": ("if (best < 0 || z > bz) {", "if (best < 0 || z >= bz) {"),
     "epilogue_insert_one_late": ("row[AL - 1] = ot[AL - 1];", "if (AL < (int32_t)W) row[AL] = ot[AL - 1];"),
     "epilogue_no_shift": ("row[j] = window[(size_t)b * W + j + 1];", "row[j] = window[(size_t)b * W + j];"),
+    "ssd_ignores_accept_len": ("if (keys_al[(size_t)b * K + k] == AL && keys_token[(size_t)b * K + k] == tok) hit = k;",
+                               "if (keys_token[(size_t)b * K + k] == tok) hit = k;"),
+    "ssd_last_match_wins": ("for (int k = 0; k < K && hit < 0; ++k)", "for (int k = 0; k < K; ++k)"),
     "epilogue_append_drops_last": ("for (int j = 0; j < AL; ++j) seq", "for (int j = 0; j + 1 < AL; ++j) seq"),
 }
 
@@ -292,9 +295,24 @@ def check_epilogue(svo, L):
     return True
 
 
+def check_ssd(svo, L):
+    import test_oracle_ssd as ts
+
+    class Shim:
+        @staticmethod
+        def ssd_lookup(*a, **k):
+            return svo.ssd_lookup(*a, L=L, **k)
+    try:
+        ts.test_lookup_worked_example(Shim)
+        ts.test_lookup_against_a_dictionary(Shim)
+    except AssertionError:
+        return False
+    return True
+
+
 CHECKS = [check_lse, check_argmax, check_kat, check_engines, check_avalanche, check_uniform, check_p_eq_q, check_al_law,
           check_residual_law, check_bonus_law, lambda s, L: check_marginal(s, L, 0),
-          lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy, check_epilogue]
+          lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy, check_epilogue, check_ssd]
 
 
 def _build_variant(tmp, text):
