@@ -178,6 +178,10 @@ typedef struct sv_params {
   void* timing_events;               /* optional cudaEvent_t[2]: recorded on the stream
                                         immediately before and after the row-statistics
                                         kernel (split) or the fused kernel (fused) */
+  int32_t* out_draft_top;            /* [B, D_max, k] device, optional (k = min(saguaro_k, V)):
+                                        for each saguaro request, the k largest logits of each
+                                        draft row it tested (logit desc, index asc), the keys
+                                        of sv_ssd_lookup; -1 elsewhere */
   const sv_epilogue_args* epilogue;  /* optional: after the verification, on the same stream,
                                         the step sv_epilogue describes, on this call's
                                         out_tokens / out_accept_len (and out_flags, which get
@@ -271,6 +275,28 @@ SV_API int sv_verify_static(const void* target_logits, const void* draft_logits,
 SV_API int sv_epilogue(const int32_t* window, const int32_t* out_tokens,
                        const int32_t* out_accept_len, int B, int D_max, int32_t* next_window,
                        int32_t* seq, int seq_cap, int32_t* seq_len, uint32_t* flags, void* stream);
+
+/*
+ * sv_ssd_lookup: the outcome lookup of speculative speculative decoding
+ * ("Speculative Speculative Decoding – асинхронизируй это.": while the target
+ * verifies, the draft predicts likely verification outcomes and prepares a
+ * speculation for each; an outcome found among them returns its speculation at
+ * once -- the page's cache hit -- and any other is a miss).  The outcome of
+ * request b is (AL, token) = (out_accept_len[b], out_tokens[b][AL - 1]); its
+ * prepared set is keys_al[b][0..K-1], keys_token[b][0..K-1] (typically AL = d+1
+ * with the draft's top tokens at position d, sv_params.out_draft_top, on which
+ * saguaro sampling concentrates the correction).
+ *   out_hit[b]  = the lowest k with keys_al[b][k] == AL and keys_token[b][k] ==
+ *                 token; -1 if none, or if AL lies outside [1, D_max + 1].
+ *   out_spec[b] = spec[b][out_hit[b]][0..S-1] on a hit, else S values of -1
+ *                 (optional: out_spec and spec may be NULL).
+ * Arrays (device, caller-owned): out_tokens [B, D_max+1], out_accept_len,
+ * out_hit [B], keys_al, keys_token [B, K], spec [B, K, S], out_spec [B, S].
+ * Asynchronous on `stream`; host-detectable errors return a negative code. */
+SV_API int sv_ssd_lookup(const int32_t* out_tokens, const int32_t* out_accept_len, int B,
+                         int D_max, const int32_t* keys_al, const int32_t* keys_token, int K,
+                         const int32_t* spec, int S, int32_t* out_hit, int32_t* out_spec,
+                         void* stream);
 
 /* Bytes of scratch one call with these sizes needs (for sv_params.workspace). */
 SV_API size_t sv_workspace_bytes(int B, int D_max, int V, int dtype);

@@ -214,12 +214,14 @@ def ssd_lookup(out_tokens, accept_len, keys_al, keys_token, spec=None, L=None):
     out_tokens = np.ascontiguousarray(out_tokens, dtype=np.int32)
     B, W = out_tokens.shape
     accept_len = np.ascontiguousarray(accept_len, dtype=np.int32).reshape(B)
-    keys_al = np.ascontiguousarray(keys_al, dtype=np.int32).reshape(B, -1)
-    keys_token = np.ascontiguousarray(keys_token, dtype=np.int32).reshape(B, -1)
+    keys_al = np.ascontiguousarray(keys_al, dtype=np.int32)
+    keys_token = np.ascontiguousarray(keys_token, dtype=np.int32)
+    assert keys_al.shape == keys_token.shape and keys_al.shape[0] == B
     K = keys_al.shape[1]
     S = 0
     if spec is not None:
-        spec = np.ascontiguousarray(spec, dtype=np.int32).reshape(B, K, -1)
+        spec = np.ascontiguousarray(spec, dtype=np.int32)
+        assert spec.ndim == 3 and spec.shape[:2] == (B, K)
         S = spec.shape[2]
     hit = np.empty(B, np.int32)
     osp = np.empty((B, S), np.int32) if spec is not None else None

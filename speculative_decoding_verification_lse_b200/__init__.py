@@ -66,6 +66,7 @@ class SvParams(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t),
         ("timing_events", ctypes.c_void_p),
+        ("out_draft_top", ctypes.c_void_p),
         ("epilogue", ctypes.POINTER(SvEpilogueArgs)),
     ]
 
@@ -108,6 +109,10 @@ def load(build_if_needed=True):
                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     L.sv_epilogue.restype = ctypes.c_int
+    L.sv_ssd_lookup.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    L.sv_ssd_lookup.restype = ctypes.c_int
     L.sv_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.sv_workspace_bytes.restype = ctypes.c_size_t
     L.sv_get_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
@@ -179,6 +184,13 @@ def sv_epilogue(window, out_tokens, out_accept_len, B, D_max, next_window, seq, 
                               _stream_ptr(stream))
 
 
+def sv_ssd_lookup(out_tokens, out_accept_len, B, D_max, keys_al, keys_token, K, spec, S, out_hit,
+                  out_spec=None, stream=None):
+    return load().sv_ssd_lookup(_p(out_tokens), _p(out_accept_len), B, D_max, _p(keys_al),
+                                _p(keys_token), int(K), _p(spec), int(S), _p(out_hit),
+                                _p(out_spec), _stream_ptr(stream))
+
+
 def sv_workspace_bytes(B, D_max, V, dtype):
     return load().sv_workspace_bytes(B, D_max, V, dtype)
 
@@ -223,12 +235,13 @@ def _dtype_code(t):
 def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHASTIC, seed=0,
            temperature_per_req=None, mode_per_req=None, saguaro_k=5, saguaro_c=0.5,
            request_offset=0, variant=SV_VARIANT_AUTO, stream=None, row_lse=False,
-           out=None, workspace=None, timing_events=None, epilogue=None):
+           out=None, workspace=None, timing_events=None, epilogue=None, draft_top=False):
     """Verify a batch held in CUDA tensors; returns dict(tokens, accept_len, flags
     [, row_lse]) as CUDA tensors, enqueued on `stream` (not synchronised).
     epilogue: optional dict(window, next_window, seq, seq_len) of int32 CUDA
     tensors (any may be None) for the on-device step after verification
-    (sv_epilogue), run on the same stream."""
+    (sv_epilogue), run on the same stream.  draft_top: also return the k
+    largest logits of each saguaro draft row (sv_params.out_draft_top)."""
     import torch
     if not target.is_cuda:
         raise ValueError("target logits must be a CUDA tensor (there is no CPU path)")
@@ -254,6 +267,9 @@ def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHA
                    flags=torch.empty((B,), dtype=torch.int32, device=dev))
         if row_lse:
             out["row_lse"] = torch.empty((B, 2 * D + 1), dtype=torch.float32, device=dev)
+        if draft_top:
+            k = int(saguaro_k) if int(saguaro_k) > 0 else 5
+            out["draft_top"] = torch.empty((B, D, min(k, V)), dtype=torch.int32, device=dev)
     prm = SvParams()
     prm.stream = _stream_ptr(stream)
     prm.temperature_per_req = _p(temperature_per_req)
@@ -264,6 +280,7 @@ def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHA
     prm.request_offset = int(request_offset)
     prm.out_row_lse = _p(out.get("row_lse"))
     prm.out_flags = _p(out.get("flags"))
+    prm.out_draft_top = _p(out.get("draft_top"))
     if workspace is not None:
         prm.workspace = _p(workspace)
         prm.workspace_bytes = workspace.numel() * workspace.element_size()

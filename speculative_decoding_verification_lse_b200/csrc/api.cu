@@ -245,6 +245,7 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.out_al = out_accept_len;
   a.out_row_lse = prm.out_row_lse;
   a.out_flags = prm.out_flags;
+  a.out_draft_top = prm.out_draft_top;
   a.status = status;
   a.pstat = (PartStat*)((char*)ws + L.pstat);
   a.tpart = (TopPart*)((char*)ws + L.tpart);
@@ -355,6 +356,20 @@ int sv_epilogue(const int32_t* window, const int32_t* out_tokens, const int32_t*
   e = launch_epilogue(window, out_tokens, out_accept_len, B, D_max, next_window, seq, seq_cap,
                       seq_len, flags, status, (cudaStream_t)stream);
   return e == cudaSuccess ? SV_OK : cuda_fail(e, "epilogue launch");
+}
+
+int sv_ssd_lookup(const int32_t* out_tokens, const int32_t* out_accept_len, int B, int D_max,
+                  const int32_t* keys_al, const int32_t* keys_token, int K, const int32_t* spec,
+                  int S, int32_t* out_hit, int32_t* out_spec, void* stream) {
+  g_last_error.clear();
+  const char* why = nullptr;
+  if (ssd_lookup_check(out_tokens, out_accept_len, B, D_max, keys_al, keys_token, K, spec, S,
+                       out_hit, out_spec, &why) != SV_OK)
+    return fail(SV_ERR_INVALID_ARG, "sv_ssd_lookup: %s", why);
+  const cudaError_t e = launch_ssd_lookup(out_tokens, out_accept_len, B, D_max, keys_al,
+                                          keys_token, K, spec, S, out_hit, out_spec,
+                                          (cudaStream_t)stream);
+  return e == cudaSuccess ? SV_OK : cuda_fail(e, "ssd lookup launch");
 }
 
 int sv_get_device_status(void* stream, uint32_t* status_bits) {

@@ -197,6 +197,18 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* row
     err |= __reduce_or_sync(0xFFFFFFFFu, nonfinite);
   }
 
+  if (a.out_draft_top) {
+    // the k largest logits of each saguaro draft row tested (the speculation
+    // keys of "Speculative Speculative Decoding": the draft's top tokens)
+    const int k = a.saguaro_k;
+    for (int i = lane; i < Dm * k; i += 32) {
+      const int d = i / k, j = i - d * k;
+      int v = -1;
+      if (!err && saguaro && d < rp.Db && j < rows[Dm + 1 + d].ntop) v = rows[Dm + 1 + d].top[j];
+      a.out_draft_top[(size_t)b * Dm * k + i] = v;
+    }
+  }
+
   if (err) {
     for (int j = lane; j <= Dm; j += 32) ot[j] = -1;
     if (a.out_row_lse)

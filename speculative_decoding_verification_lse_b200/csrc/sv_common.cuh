@@ -117,6 +117,7 @@ struct VerifyArgs {
   int32_t* out_al;
   float* out_row_lse;
   uint32_t* out_flags;
+  int32_t* out_draft_top;  // [B, D_max, saguaro_k] optional: K of each saguaro draft row
   unsigned int* status;    // the device status word
   PartStat* pstat;         // [B, slots, nseg]
   TopPart* tpart;          // [B, D_max, nseg] (saguaro draft rows)
@@ -343,6 +344,14 @@ cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);
 cudaError_t launch_cluster(const VerifyArgs& a, cudaStream_t s);
+int ssd_lookup_check(const int32_t* out_tokens, const int32_t* out_accept_len, int B, int D_max,
+                     const int32_t* keys_al, const int32_t* keys_token, int K,
+                     const int32_t* spec, int S, const int32_t* out_hit, const int32_t* out_spec,
+                     const char** why);
+cudaError_t launch_ssd_lookup(const int32_t* out_tokens, const int32_t* out_accept_len, int B,
+                              int D_max, const int32_t* keys_al, const int32_t* keys_token, int K,
+                              const int32_t* spec, int S, int32_t* out_hit, int32_t* out_spec,
+                              cudaStream_t s);
 int cluster_size(const VerifyArgs& a);
 int epilogue_check(const int32_t* window, const int32_t* out_tokens, const int32_t* out_accept_len,
                    int B, int D_max, const int32_t* next_window, const int32_t* seq, int seq_cap,
