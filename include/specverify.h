@@ -298,6 +298,47 @@ SV_API int sv_ssd_lookup(const int32_t* out_tokens, const int32_t* out_accept_le
                          const int32_t* spec, int S, int32_t* out_hit, int32_t* out_spec,
                          void* stream);
 
+/*
+ * Verification with the vocabulary split across ranks (tensor-parallel logits):
+ * rank r of n_shards holds columns [r V_local, (r + 1) V_local) of every target
+ * and draft row, as [B, D_max+1, V_local] and [B, D_max, V_local] arrays; draft
+ * tokens and every token the calls write are global indices in
+ * [0, n_shards V_local).  ("Accélérer Sonar par la Spéculation", section
+ * "Calendrier Brouillon-Cible": the verification batch is synchronised with
+ * the tensor-parallel workers.)  Three calls per rank, with two all-gathers of
+ * byte buffers in rank order between them (the caller's collectives, e.g.
+ * NCCL over NVLink):
+ *   sv_shard_stats   -> exchange1 (sv_shard_exchange_bytes(.., 1) bytes per rank):
+ *                       the statistics of this rank's columns and the logits of
+ *                       the draft tokens it owns;
+ *   all-gather exchange1 of every rank -> gathered1 (n_shards x those bytes);
+ *   sv_shard_race    -> out_tokens (accepted prefix), out_accept_len, and
+ *                       sv_params' out_flags / out_row_lse / out_draft_top, the
+ *                       same on every rank; exchange2 (.., 2 bytes): this rank's
+ *                       race result per request;
+ *   all-gather exchange2 -> gathered2;
+ *   sv_shard_finish  -> the token at slot AL-1 of out_tokens (and out_flags).
+ * The accept decisions and the tokens follow the same rule, the same random
+ * numbers (the race's Philox words are those of the global token indices) and
+ * the same tie rules as sv_verify_ex on the whole rows; the statistics are
+ * merged over every rank's segments in global order, so they differ from an
+ * unsharded call only in rounding.  V_local must be a multiple of 4; every rank
+ * passes the same B, D_max, V_local, dtype, mode, seed and per-request arrays.
+ * sv_params.variant and .epilogue are ignored (run sv_epilogue afterwards).
+ * The calls use the library's workspace like sv_verify_ex; none synchronises. */
+SV_API size_t sv_shard_exchange_bytes(int B, int D_max, int V_local, int dtype, int stage);
+SV_API int sv_shard_stats(const void* target_local, const void* draft_local,
+                          const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max,
+                          int V_local, int dtype, float temperature, int mode, uint64_t seed,
+                          int n_shards, int shard, const sv_params* p, void* exchange1);
+SV_API int sv_shard_race(const void* target_local, const void* draft_local,
+                         const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max,
+                         int V_local, int dtype, float temperature, int mode, uint64_t seed,
+                         int n_shards, int shard, const sv_params* p, const void* gathered1,
+                         int32_t* out_tokens, int32_t* out_accept_len, void* exchange2);
+SV_API int sv_shard_finish(int B, int D_max, int n_shards, const void* gathered2,
+                           int32_t* out_tokens, const sv_params* p);
+
 /* Bytes of scratch one call with these sizes needs (for sv_params.workspace). */
 SV_API size_t sv_workspace_bytes(int B, int D_max, int V, int dtype);
 

@@ -113,6 +113,19 @@ def load(build_if_needed=True):
                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     L.sv_ssd_lookup.restype = ctypes.c_int
+    L.sv_shard_exchange_bytes.argtypes = [ctypes.c_int] * 5
+    L.sv_shard_exchange_bytes.restype = ctypes.c_size_t
+    L.sv_shard_stats.argtypes = _VERIFY_ARGS[:11] + [ctypes.c_int, ctypes.c_int,
+                                                     ctypes.POINTER(SvParams), ctypes.c_void_p]
+    L.sv_shard_stats.restype = ctypes.c_int
+    L.sv_shard_race.argtypes = _VERIFY_ARGS[:11] + [ctypes.c_int, ctypes.c_int,
+                                                    ctypes.POINTER(SvParams), ctypes.c_void_p,
+                                                    ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_void_p]
+    L.sv_shard_race.restype = ctypes.c_int
+    L.sv_shard_finish.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.POINTER(SvParams)]
+    L.sv_shard_finish.restype = ctypes.c_int
     L.sv_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.sv_workspace_bytes.restype = ctypes.c_size_t
     L.sv_get_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
@@ -189,6 +202,34 @@ def sv_ssd_lookup(out_tokens, out_accept_len, B, D_max, keys_al, keys_token, K, 
     return load().sv_ssd_lookup(_p(out_tokens), _p(out_accept_len), B, D_max, _p(keys_al),
                                 _p(keys_token), int(K), _p(spec), int(S), _p(out_hit),
                                 _p(out_spec), _stream_ptr(stream))
+
+
+def sv_shard_exchange_bytes(B, D_max, V_local, dtype, stage):
+    return load().sv_shard_exchange_bytes(B, D_max, V_local, dtype, stage)
+
+
+def sv_shard_stats(target_local, draft_local, draft_tokens, row_D, B, D_max, V_local, dtype,
+                   temperature, mode, seed, n_shards, shard, params, exchange1):
+    return load().sv_shard_stats(_p(target_local), _p(draft_local), _p(draft_tokens), _p(row_D),
+                                 B, D_max, V_local, dtype, temperature, mode, seed & (2**64 - 1),
+                                 n_shards, shard,
+                                 ctypes.byref(params) if params is not None else None,
+                                 _p(exchange1))
+
+
+def sv_shard_race(target_local, draft_local, draft_tokens, row_D, B, D_max, V_local, dtype,
+                  temperature, mode, seed, n_shards, shard, params, gathered1, out_tokens,
+                  out_accept_len, exchange2):
+    return load().sv_shard_race(_p(target_local), _p(draft_local), _p(draft_tokens), _p(row_D),
+                                B, D_max, V_local, dtype, temperature, mode, seed & (2**64 - 1),
+                                n_shards, shard,
+                                ctypes.byref(params) if params is not None else None,
+                                _p(gathered1), _p(out_tokens), _p(out_accept_len), _p(exchange2))
+
+
+def sv_shard_finish(B, D_max, n_shards, gathered2, out_tokens, params=None):
+    return load().sv_shard_finish(B, D_max, n_shards, _p(gathered2), _p(out_tokens),
+                                  ctypes.byref(params) if params is not None else None)
 
 
 def sv_workspace_bytes(B, D_max, V, dtype):

@@ -167,36 +167,36 @@ int check_args(const void* target_logits, const void* draft_logits, const int32_
 
 int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
-}  // namespace sv
+// The state of one call between its checks and its launches.
+struct Call {
+  VerifyArgs a;
+  WsLayout L;
+  void* ws;
+  unsigned int* status;
+  int grid, base_variant;
+  bool fused;
+};
 
-using namespace sv;
-
-extern "C" {
-
-int sv_version(void) { return 10000; }
-
-const char* sv_last_error(void) { return g_last_error.c_str(); }
-
-size_t sv_workspace_bytes(int B, int D_max, int V, int dtype) {
-  if (B < 0 || D_max < 0 || V < 1 || (dtype != SV_F32 && dtype != SV_BF16)) return 0;
-  return ws_layout(B, D_max, V, dtype, true).total;
-}
-
-int sv_verify_ex(const void* target_logits, const void* draft_logits,
+// Everything sv_verify_ex does before its launches: the argument checks, the
+// workspace, the device queries and the kernels' argument block.  V is the row
+// length (a shard's columns when the vocabulary is split, V_global = n_shards V,
+// offset = the shard's first column); B == 0 returns SV_OK with *empty set.
+int prepare_call(const void* target_logits, const void* draft_logits,
                  const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max, int V,
                  int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
-                 int32_t* out_accept_len, const sv_params* p) {
-  sv_params prm;
-  memset(&prm, 0, sizeof prm);
-  if (p) prm = *p;
-  g_last_error.clear();
+                 int32_t* out_accept_len, const sv_params& prm, int V_global, int offset,
+                 Call* call, bool* empty) {
+  *empty = false;
 
   {
     const int rc = check_args(target_logits, draft_logits, draft_tokens, B, D_max, V, dtype,
                               temperature, mode, out_tokens, out_accept_len, prm);
     if (rc != SV_OK) return rc;
   }
-  if (B == 0) return SV_OK;
+  if (B == 0) {
+    *empty = true;
+    return SV_OK;
+  }
   int k = prm.saguaro_k <= 0 ? 5 : prm.saguaro_k;
   if (k > V) k = V;
   const float c = prm.saguaro_c <= 0.0f ? 0.5f : prm.saguaro_c;
@@ -233,7 +233,7 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     }
   }
 
-  VerifyArgs a;
+  VerifyArgs& a = call->a;
   memset(&a, 0, sizeof a);
   a.target = target_logits;
   a.draft = draft_logits;
@@ -264,6 +264,8 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.B = B;
   a.D_max = D_max;
   a.V = V;
+  a.V_global = V_global;
+  a.vocab_offset = offset;
   a.dtype = dtype;
   a.nvec = nvec;
   a.nseg = nseg;
@@ -280,7 +282,53 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
   a.saguaro_k = k;
   a.saguaro_c = c;
   a.request_offset = prm.request_offset;
+  call->L = L;
+  call->ws = ws;
+  call->status = status;
+  call->grid = grid;
+  call->base_variant = base_variant;
+  call->fused = fused;
+  return SV_OK;
+}
 
+}  // namespace sv
+
+using namespace sv;
+
+extern "C" {
+
+int sv_version(void) { return 10000; }
+
+const char* sv_last_error(void) { return g_last_error.c_str(); }
+
+size_t sv_workspace_bytes(int B, int D_max, int V, int dtype) {
+  if (B < 0 || D_max < 0 || V < 1 || (dtype != SV_F32 && dtype != SV_BF16)) return 0;
+  return ws_layout(B, D_max, V, dtype, true).total;
+}
+
+int sv_verify_ex(const void* target_logits, const void* draft_logits,
+                 const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max, int V,
+                 int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
+                 int32_t* out_accept_len, const sv_params* p) {
+  sv_params prm;
+  memset(&prm, 0, sizeof prm);
+  if (p) prm = *p;
+  g_last_error.clear();
+  Call call;
+  bool empty = false;
+  {
+    const int rc = prepare_call(target_logits, draft_logits, draft_tokens, row_D, B, D_max, V,
+                                dtype, temperature, mode, seed, out_tokens, out_accept_len, prm, V,
+                                0, &call, &empty);
+    if (rc != SV_OK || empty) return rc;
+  }
+  VerifyArgs& a = call.a;
+  const WsLayout& L = call.L;
+  void* ws = call.ws;
+  unsigned int* status = call.status;
+  const int grid = call.grid, base_variant = call.base_variant;
+  const bool fused = call.fused;
+  cudaError_t e;
   cudaStream_t s = (cudaStream_t)prm.stream;
   cudaEvent_t* ev = (cudaEvent_t*)prm.timing_events;
   if (prm.epilogue) {
@@ -319,6 +367,126 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");
   }
   return run_epilogue(prm, out_tokens, out_accept_len, B, D_max, status, s);
+}
+
+size_t sv_shard_exchange_bytes(int B, int D_max, int V_local, int dtype, int stage) {
+  if (B < 0 || D_max < 0 || D_max > SV_MAX_DRAFT || V_local < 1 ||
+      (dtype != SV_F32 && dtype != SV_BF16) || (stage != 1 && stage != 2))
+    return 0;
+  const ShardLayout L = shard_layout(B, D_max, V_local, dtype);
+  return stage == 1 ? L.x1 : L.x2;
+}
+
+}  // extern "C"
+
+namespace {
+
+// The shard geometry: n_shards ranks of V_local columns each.
+int shard_check(int n_shards, int shard, int V_local, int dtype) {
+  if (n_shards < 1 || shard < 0 || shard >= n_shards)
+    return fail(SV_ERR_INVALID_ARG, "shard %d of %d is out of range", shard, n_shards);
+  if (V_local < 1 || V_local % 4)
+    return fail(SV_ERR_INVALID_ARG, "V_local must be a positive multiple of 4 (got %d)", V_local);
+  if ((long long)n_shards * V_local > 0x7FFFFFFFLL)
+    return fail(SV_ERR_UNSUPPORTED, "n_shards * V_local exceeds 2^31");
+  int nvec, nseg;
+  row_geometry(V_local, dtype == SV_F32 ? SV_F32 : SV_BF16, &nvec, &nseg);
+  if ((long long)nseg * n_shards > kMaxSegs)
+    return fail(SV_ERR_UNSUPPORTED, "n_shards * segments per shard exceeds %d", kMaxSegs);
+  return SV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sv_shard_stats(const void* target_local, const void* draft_local, const int32_t* draft_tokens,
+                   const int32_t* row_D, int B, int D_max, int V_local, int dtype,
+                   float temperature, int mode, uint64_t seed, int n_shards, int shard,
+                   const sv_params* p, void* exchange1) {
+  sv_params prm;
+  memset(&prm, 0, sizeof prm);
+  if (p) prm = *p;
+  prm.variant = SV_VARIANT_SPLIT;
+  prm.epilogue = nullptr;
+  g_last_error.clear();
+  int rc = shard_check(n_shards, shard, V_local, dtype);
+  if (rc != SV_OK) return rc;
+  if (B > 0 && !exchange1) return fail(SV_ERR_INVALID_ARG, "exchange1 is NULL");
+  // this stage writes no outputs; the exchange buffer stands in for them in the checks
+  Call call;
+  bool empty = false;
+  rc = prepare_call(target_local, draft_local, draft_tokens, row_D, B, D_max, V_local, dtype,
+                    temperature, mode, seed, (int32_t*)exchange1, (int32_t*)exchange1, prm,
+                    n_shards * V_local, shard * V_local, &call, &empty);
+  if (rc != SV_OK || empty) return rc;
+  VerifyArgs& a = call.a;
+  const ShardLayout X = shard_layout(B, D_max, V_local, dtype);
+  a.pstat = (PartStat*)((char*)exchange1 + X.parts);
+  a.tpart = (TopPart*)((char*)exchange1 + X.tops);
+  cudaStream_t s = (cudaStream_t)prm.stream;
+  cudaError_t e;
+  const bool tickets = row_stats_tickets(a, call.grid);
+  if (tickets && (e = cudaMemsetAsync(a.ticket, 0, 8 * 128, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync(ticket)");
+  if ((e = launch_row_stats(a, s, call.grid, tickets)) != cudaSuccess)
+    return cuda_fail(e, "row statistics launch");
+  if ((e = launch_shard_z(a, (char*)exchange1 + X.zx, s)) != cudaSuccess)
+    return cuda_fail(e, "owned logits launch");
+  return SV_OK;
+}
+
+int sv_shard_race(const void* target_local, const void* draft_local, const int32_t* draft_tokens,
+                  const int32_t* row_D, int B, int D_max, int V_local, int dtype,
+                  float temperature, int mode, uint64_t seed, int n_shards, int shard,
+                  const sv_params* p, const void* gathered1, int32_t* out_tokens,
+                  int32_t* out_accept_len, void* exchange2) {
+  sv_params prm;
+  memset(&prm, 0, sizeof prm);
+  if (p) prm = *p;
+  prm.variant = SV_VARIANT_SPLIT;
+  prm.epilogue = nullptr;
+  g_last_error.clear();
+  int rc = shard_check(n_shards, shard, V_local, dtype);
+  if (rc != SV_OK) return rc;
+  if (B > 0 && (!gathered1 || !exchange2))
+    return fail(SV_ERR_INVALID_ARG, "gathered1 and exchange2 must be non-NULL");
+  Call call;
+  bool empty = false;
+  rc = prepare_call(target_local, draft_local, draft_tokens, row_D, B, D_max, V_local, dtype,
+                    temperature, mode, seed, out_tokens, out_accept_len, prm, n_shards * V_local,
+                    shard * V_local, &call, &empty);
+  if (rc != SV_OK || empty) return rc;
+  const cudaError_t e =
+      launch_shard_tail(call.a, gathered1, n_shards, exchange2, (cudaStream_t)prm.stream);
+  return e == cudaSuccess ? SV_OK : cuda_fail(e, "shard scan and race launch");
+}
+
+int sv_shard_finish(int B, int D_max, int n_shards, const void* gathered2, int32_t* out_tokens,
+                    const sv_params* p) {
+  sv_params prm;
+  memset(&prm, 0, sizeof prm);
+  if (p) prm = *p;
+  g_last_error.clear();
+  if (B < 0) return fail(SV_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  if (D_max < 0 || D_max > SV_MAX_DRAFT)
+    return fail(SV_ERR_INVALID_ARG, "D_max must be in [0, %d] (got %d)", SV_MAX_DRAFT, D_max);
+  if (n_shards < 1) return fail(SV_ERR_INVALID_ARG, "n_shards must be >= 1 (got %d)", n_shards);
+  if (B == 0) return SV_OK;
+  if (!gathered2 || !out_tokens)
+    return fail(SV_ERR_INVALID_ARG, "gathered2 and out_tokens must be non-NULL");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  unsigned int* status = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    const int rc = status_word(dev, &status);
+    if (rc) return rc;
+  }
+  e = launch_shard_finish(gathered2, B, D_max, n_shards, out_tokens, prm.out_flags, status,
+                          (cudaStream_t)prm.stream);
+  return e == cudaSuccess ? SV_OK : cuda_fail(e, "shard finish launch");
 }
 
 int sv_verify(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,

@@ -83,15 +83,17 @@ __device__ __forceinline__ void philox_round(uint4& c, uint32_t k0, uint32_t k1)
 // i); the rest of the rounds are the published ones.
 struct RaceStream {
   PhiloxKey K;
+  uint32_t i0;    // counter of the row's first four tokens (vocabulary offset / 4)
   uint32_t x1;    // round-1 word 0: hi(B*1) ^ g ^ k0[0] = g ^ k0[0]
   uint32_t y2c;   // round-2 word 0 term: lo(B*1) ^ k0[1] = B ^ k0[1]
   uint32_t z2c;   // round-2 word 2 term: hi(A*x1) ^ k1[1]
   uint32_t w2;    // round-2 word 3: lo(A*x1)
 };
 
-__device__ __forceinline__ RaceStream race_stream(uint64_t seed, uint32_t g) {
+__device__ __forceinline__ RaceStream race_stream(uint64_t seed, uint32_t g, uint32_t i0 = 0) {
   RaceStream R;
   R.K = philox_key(seed);
+  R.i0 = i0;
   R.x1 = g ^ R.K.k0[0];
   R.y2c = kPhiloxMulB ^ R.K.k0[1];
   const unsigned long long pa = (unsigned long long)kPhiloxMulA * R.x1;
@@ -101,6 +103,7 @@ __device__ __forceinline__ RaceStream race_stream(uint64_t seed, uint32_t g) {
 }
 
 __device__ __forceinline__ uint4 race_words_fast(const RaceStream& R, uint32_t i) {
+  i += R.i0;
   // round 1 on (i, g, 1, 0)
   const unsigned long long pa = mul_wide(kPhiloxMulA, i);
   const uint32_t z1 = (uint32_t)(pa >> 32) ^ R.K.k1[0];

@@ -135,7 +135,8 @@ __device__ __forceinline__ double exact_key_of(const VerifyArgs& a, const RaceDe
   const float zt = (a.dtype == kF32) ? logit_at<kF32>(trow, x) : logit_at<kBF16>(trow, x);
   float zq = 0.0f;
   if (residual) zq = (a.dtype == kF32) ? logit_at<kF32>(qrow, x) : logit_at<kBF16>(qrow, x);
-  return exact_key(zt, zq, x, race_word(a.seed, rd.g, x), rd, residual);
+  const int gx = x + a.vocab_offset;  // the token's global index (Philox counter, saguaro K)
+  return exact_key(zt, zq, gx, race_word(a.seed, rd.g, gx), rd, residual);
 }
 
 constexpr double kRaceBand = 1e-5;  // delta: the 1e-6 near-tie band plus every rounding error
@@ -215,14 +216,14 @@ __device__ __forceinline__ uint32_t word_filter(const uint4 (&raw)[32 / Lanes<DT
 // instruction cache with the statistics pass.
 template <int DT>
 __device__ __forceinline__ uint32_t word_filter_compact(const uint4 (&raw)[32 / Lanes<DT>::VEC],
-                                                        int j0, uint64_t seed, uint32_t g, int v0,
-                                                        float k2, float cup) {
+                                                        int j0, uint64_t seed, uint32_t g,
+                                                        uint32_t i0, int v0, float k2, float cup) {
   constexpr int VEC = Lanes<DT>::VEC, QV = 32 / VEC, NC = 8;  // eight blocks of four tokens
   uint4 c[NC];
 #pragma unroll
   for (int n = 0; n < NC; ++n) {
     const int jj = n / (VEC / 4), h = n % (VEC / 4);
-    c[n] = make_uint4((uint32_t)((v0 + 32 * (j0 + jj)) * VEC + 4 * h) >> 2, g, 1u, 0u);
+    c[n] = make_uint4(i0 + ((uint32_t)((v0 + 32 * (j0 + jj)) * VEC + 4 * h) >> 2), g, 1u, 0u);
   }
   uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
 #pragma unroll 1
@@ -300,7 +301,7 @@ static __device__ __noinline__ float key2_upper(const VerifyArgs& a, const RaceD
       float lc = 0.0f;
       if (rd.ntop > 0) {
         bool in_k = false;
-        for (int i = 0; i < rd.ntop; ++i) in_k |= (rd.top[i] == x);
+        for (int i = 0; i < rd.ntop; ++i) in_k |= (rd.top[i] == x + a.vocab_offset);
         if (in_k) lc = (float)(rd.ln_c * 1.4426950408889634);
       }
       l2q += lc;
@@ -314,7 +315,7 @@ static __device__ __noinline__ float key2_upper(const VerifyArgs& a, const RaceD
       h = hl + fabsf(hl) * 0x1p-21f + 0x1p-40f;
     }
   }
-  const uint32_t o = race_word(a.seed, rd.g, x);
+  const uint32_t o = race_word(a.seed, rd.g, x + a.vocab_offset);
   const float lw = log2f((float)o + 0.5f);
   const float nlw = 32.0f - lw + fabsf(lw) * 0x1p-21f + 0x1p-20f;
   const float sum = l2p + h + nlw;
@@ -517,7 +518,8 @@ __device__ __forceinline__ Best race_part(const VerifyArgs& a, const RaceDesc& r
     const float cup = filter_offset(K, rd.lse_t);
     const float thr2 = K > -INFINITY ? __double2float_rd((K - kRaceBand) * 1.4426950408889634 - 1e-5)
                                      : -INFINITY;
-    uint32_t keep = ~word_filter_compact<DT>(cur, gi * QV, a.seed, rd.g, v0, rd.k2, cup);
+    uint32_t keep = ~word_filter_compact<DT>(cur, gi * QV, a.seed, rd.g,
+                                             (uint32_t)a.vocab_offset >> 2, v0, rd.k2, cup);
     // exact keys of the survivors, one token per lane at a time
     while (__any_sync(0xFFFFFFFFu, keep != 0u)) {
       if (keep) {
@@ -543,7 +545,7 @@ template <int DT>
 __device__ __noinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
                                           const char* trow, const char* qrow, bool residual,
                                           int seg, double K0, float cup) {
-  return race_segment_in<DT>(a, rd, race_stream(a.seed, rd.g), trow, qrow, residual, seg, K0, cup);
+  return race_segment_in<DT>(a, rd, race_stream(a.seed, rd.g, (uint32_t)a.vocab_offset >> 2), trow, qrow, residual, seg, K0, cup);
 }
 
 // A quick approximate key (natural-log units) with the hardware's approximate

@@ -36,15 +36,18 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 // segments l, l+32, ...; the partials were written by other warps, so they are
 // read through L2).  Every lane returns the same RowRes.
 //   LSE = ln2 * (Mk + log2 sum_s S_s 2^(m_s k2 - Mk)),  Mk = M k2, M = max_s m_s
-__device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg, bool lse,
-                                 float k2, int k, RowRes& r) {
+// PS(s) and TP(s): the partial and the top list of segment s (the row's
+// segments in order, wherever they are stored).
+template <class PS, class TP>
+__device__ inline void merge_row_at(PS ps_at, TP tp_at, bool has_tp, int nseg, bool lse, float k2,
+                                    int k, RowRes& r) {
   const int lane = threadIdx.x & 31;
   float mx = -INFINITY;
   int am = INT_MAX, ms = nseg;
   uint32_t bad = 0;
   double Sd = 0.0;  // relative to 2^(mx*k2)
   for (int s = lane; s < nseg; s += 32) {
-    const float4 raw = __ldcg(reinterpret_cast<const float4*>(ps + s));
+    const float4 raw = __ldcg(reinterpret_cast<const float4*>(ps_at(s)));
     const float m = raw.x, S = raw.y;
     const int ai = __float_as_int(raw.z);
     bad |= __float_as_uint(raw.w);
@@ -75,7 +78,7 @@ __device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg
     if (!bad) r.lse = (Mk + log2(S)) * kLn2d;
   }
   r.ntop = 0;
-  if (tp) {
+  if (has_tp) {
     // k rounds: each lane offers the best head of its segments' lists
     int head[kMaxSegs / 32];
     const int mine = (nseg - lane + 31) / 32;
@@ -85,7 +88,7 @@ __device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg
       int bi = -1;
       for (int i = 0; i < mine; ++i) {
         if (head[i] >= k) continue;
-        const TopPart* t = tp + lane + 32 * i;
+        const TopPart* t = tp_at(lane + 32 * i);
         const int ci = __ldcg(&t->i[head[i]]);
         if (ci == INT_MAX) continue;
         const unsigned long long kk = value_index_key(__ldcg(&t->v[head[i]]), ci);
@@ -105,6 +108,13 @@ __device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg
   r.bad = bad;
 }
 
+// A row whose segments' partials are consecutive at ps (and top lists at tp).
+__device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg, bool lse,
+                                 float k2, int k, RowRes& r) {
+  merge_row_at([=](int s) { return ps + s; }, [=](int s) { return tp + s; }, tp != nullptr, nseg,
+               lse, k2, k, r);
+}
+
 // Whether row `slot` of a request with parameters rp is read by the rule.
 __device__ __forceinline__ bool slot_needed(const VerifyArgs& a, int slot, const ReqParams& rp) {
   if (rp.err) return false;
@@ -113,21 +123,19 @@ __device__ __forceinline__ bool slot_needed(const VerifyArgs& a, int slot, const
   return is_t ? d <= rp.Db : (d < rp.Db && rp.mode != kGreedy);
 }
 
-// Merge row `slot` of request b (one full warp); lane 0 writes the result to dst.
-__device__ inline void merge_row_into(const VerifyArgs& a, int b, int slot, const ReqParams& rp,
-                                      RowRes* dst) {
-  const int Dm = a.D_max;
+// Merge row `slot` of request b (one full warp) from the partials PS(s) and
+// top lists TP(s) of its nseg segments (has_tp: a saguaro draft row); lane 0
+// writes the result to dst.
+template <class PS, class TP>
+__device__ inline void merge_into_at(const VerifyArgs& a, const ReqParams& rp, int slot, PS ps_at,
+                                     TP tp_at, bool has_tp, int nseg, RowRes* dst) {
   const bool greedy = rp.mode == kGreedy;
-  const bool is_t = slot <= Dm;
-  const int d = is_t ? slot : slot - Dm - 1;
   const float k2 = greedy ? 0.0f : log2e_over_T(rp.T);
-  const PartStat* ps = a.pstat + ((size_t)b * a.slots + slot) * a.nseg;
-  const TopPart* tp =
-      (!is_t && rp.mode == kSaguaro) ? a.tpart + ((size_t)b * Dm + d) * a.nseg : nullptr;
+  (void)slot;
   RowRes rr;
-  merge_row(ps, tp, a.nseg, !greedy, k2, a.saguaro_k, rr);
+  merge_row_at(ps_at, tp_at, has_tp, nseg, !greedy, k2, a.saguaro_k, rr);
   rr.lnZ = 0.0;
-  if (tp && !rr.bad) {
+  if (has_tp && !rr.bad) {
     // Z = 1 - (1 - c) * sum_{x in K} q(x)
     const double Td = (double)rp.T;
     double mass = 0.0;
@@ -135,6 +143,19 @@ __device__ inline void merge_row_into(const VerifyArgs& a, int b, int slot, cons
     rr.lnZ = log1p(-(1.0 - (double)a.saguaro_c) * mass);
   }
   if ((threadIdx.x & 31) == 0) *dst = rr;
+}
+
+// Merge row `slot` of request b from the workspace's partials.
+__device__ inline void merge_row_into(const VerifyArgs& a, int b, int slot, const ReqParams& rp,
+                                      RowRes* dst) {
+  const int Dm = a.D_max;
+  const bool is_t = slot <= Dm;
+  const int d = is_t ? slot : slot - Dm - 1;
+  const PartStat* ps = a.pstat + ((size_t)b * a.slots + slot) * a.nseg;
+  const TopPart* tp =
+      (!is_t && rp.mode == kSaguaro) ? a.tpart + ((size_t)b * Dm + d) * a.nseg : nullptr;
+  merge_into_at(a, rp, slot, [=](int s) { return ps + s; }, [=](int s) { return tp + s; },
+                tp != nullptr, a.nseg, dst);
 }
 
 // The scan's per-position inputs, which do not depend on the merged rows: lane
@@ -157,7 +178,7 @@ __device__ __forceinline__ ScanInputs scan_inputs(const VerifyArgs& a, int b, co
   in.err = rp.err;
   if (!rp.err && lane < rp.Db) {
     in.x = a.tokens[(size_t)b * a.D_max + lane];
-    if (in.x < 0 || in.x >= a.V) {
+    if (in.x < 0 || in.x >= a.V_global) {
       in.err |= kFlagBadToken;
     } else if (rp.mode != kGreedy) {
       in.zt = load_logit(a, row_base(a, b, lane), in.x);

@@ -115,7 +115,7 @@ __device__ __forceinline__ int key32_index(uint32_t k) { return (int)(0xFFFFu - 
 template <int DT, bool LSE, bool ARGMAX, bool TOP>
 __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], const char* row,
                                              int V, int seg, float k2, int topk, PartStat* out,
-                                             TopPart* tout) {
+                                             TopPart* tout, int off = 0) {
   constexpr int VEC = DT == kF32 ? 4 : 8;
   const int lane = threadIdx.x & 31;
   const int v0 = seg * kSegVecs + lane;
@@ -280,7 +280,7 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
         if (win != 0u && key == win) ++h;
         if (lane == 0) {
           tout->v[r] = win ? key32_value(win) : -INFINITY;
-          tout->i[r] = win ? base + key32_index(win) : INT_MAX;
+          tout->i[r] = win ? off + base + key32_index(win) : INT_MAX;
         }
       } else {
         const unsigned long long key = hi == INT_MAX ? 0ull : value_index_key(hv, hi);
@@ -288,7 +288,7 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
         if (win != 0ull && key == win) ++h;
         if (lane == 0) {
           tout->v[r] = win ? key_value(win) : -INFINITY;
-          tout->i[r] = win ? key_index(win) : INT_MAX;
+          tout->i[r] = win ? off + key_index(win) : INT_MAX;
         }
       }
     }
@@ -298,7 +298,7 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
     PartStat p;
     p.m = m_w;
     p.S = S_w;
-    p.argmax = idx_w;
+    p.argmax = idx_w == INT_MAX ? INT_MAX : off + idx_w;  // global index
     p.bad = bad_w;
     *out = p;
   }
@@ -310,7 +310,7 @@ __device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* r
                                               float k2, int topk, PartStat* out, TopPart* tout) {
   uint4 raw[kLaneVecs];
   load_segment<DT>(a, row, seg, raw);
-  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, row, a.V, seg, k2, topk, out, tout);
+  stats_reduce<DT, LSE, ARGMAX, TOP>(raw, row, a.V, seg, k2, topk, out, tout, a.vocab_offset);
 }
 
 // The statistics of a saguaro draft-row segment (with its top list), compiled

@@ -105,6 +105,23 @@ struct __align__(16) RacePart {
   int pad;
 };
 
+// Vocabulary-sharded verification: one rank's race result for one request
+// (exchanged between ranks; shard_verify.cu).
+struct __align__(16) ShardRace {
+  double best, second;    // the race of the request's kind on this rank's columns
+  double bbest, bsecond;  // the bonus race there, when no column here was a residual candidate
+  int idx, bidx;          // global token indices (-1: none)
+  int kind, n;            // from the accept scan (identical on every rank)
+  uint32_t flags;
+  int pad;
+};
+
+// Byte offsets of one rank's exchange 1 (partials, top lists, owned logits of
+// the draft tokens) and the sizes of both exchanges.
+struct ShardLayout {
+  size_t parts, tops, zx, x1, x2;
+};
+
 // Everything a kernel needs, passed by value.
 struct VerifyArgs {
   const void* target;
@@ -134,7 +151,9 @@ struct VerifyArgs {
   unsigned int* pubq;      // [B] published races in order, as request index + 1
   unsigned int* ctl;       // control words, one per 128-byte line (fused_verify.cu)
   uint64_t seed;
-  int B, D_max, V, dtype;
+  int B, D_max, V, dtype;   // V: the row length (this shard's columns when sharded)
+  int V_global;             // the vocabulary (V unless sharded)
+  int vocab_offset;         // global index of column 0 (0 unless sharded; a multiple of 4)
   int nvec, nseg, slots;
   int mode;
   int per_request;         // after the statistics: 1 = one CTA per request, 0 = scan then race items
@@ -344,6 +363,13 @@ cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);
 cudaError_t launch_cluster(const VerifyArgs& a, cudaStream_t s);
+ShardLayout shard_layout(int B, int D_max, int V_local, int dtype);
+cudaError_t launch_shard_z(const VerifyArgs& a, void* zx, cudaStream_t s);
+cudaError_t launch_shard_tail(const VerifyArgs& a, const void* gathered1, int n_shards,
+                              void* exchange2, cudaStream_t s);
+cudaError_t launch_shard_finish(const void* gathered2, int B, int D_max, int n_shards,
+                                int32_t* out_tokens, uint32_t* out_flags, unsigned* status,
+                                cudaStream_t s);
 int ssd_lookup_check(const int32_t* out_tokens, const int32_t* out_accept_len, int B, int D_max,
                      const int32_t* keys_al, const int32_t* keys_token, int K,
                      const int32_t* spec, int S, const int32_t* out_hit, const int32_t* out_spec,

@@ -196,3 +196,20 @@ def test_epilogue_rejects_invalid_arguments_on_the_host(lib):
     rc = sv.sv_verify_ex(fake, fake, fake, None, 2, 3, 100, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC, 0,
                          fake, fake, p)
     assert rc in (sv.SV_ERR_INVALID_ARG, sv.SV_ERR_CUDA)
+
+
+def test_shard_calls_reject_invalid_arguments_on_the_host(lib):
+    fake = 1 << 20  # never dereferenced
+    base = (fake, fake, fake, None, 4, 3, 1000, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC, 0)
+    for n, r, Vl, needle in ((2, 2, 1000, "out of range"), (0, 0, 1000, "out of range"),
+                             (2, 0, 1002, "multiple of 4")):
+        args = base[:6] + (Vl,) + base[7:]
+        rc = sv.sv_shard_stats(*args, n, r, None, fake)
+        assert rc == sv.SV_ERR_INVALID_ARG and needle in sv.sv_last_error(), (n, r, Vl)
+        rc = sv.sv_shard_race(*args, n, r, None, fake, fake, fake, fake)
+        assert rc == sv.SV_ERR_INVALID_ARG and needle in sv.sv_last_error(), (n, r, Vl)
+    rc = sv.sv_shard_stats(*base, 2, 0, None, None)
+    assert rc == sv.SV_ERR_INVALID_ARG and "exchange1" in sv.sv_last_error()
+    assert sv.sv_shard_finish(4, 3, 0, fake, fake) == sv.SV_ERR_INVALID_ARG
+    assert sv.sv_shard_exchange_bytes(4, 3, 1000, sv.SV_BF16, 1) > 0
+    assert sv.sv_shard_exchange_bytes(4, 3, 1000, sv.SV_BF16, 3) == 0

@@ -83,3 +83,49 @@ def test_two_gloo_ranks_reproduce_the_single_batch(tmp_path):
     ok = np.load(tmp_path / "ok.npy")
     assert ok[0], "sharded outputs differ from the single-batch outputs"
     assert ok[1], "max over ranks is wrong"
+
+
+def _vocab_rank_main(rank, world, port, out_dir):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from speculative_decoding_verification_lse_b200.sharding import (all_gather_bytes, vocab_shard,
+                                                                    vocab_shard_width)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = torch.Generator().manual_seed(5)
+        V = 1003
+        rows = torch.randn((4, V), generator=g) * 3  # the same on every rank
+        mine = vocab_shard(rows, rank, world)
+        Vl = vocab_shard_width(V, world)
+        # one exchange: this rank's partial (max, sum of exp) per row and its columns
+        m = mine.max(dim=-1).values
+        s = torch.exp(mine - m[:, None]).sum(dim=-1)
+        rec = torch.cat([m[:, None], s[:, None], mine], dim=1).contiguous()
+        got = all_gather_bytes(rec.view(torch.uint8).flatten())
+        parts = got.view(world, -1).view(torch.float32).view(world, 4, Vl + 2)
+        if rank == 0:
+            cols = torch.cat([parts[r, :, 2:] for r in range(world)], dim=1)[:, :V]
+            # the partials merged in rank order give the whole row's log-sum-exp
+            M = parts[:, :, 0].max(dim=0).values
+            S = (parts[:, :, 1] * torch.exp(parts[:, :, 0] - M[None])).sum(dim=0)
+            lse = (M + torch.log(S)).double()
+            want = torch.logsumexp(rows.double(), dim=-1)
+            np.save(os.path.join(out_dir, "vocab_ok.npy"),
+                    np.array([torch.equal(cols, rows),
+                              bool(torch.allclose(lse, want, rtol=1e-6, atol=1e-6))]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_the_vocabulary(tmp_path):
+    """The host side of vocabulary-parallel verification over gloo: each rank
+    cuts its columns (vocab_shard), the byte exchange (all_gather_bytes)
+    returns every rank's buffer in rank order, and partial (max, sum) pairs
+    merged in that order give the whole row's log-sum-exp."""
+    world = 2
+    mp.start_processes(_vocab_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    ok = np.load(tmp_path / "vocab_ok.npy")
+    assert ok[0], "gathered columns are out of rank order"
+    assert ok[1], "merged partials differ from the row's log-sum-exp"
