@@ -73,6 +73,12 @@ def _declare(L):
                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
     L.svo_ssd_lookup.restype = ctypes.c_int
+    L.svo_verify_tree.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+        ctypes.c_uint64, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p, ctypes.c_int]
+    L.svo_verify_tree.restype = ctypes.c_int
     L.svo_has_openmp.argtypes = []
     L.svo_has_openmp.restype = ctypes.c_int
     return L
@@ -230,3 +236,33 @@ def ssd_lookup(out_tokens, accept_len, keys_al, keys_token, spec=None, L=None):
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
     return dict(hit=hit, spec=osp)
+
+
+def verify_tree(target, draft, tokens, parents, n_nodes=None, *, temperature=1.0, mode=SVO_STOCHASTIC,
+                seed=0, request_offset=0, nthreads=1, L=None):
+    """Tree verification on host arrays (svo_verify_tree): target [B, N+1, V],
+    draft [B, N, V] (or None when greedy), tokens and parents [B, N] int32,
+    n_nodes [B] or None.  Returns dict(tokens [B, N+1], accept_len [B],
+    nodes [B, N], flags [B])."""
+    target = np.ascontiguousarray(target)
+    B, Np1, V = target.shape
+    N = Np1 - 1
+    dt = _dtype_code(target)
+    if draft is not None:
+        draft = np.ascontiguousarray(draft)
+        assert draft.dtype == target.dtype and draft.shape == (B, N, V)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, N)
+    parents = np.ascontiguousarray(parents, dtype=np.int32).reshape(B, N)
+    if n_nodes is not None:
+        n_nodes = np.ascontiguousarray(n_nodes, dtype=np.int32).reshape(B)
+    out_tokens = np.empty((B, N + 1), np.int32)
+    out_al = np.empty((B,), np.int32)
+    out_nodes = np.empty((B, N), np.int32)
+    out_flags = np.empty((B,), np.uint32)
+    rc = (L or lib()).svo_verify_tree(
+        _ptr(target), _ptr(draft), _ptr(tokens), _ptr(parents), _ptr(n_nodes), B, N, V, dt,
+        float(temperature), int(mode), int(seed) & (2**64 - 1), int(request_offset),
+        _ptr(out_tokens), _ptr(out_al), _ptr(out_nodes), _ptr(out_flags), int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (rc={rc})")
+    return dict(tokens=out_tokens, accept_len=out_al, nodes=out_nodes, flags=out_flags)

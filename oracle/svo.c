@@ -446,6 +446,231 @@ int svo_verify(const void* target, const void* draft, const int32_t* tokens,
   return 0;
 }
 
+/* ---------------------------------------------------------------- trees */
+
+/* The exponential race over an explicit distribution P (the candidates are the
+ * tokens with P(x) > 0): argmax of ln P(x) - ln E_x, ties to the lowest index. */
+static int race_vec(const double* P, int V, uint64_t seed, uint32_t g, double* gap) {
+  int best_x = -1;
+  double best = -INFINITY, second = -INFINITY;
+  for (int x = 0; x < V; ++x) {
+    if (!(P[x] > 0.0)) continue;
+    double key = log(P[x]) - log(svo_race_exponential(seed, g, (uint32_t)x));
+    if (key > best) {
+      second = best;
+      best = key;
+      best_x = x;
+    } else if (key > second) {
+      second = key;
+    }
+  }
+  *gap = best - second;
+  return best_x;
+}
+
+/* Softmax of one row at temperature T into P (0 for masked entries). */
+static void row_probs(const void* row, int V, int dtype, double T, double* P) {
+  const double lse = svo_row_lse(row, V, dtype, T);
+  for (int x = 0; x < V; ++x) P[x] = exp(logit_at(row, (size_t)x, dtype) / T - lse);
+}
+
+typedef struct {
+  const void* target;
+  const void* draft;
+  const int32_t* tokens;
+  const int32_t* parents;
+  const int32_t* n_nodes;
+  int B, N_max, V, dtype;
+  double T;
+  int mode;
+  uint64_t seed;
+  uint32_t request_offset;
+  int32_t* out_tokens;
+  int32_t* out_accept_len;
+  int32_t* out_nodes;
+  uint32_t* out_flags;
+} tree_args;
+
+/* One request's tree walk ("Accélérer Sonar par la Spéculation", section
+ * "EAGLE": several candidates per node).  Reading: the candidates at a node are
+ * tried in node order with the rule of "Speculative Speculative Decoding –
+ * асинхронизируй это." (items 1-3) applied recursively -- accept with
+ * probability min(1, P/q); on rejection the next candidate is tested against
+ * the normalised residual P = norm(max(0, P - q)), and after the last one the
+ * token is drawn from that residual -- which keeps the output distributed like
+ * p when the candidates are independent draws from q.  A chain (one child per
+ * node) is the linear rule. */
+static void verify_tree_one(const tree_args* a, int b) {
+  const int Nm = a->N_max, V = a->V, dt = a->dtype;
+  const uint32_t g = a->request_offset + (uint32_t)b;
+  int32_t* ot = a->out_tokens + (size_t)b * (size_t)(Nm + 1);
+  int32_t* on = a->out_nodes ? a->out_nodes + (size_t)b * (size_t)Nm : NULL;
+  const int32_t* tok = a->tokens + (size_t)b * (size_t)Nm;
+  const int32_t* par = a->parents + (size_t)b * (size_t)Nm;
+  uint32_t flags = 0;
+  for (int j = 0; j <= Nm; ++j) ot[j] = -1;
+  if (on)
+    for (int j = 0; j < Nm; ++j) on[j] = -1;
+  a->out_accept_len[b] = -1;
+
+  const int n = a->n_nodes ? a->n_nodes[b] : Nm;
+  if (n < 0 || n > Nm) {
+    flags |= SVO_FLAG_BAD_ROW_D;
+    goto done;
+  }
+  if (a->mode != SVO_STOCHASTIC && a->mode != SVO_GREEDY) {
+    flags |= 1u << 11;
+    goto done;
+  }
+  if (a->mode != SVO_GREEDY && !(a->T > 0.0 && isfinite(a->T))) {
+    flags |= 1u << 11;
+    goto done;
+  }
+  for (int i = 0; i < n; ++i) {
+    if (par[i] < 0 || par[i] > i) {
+      flags |= 1u << 11;
+      goto done;
+    }
+    if (tok[i] < 0 || tok[i] >= V) {
+      flags |= SVO_FLAG_BAD_TOKEN;
+      goto done;
+    }
+  }
+  {
+    const size_t trow0 = (size_t)b * (size_t)(Nm + 1);
+    const size_t qrow0 = (size_t)b * (size_t)Nm;
+    int has_child[Nm + 1];
+    for (int p = 0; p <= n; ++p) has_child[p] = 0;
+    for (int i = 0; i < n; ++i) has_child[par[i]] = 1;
+    for (int p = 0; p <= n; ++p)
+      if (!row_is_valid(row_ptr(a->target, trow0 + p, V, dt), V, dt)) {
+        flags |= SVO_FLAG_NONFINITE;
+        goto done;
+      }
+    if (a->mode != SVO_GREEDY)
+      for (int p = 0; p < n; ++p)
+        if (has_child[p] && !row_is_valid(row_ptr(a->draft, qrow0 + p, V, dt), V, dt)) {
+          flags |= SVO_FLAG_NONFINITE;
+          goto done;
+        }
+
+    int path[Nm > 0 ? Nm : 1];
+    int len = 0, pos = 0, emitted = -1;
+    double* P = (double*)malloc(sizeof(double) * (size_t)V);
+    double* q = (double*)malloc(sizeof(double) * (size_t)V);
+    for (;;) {
+      const void* trow = row_ptr(a->target, trow0 + pos, V, dt);
+      if (a->mode == SVO_GREEDY) {
+        /* accept the first child holding the target's top token */
+        const int am = svo_row_argmax(trow, V, dt);
+        int found = -1;
+        for (int i = 0; i < n && found < 0; ++i)
+          if (par[i] == pos && tok[i] == am) found = i;
+        if (found < 0) {
+          emitted = am;
+          break;
+        }
+        path[len++] = found;
+        pos = found + 1;
+        continue;
+      }
+      row_probs(trow, V, dt, a->T, P);
+      if (!has_child[pos]) {
+        /* no candidate: the bonus token from p */
+        double gap;
+        emitted = race_vec(P, V, a->seed, g, &gap);
+        if (gap < 1e-6) flags |= SVO_FLAG_RACE_NEAR_TIE;
+        break;
+      }
+      row_probs(row_ptr(a->draft, qrow0 + pos, V, dt), V, dt, a->T, q);
+      int accepted = -1;
+      for (int i = 0; i < n && accepted < 0; ++i) {
+        if (par[i] != pos) continue;
+        const int x = tok[i];
+        double acc;
+        if (q[x] > 0.0)
+          acc = fmin(1.0, P[x] / q[x]);
+        else
+          acc = P[x] > 0.0 ? 1.0 : 0.0;
+        const double u = svo_accept_uniform(a->seed, g, (uint32_t)i);
+        if (fabs(u - acc) < 1e-5) flags |= SVO_FLAG_ACCEPT_NEAR_TIE;
+        if (u < acc) {
+          accepted = i;
+          break;
+        }
+        /* rejected: the next candidate faces the normalised residual */
+        double Z = 0.0;
+        for (int y = 0; y < V; ++y) Z += fmax(0.0, P[y] - q[y]);
+        if (Z > 0.0) {
+          for (int y = 0; y < V; ++y) P[y] = fmax(0.0, P[y] - q[y]) / Z;
+        } else {
+          /* reading: an empty residual (only through rounding) keeps P */
+          flags |= SVO_FLAG_RESIDUAL_EMPTY;
+        }
+      }
+      if (accepted >= 0) {
+        path[len++] = accepted;
+        pos = accepted + 1;
+        continue;
+      }
+      double gap;
+      emitted = race_vec(P, V, a->seed, g, &gap);
+      if (gap < 1e-6) flags |= SVO_FLAG_RACE_NEAR_TIE;
+      break;
+    }
+    free(P);
+    free(q);
+    for (int j = 0; j < len; ++j) {
+      ot[j] = tok[path[j]];
+      if (on) on[j] = path[j];
+    }
+    ot[len] = emitted;
+    a->out_accept_len[b] = len + 1;
+  }
+done:
+  if (a->out_flags) a->out_flags[b] = flags;
+}
+
+int svo_verify_tree(const void* target, const void* draft, const int32_t* tokens,
+                    const int32_t* parents, const int32_t* n_nodes, int B, int N_max, int V,
+                    int dtype, float temperature, int mode, uint64_t seed,
+                    uint32_t request_offset, int32_t* out_tokens, int32_t* out_accept_len,
+                    int32_t* out_nodes, uint32_t* out_flags, int nthreads) {
+  if (B < 0 || N_max < 0 || V <= 0 || (dtype != SVO_F32 && dtype != SVO_BF16)) return -1;
+  if (B > 0 && (!target || !out_tokens || !out_accept_len)) return -1;
+  if (B > 0 && N_max > 0 && (!tokens || !parents)) return -1;
+  if (B > 0 && N_max > 0 && mode != SVO_GREEDY && !draft) return -1;
+  tree_args a;
+  memset(&a, 0, sizeof a);
+  a.target = target;
+  a.draft = draft;
+  a.tokens = tokens;
+  a.parents = parents;
+  a.n_nodes = n_nodes;
+  a.B = B;
+  a.N_max = N_max;
+  a.V = V;
+  a.dtype = dtype;
+  a.T = (double)temperature;
+  a.mode = mode;
+  a.seed = seed;
+  a.request_offset = request_offset;
+  a.out_tokens = out_tokens;
+  a.out_accept_len = out_accept_len;
+  a.out_nodes = out_nodes;
+  a.out_flags = out_flags;
+#ifdef _OPENMP
+  if (nthreads > 1) {
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int b = 0; b < B; ++b) verify_tree_one(&a, b);
+    return 0;
+  }
+#endif
+  (void)nthreads;
+  for (int b = 0; b < B; ++b) verify_tree_one(&a, b);
+  return 0;
+}
+
 /* ---------------------------------------------------------------- epilogue */
 
 /* "Accélérer Sonar par la Spéculation", section "Calendrier MTP pour un jeton

@@ -138,6 +138,38 @@ int svo_ssd_lookup(const int32_t* out_tokens, const int32_t* accept_len, int B, 
                    const int32_t* keys_al, const int32_t* keys_token, int K, const int32_t* spec,
                    int S, int32_t* out_hit, int32_t* out_spec);
 
+/*
+ * Tree (multi-candidate) verification ("Accélérer Sonar par la Spéculation",
+ * section "EAGLE": draft trees whose nodes hold several candidate tokens, the
+ * top candidates at each node).  Request b has n = n_nodes[b] (or N_max) draft
+ * nodes; node i holds token tokens[b][i] and hangs under position
+ * parents[b][i] in [0, i] (position 0 is the root -- the last committed token --
+ * and position i + 1 is node i).  Target row p of [B, N_max+1, V] is the
+ * target's distribution after position p's path; draft row p of
+ * [B, N_max, V] is the distribution position p's children were drawn from
+ * (only rows of positions with children are read).
+ * The walk from the root: at position p with children c_1 < c_2 < ... (node
+ * order), with P = p_p (softmax of target row p at T) and q = q_p:
+ *   candidate c_j is accepted with probability min(1, P(x)/q(x)), x its token,
+ *   u from Philox at counter (c_j, g, 0, 0); accepted -> its token is emitted
+ *   and the walk moves to position c_j + 1; rejected -> P = norm(max(0, P - q))
+ *   and the next candidate is tried;
+ *   every candidate rejected -> a token is drawn from P by the race and the
+ *   walk ends; no candidate at all -> the bonus token is drawn from p_p.
+ * Greedy: the first child whose token is the argmax of target row p is
+ * accepted; otherwise that argmax is emitted and the walk ends.
+ * Outputs: out_tokens [B, N_max+1] (the accepted tokens, then the drawn one,
+ * then -1), out_accept_len [B] (AL), out_nodes [B, N_max] (the accepted nodes,
+ * then -1; may be NULL), out_flags [B] (may be NULL).  A parent outside
+ * [0, i] sets SVO_FLAG_BAD_PARAM (1 << 11); other errors as svo_verify.
+ * Returns 0, or -1 for invalid arguments.
+ */
+int svo_verify_tree(const void* target, const void* draft, const int32_t* tokens,
+                    const int32_t* parents, const int32_t* n_nodes, int B, int N_max, int V,
+                    int dtype, float temperature, int mode, uint64_t seed,
+                    uint32_t request_offset, int32_t* out_tokens, int32_t* out_accept_len,
+                    int32_t* out_nodes, uint32_t* out_flags, int nthreads);
+
 /* 1 when built with OpenMP, else 0. */
 int svo_has_openmp(void);
 

@@ -60,6 +60,11 @@ MUTANTS = {
     "ssd_ignores_accept_len": ("if (keys_al[(size_t)b * K + k] == AL && keys_token[(size_t)b * K + k] == tok) hit = k;",
                                "if (keys_token[(size_t)b * K + k] == tok) hit = k;"),
     "ssd_last_match_wins": ("for (int k = 0; k < K && hit < 0; ++k)", "for (int k = 0; k < K; ++k)"),
+    "tree_no_renormalise": ("for (int y = 0; y < V; ++y) P[y] = fmax(0.0, P[y] - q[y]) / Z;",
+                            "for (int y = 0; y < V; ++y) P[y] = fmax(0.0, P[y] - q[y]);"),
+    "tree_uniform_per_position": ("const double u = svo_accept_uniform(a->seed, g, (uint32_t)i);",
+                                  "const double u = svo_accept_uniform(a->seed, g, (uint32_t)pos);"),
+    "tree_greedy_last_child": ("for (int i = 0; i < n && found < 0; ++i)", "for (int i = 0; i < n; ++i)"),
     "epilogue_append_drops_last": ("for (int j = 0; j < AL; ++j) seq", "for (int j = 0; j + 1 < AL; ++j) seq"),
 }
 
@@ -310,9 +315,33 @@ def check_ssd(svo, L):
     return True
 
 
+def check_tree(svo, L):
+    import test_oracle_tree as tt
+
+    class Shim:
+        SVO_STOCHASTIC, SVO_GREEDY = svo.SVO_STOCHASTIC, svo.SVO_GREEDY
+        FLAG_NEAR_TIE, FLAG_BAD_TOKEN = svo.FLAG_NEAR_TIE, svo.FLAG_BAD_TOKEN
+
+        @staticmethod
+        def verify(*a, **k):
+            return svo.verify(*a, L=L, **k)
+
+        @staticmethod
+        def verify_tree(*a, **k):
+            return svo.verify_tree(*a, L=L, **k)
+    try:
+        tt.test_chain_tree_is_the_linear_rule(Shim)
+        tt.test_greedy_tree_reproduces_argmax_decoding(Shim)
+        tt.test_emitted_tokens_follow_the_target(Shim)
+        tt.test_the_first_matching_candidate_is_taken(Shim)
+    except AssertionError:
+        return False
+    return True
+
+
 CHECKS = [check_lse, check_argmax, check_kat, check_engines, check_avalanche, check_uniform, check_p_eq_q, check_al_law,
           check_residual_law, check_bonus_law, lambda s, L: check_marginal(s, L, 0),
-          lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy, check_epilogue, check_ssd]
+          lambda s, L: check_marginal(s, L, 2), check_saguaro_ties, check_greedy, check_epilogue, check_ssd, check_tree]
 
 
 def _build_variant(tmp, text):
