@@ -50,6 +50,12 @@ def measured_peak():
 
 def workload_desc(w):
     m = w.meta
+    if hasattr(w, "parents"):
+        return (f"{w.name}: B={w.B}, draft tree with branching {tuple(m['branching'])} "
+                f"({w.N} nodes), V={w.V}, {'bf16' if w.dtype == 1 else 'fp32'} logits, target "
+                f"N(0,{m['target_sd']}^2), draft = target + N(0,{m['draft_sd']}^2), candidates drawn "
+                f"from q at their parent, T={w.temperature}, "
+                f"{['stochastic', 'greedy', 'saguaro'][w.mode]}")
     return (f"{w.name}: B={w.B}, D={w.D_max}, V={w.V}, "
             f"{'bf16' if w.dtype == 1 else 'fp32'} logits, target N(0,{m['target_sd']}^2), "
             f"draft = target + N(0,{m['draft_sd']}^2), draft tokens sampled from q, T={w.temperature}, "
@@ -157,8 +163,10 @@ def cpu_baseline(w, target_seconds=10.0, single_seconds=5.0):
     about `target_seconds` pass, and the plain single-threaded loop on the first
     requests of the batch for about `single_seconds`."""
     import oracle
-    h = w.host_arrays()
     cores = os.cpu_count() or 1
+    if hasattr(w, "parents"):
+        return tree_cpu_baseline(w, target_seconds, single_seconds, cores)
+    h = w.host_arrays()
 
     def run(sl, nthreads):
         oracle.verify(h["target"][sl], h["draft"][sl], h["tokens"][sl],
@@ -194,6 +202,49 @@ def cpu_baseline(w, target_seconds=10.0, single_seconds=5.0):
             "single_core": {"value": rows1 / el1, "unit": "rows/s", "cores": 1,
                             "sample": f"the first {n1} requests ({rows1} verified rows), "
                                       f"{el1:.1f} s, the plain single-threaded loop"}}
+
+
+def tree_cpu_baseline(w, target_seconds, single_seconds, cores):
+    """cpu_baseline for a tree workload: the oracle's tree walk."""
+    import numpy as np
+    import oracle
+
+    def host(t):
+        t = t.detach().cpu().contiguous()
+        return t.view(torch_int16()).numpy().view(np.uint16) if w.dtype == 1 else t.numpy()
+    tgt, dft = host(w.target), host(w.draft)
+    tok, par = w.tokens.cpu().numpy(), w.parents.cpu().numpy()
+
+    def run(sl, nthreads):
+        oracle.verify_tree(tgt[sl], dft[sl], tok[sl], par[sl], temperature=w.temperature,
+                           mode=w.mode, seed=0, request_offset=sl.start, nthreads=nthreads)
+
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run(slice(0, w.B), cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= target_seconds or reps >= 50:
+            break
+    n1, t1 = 0, time.perf_counter()
+    while n1 < w.B:
+        run(slice(n1, n1 + 1), 1)
+        n1 += 1
+        if time.perf_counter() - t1 >= single_seconds:
+            break
+    el1 = time.perf_counter() - t1
+    per_req = w.verified_rows() // w.B
+    return {"value": reps * w.verified_rows() / el, "unit": "rows/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"the whole {w.name} batch ({w.B} requests) x {reps} repetitions, {el:.1f} s, "
+                      f"OpenMP over requests on {cores} threads",
+            "single_core": {"value": n1 * per_req / el1, "unit": "rows/s", "cores": 1,
+                            "sample": f"the first {n1} requests, {el1:.1f} s, single-threaded"}}
+
+
+def torch_int16():
+    import torch
+    return torch.int16
 
 
 def acceptance_stats(sv, w, variant, nseeds, stream):
@@ -311,7 +362,13 @@ def run_ours(args):
                "fused": sv.SV_VARIANT_FUSED, "cluster": sv.SV_VARIANT_CLUSTER}[args.variant]
 
     # every rank verifies its own batch (its own seed and request range)
-    w = workloads.make(args.workload, dev, seed=workloads.CONFIGS[args.workload]["seed"] + 97 * rank)
+    tree = args.workload in workloads.TREE_CONFIGS
+    if tree:
+        w = workloads.make_tree(args.workload, dev,
+                                seed=workloads.TREE_CONFIGS[args.workload]["seed"] + 97 * rank)
+    else:
+        w = workloads.make(args.workload, dev,
+                           seed=workloads.CONFIGS[args.workload]["seed"] + 97 * rank)
     offset = rank * w.B
     stream = torch.cuda.current_stream(dev)
     out = dict(tokens=torch.empty((w.B, w.D_max + 1), dtype=torch.int32, device=dev),
@@ -332,7 +389,16 @@ def run_ours(args):
         copies = [dataclasses.replace(w, target=big[0][c], draft=big[1][c], tokens=big[2][c])
                   for c in range(ncopies)]
 
+    if tree:
+        out = None
+
     def step(i, ev=None):
+        if tree:
+            c = copies[i % ncopies]
+            sv.verify_tree(c.target, c.draft, c.tokens, c.parents, temperature=c.temperature,
+                           mode=c.mode, seed=1000 + i, request_offset=offset, stream=stream,
+                           timing_events=ev)
+            return
         sv.verify_workload(copies[i % ncopies], seed=1000 + i, request_offset=offset,
                            variant=variant, stream=stream, out=out, timing_events=ev)
 
@@ -395,7 +461,7 @@ def run_ours(args):
     # acceptance: mean AL and its histogram (for saguaro next to the plain rule
     # on the same logits, its draft tokens drawn from q instead of q')
     acceptance = None
-    if args.al_seeds > 0:
+    if args.al_seeds > 0 and not tree:
         acceptance = acceptance_stats(sv, w, variant, args.al_seeds, stream)
         if w.mode == sv.SV_SAGUARO:
             wp = workloads.make(args.workload, dev, mode=sv.SV_STOCHASTIC,
@@ -408,7 +474,7 @@ def run_ours(args):
     # end to end through the same call with host buffers: pinned H2D of the
     # step's inputs, the call, D2H of the step's outputs, all in the timed region
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not tree:
         h_t = torch.empty(w.target.shape, dtype=w.target.dtype, pin_memory=True)
         h_q = torch.empty(w.draft.shape, dtype=w.draft.dtype, pin_memory=True)
         h_x = torch.empty(w.tokens.shape, dtype=w.tokens.dtype, pin_memory=True)
@@ -472,7 +538,9 @@ def run_ours(args):
         else:
             # the statistics pass reads every needed logit row once
             rows_read = 0
-            for d, m in zip(w.row_D_list(), w.modes()):
+            if tree:
+                rows_read = w.B * ((w.N + 1) + (0 if w.mode == 1 else len(set(w.parent_list()))))
+            for d, m in ([] if tree else zip(w.row_D_list(), w.modes())):
                 rows_read += (d + 1) + (0 if m == 1 else d)
             kname, kbytes = "row_stats", rows_read * w.V * (2 if w.dtype == 1 else 4)
             ksrc = ["speculative_decoding_verification_lse_b200/csrc/row_stats.cu",
@@ -528,7 +596,7 @@ def run_ours(args):
                 f"untimed steps after the timed region, every step the same call")),
             # fused: one launch; split: statistics, then one kernel per request or
             # the scan and the race items (the library's rule, in include/specverify.h)
-            "gpu_launches": (1 if used_variant in ("fused", "cluster") else
+            "gpu_launches": (2 if tree else 1 if used_variant in ("fused", "cluster") else
                              3 if (used_variant == "split-items" or (used_variant == "split" and tail_items(
                                  w, torch.cuda.get_device_properties(dev).multi_processor_count)))
                              else 2) * args.steps,

@@ -221,6 +221,40 @@ SV_API int sv_verify_ex(const void* target_logits, const void* draft_logits,
                  int32_t* out_accept_len, const sv_params* p);
 
 /*
+ * sv_verify_tree: tree (multi-candidate) verification ("Accélérer Sonar par la
+ * Spéculation", section "EAGLE": the draft proposes a tree whose nodes hold
+ * several candidate tokens).  Request b has n = n_nodes[b] (NULL: N_max) nodes;
+ * node i holds node_tokens[b][i] and hangs under position parents[b][i] in
+ * [0, i]: position 0 is the root (the last committed token), position i + 1 is
+ * node i.  target_logits [B, N_max+1, V]: row p is the target's distribution
+ * after position p's path; draft_logits [B, N_max, V]: row p is the
+ * distribution position p's candidates were drawn from (read only for
+ * positions with candidates; NULL allowed when greedy).
+ * From the root, at position p the candidates under p are tried in node
+ * order: candidate j is accepted with probability min(1, P_j(x)/q_p(x)) (u_j
+ * from Philox at counter (node, g, 0, 0)), P_0 = p_p and a rejection replaces
+ * P_j by norm(max(0, P_j - q_p)) ("Speculative Speculative Decoding", rule
+ * items 1-3, applied recursively); an accepted candidate's token is emitted and
+ * the walk moves to its position; after the last candidate the token is drawn
+ * from the residual by the exponential race, and at a position with no
+ * candidate the bonus token is drawn from p_p.  Greedy (mode SV_GREEDY): the
+ * first candidate holding the argmax of target row p is accepted, otherwise
+ * that argmax is emitted.  A chain (parents[b][i] == i) is sv_verify's rule.
+ * Outputs: out_tokens [B, N_max+1] (the accepted path's tokens, then the drawn
+ * token, then -1), out_accept_len [B] (AL = path length + 1), out_nodes
+ * [B, N_max] (optional: the accepted nodes, then -1), and sv_params'
+ * out_flags / out_row_lse.  mode: SV_STOCHASTIC or SV_GREEDY (per-request
+ * modes likewise; saguaro requests are flagged SV_FLAG_BAD_PARAM, as are
+ * parents outside [0, i]).  sv_params.variant, .epilogue and .out_draft_top
+ * are ignored.  Otherwise as sv_verify_ex.
+ */
+SV_API int sv_verify_tree(const void* target_logits, const void* draft_logits,
+                          const int32_t* node_tokens, const int32_t* parents,
+                          const int32_t* n_nodes, int B, int N_max, int V, int dtype,
+                          float temperature, int mode, uint64_t seed, int32_t* out_tokens,
+                          int32_t* out_accept_len, int32_t* out_nodes, const sv_params* p);
+
+/*
  * sv_verify_static: sv_verify_ex that allocates nothing.  (The pages have no
  * counterpart; this is a service for callers.)
  *

@@ -126,6 +126,10 @@ def load(build_if_needed=True):
     L.sv_shard_finish.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                   ctypes.c_void_p, ctypes.POINTER(SvParams)]
     L.sv_shard_finish.restype = ctypes.c_int
+    L.sv_verify_tree.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 4 + [
+        ctypes.c_float, ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p, ctypes.POINTER(SvParams)]
+    L.sv_verify_tree.restype = ctypes.c_int
     L.sv_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.sv_workspace_bytes.restype = ctypes.c_size_t
     L.sv_get_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
@@ -230,6 +234,54 @@ def sv_shard_race(target_local, draft_local, draft_tokens, row_D, B, D_max, V_lo
 def sv_shard_finish(B, D_max, n_shards, gathered2, out_tokens, params=None):
     return load().sv_shard_finish(B, D_max, n_shards, _p(gathered2), _p(out_tokens),
                                   ctypes.byref(params) if params is not None else None)
+
+
+def sv_verify_tree(target_logits, draft_logits, node_tokens, parents, n_nodes, B, N_max, V, dtype,
+                   temperature, mode, seed, out_tokens, out_accept_len, out_nodes, params=None):
+    return load().sv_verify_tree(_p(target_logits), _p(draft_logits), _p(node_tokens), _p(parents),
+                                 _p(n_nodes), B, N_max, V, dtype, temperature, mode,
+                                 seed & (2**64 - 1), _p(out_tokens), _p(out_accept_len),
+                                 _p(out_nodes), ctypes.byref(params) if params is not None else None)
+
+
+def verify_tree(target, draft, tokens, parents, n_nodes=None, *, temperature=1.0,
+                mode=SV_STOCHASTIC, seed=0, temperature_per_req=None, mode_per_req=None,
+                request_offset=0, stream=None, row_lse=False, timing_events=None):
+    """Tree verification of a batch held in CUDA tensors (sv_verify_tree):
+    target [B, N+1, V], draft [B, N, V] (or None when greedy), tokens and parents
+    [B, N] int32, n_nodes [B] int32 or None.  Returns dict(tokens, accept_len,
+    nodes, flags [, row_lse]) as CUDA tensors (not synchronised)."""
+    import torch
+    if not target.is_cuda:
+        raise ValueError("target logits must be a CUDA tensor (there is no CPU path)")
+    dt = _dtype_code(target)
+    B, Np1, V = target.shape
+    N = Np1 - 1
+    for name, t in (("tokens", tokens), ("parents", parents)):
+        if t.dtype != torch.int32 or tuple(t.shape) != (B, N) or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous int32 [B, N]")
+    dev = target.device
+    out = dict(tokens=torch.empty((B, N + 1), dtype=torch.int32, device=dev),
+               accept_len=torch.empty((B,), dtype=torch.int32, device=dev),
+               nodes=torch.empty((B, N), dtype=torch.int32, device=dev),
+               flags=torch.empty((B,), dtype=torch.int32, device=dev))
+    if row_lse:
+        out["row_lse"] = torch.empty((B, 2 * N + 1), dtype=torch.float32, device=dev)
+    prm = SvParams()
+    prm.stream = _stream_ptr(stream)
+    prm.temperature_per_req = _p(temperature_per_req)
+    prm.mode_per_req = _p(mode_per_req)
+    prm.request_offset = int(request_offset)
+    prm.out_flags = _p(out["flags"])
+    prm.out_row_lse = _p(out.get("row_lse"))
+    if timing_events is not None:
+        arr = (ctypes.c_void_p * 2)(timing_events[0].cuda_event, timing_events[1].cuda_event)
+        prm.timing_events = ctypes.cast(arr, ctypes.c_void_p)
+    with torch.cuda.device(dev):
+        _check(sv_verify_tree(target, draft, tokens, parents, n_nodes, B, N, V, dt,
+                              float(temperature), int(mode), int(seed), out["tokens"],
+                              out["accept_len"], out["nodes"], prm))
+    return out
 
 
 def sv_workspace_bytes(B, D_max, V, dtype):

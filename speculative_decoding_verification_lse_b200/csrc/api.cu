@@ -489,6 +489,45 @@ int sv_shard_finish(int B, int D_max, int n_shards, const void* gathered2, int32
   return e == cudaSuccess ? SV_OK : cuda_fail(e, "shard finish launch");
 }
 
+int sv_verify_tree(const void* target_logits, const void* draft_logits,
+                   const int32_t* node_tokens, const int32_t* parents, const int32_t* n_nodes,
+                   int B, int N_max, int V, int dtype, float temperature, int mode, uint64_t seed,
+                   int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_nodes,
+                   const sv_params* p) {
+  sv_params prm;
+  memset(&prm, 0, sizeof prm);
+  if (p) prm = *p;
+  prm.variant = SV_VARIANT_SPLIT;
+  prm.epilogue = nullptr;
+  prm.out_draft_top = nullptr;
+  g_last_error.clear();
+  if (mode != SV_STOCHASTIC && mode != SV_GREEDY)
+    return fail(SV_ERR_INVALID_ARG, "tree verification takes SV_STOCHASTIC or SV_GREEDY (got %d)",
+                mode);
+  if (B > 0 && N_max > 0 && !parents) return fail(SV_ERR_INVALID_ARG, "parents is NULL");
+  Call call;
+  bool empty = false;
+  int rc = prepare_call(target_logits, draft_logits, node_tokens, n_nodes, B, N_max, V, dtype,
+                        temperature, mode, seed, out_tokens, out_accept_len, prm, V, 0, &call,
+                        &empty);
+  if (rc != SV_OK || empty) return rc;
+  VerifyArgs& a = call.a;
+  a.parents = parents;
+  a.out_nodes = out_nodes;
+  cudaStream_t s = (cudaStream_t)prm.stream;
+  cudaEvent_t* ev = (cudaEvent_t*)prm.timing_events;
+  cudaError_t e;
+  const bool tickets = row_stats_tickets(a, call.grid);
+  if (tickets && (e = cudaMemsetAsync(a.ticket, 0, 8 * 128, s)) != cudaSuccess)
+    return cuda_fail(e, "cudaMemsetAsync(ticket)");
+  if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = launch_row_stats(a, s, call.grid, tickets)) != cudaSuccess)
+    return cuda_fail(e, "row statistics launch");
+  if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = launch_tree(a, s)) != cudaSuccess) return cuda_fail(e, "tree walk launch");
+  return SV_OK;
+}
+
 int sv_verify(const void* target_logits, const void* draft_logits, const int32_t* draft_tokens,
               const int32_t* row_D, int B, int D_max, int V, int dtype, float temperature,
               int mode, uint64_t seed, int32_t* out_tokens, int32_t* out_accept_len) {

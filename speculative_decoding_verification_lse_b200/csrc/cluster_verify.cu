@@ -86,13 +86,13 @@ __global__ void __launch_bounds__(kThreads, 2) cluster_kernel(VerifyArgs a) {
   const int items = a.slots * a.nseg;
   for (int i = gw; i < items; i += nw) {
     const int slot = i / a.nseg, seg = i - slot * a.nseg;
-    if (row_needed(a, slot, rp)) stats_item<DT, WITH_TOP>(a, b, slot, seg, rp);
+    if (row_needed(a, b, slot, rp)) stats_item<DT, WITH_TOP>(a, b, slot, seg, rp);
   }
   cluster.sync();
 
   // 2. one row per warp
   for (int slot = gw; slot < a.slots; slot += nw)
-    if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &a.rowres[(size_t)b * a.slots + slot]);
+    if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &a.rowres[(size_t)b * a.slots + slot]);
   cluster.sync();
 
   // 3. the accept scan and the reference key

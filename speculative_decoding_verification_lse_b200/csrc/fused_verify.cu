@@ -103,7 +103,7 @@ __device__ __noinline__ void row_done(const VerifyArgs& a, int b, int slot, unsi
   }
   if (!__shfl_sync(0xFFFFFFFFu, last, 0)) return;
   const ReqParams rp = load_req(a, b);
-  if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &a.rowres[row]);
+  if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &a.rowres[row]);
   unsigned req_last = 0;
   if (lane == 0) {
     __threadfence();
@@ -133,7 +133,7 @@ __device__ void stats_batch(const VerifyArgs& a, unsigned t, unsigned total, War
     cb = b;
     cs = slot;
     const ReqParams rp = load_req(a, b);
-    if (row_needed(a, slot, rp)) stats_item<DT, WITH_TOP>(a, b, slot, seg, rp);
+    if (row_needed(a, b, slot, rp)) stats_item<DT, WITH_TOP>(a, b, slot, seg, rp);
     ++cnt;
   }
   if (cnt) row_done<DT>(a, cb, cs, cnt, W, rows);

@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(kThreads, 3) row_stats_kernel(VerifyArgs a) {
         const unsigned r = i % per_req;
         const int slot = (int)(r / (unsigned)a.nseg), seg = (int)(r % (unsigned)a.nseg);
         const ReqParams rp = load_req(a, b);
-        if (row_needed(a, slot, rp)) stats_item<DT, WITH_TOP>(a, b, slot, seg, rp);
+        if (row_needed(a, b, slot, rp)) stats_item<DT, WITH_TOP>(a, b, slot, seg, rp);
       }
       t = __shfl_sync(0xFFFFFFFFu, tn, 0);
     }

@@ -116,11 +116,8 @@ __device__ inline void merge_row(const PartStat* ps, const TopPart* tp, int nseg
 }
 
 // Whether row `slot` of a request with parameters rp is read by the rule.
-__device__ __forceinline__ bool slot_needed(const VerifyArgs& a, int slot, const ReqParams& rp) {
-  if (rp.err) return false;
-  const bool is_t = slot <= a.D_max;
-  const int d = is_t ? slot : slot - a.D_max - 1;
-  return is_t ? d <= rp.Db : (d < rp.Db && rp.mode != kGreedy);
+__device__ __forceinline__ bool slot_needed(const VerifyArgs& a, int b, int slot, const ReqParams& rp) {
+  return row_read(a, b, slot, rp);
 }
 
 // Merge row `slot` of request b (one full warp) from the partials PS(s) and
@@ -214,7 +211,7 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* row
   if (!err) {
     uint32_t nonfinite = 0;
     for (int slot = lane; slot < a.slots; slot += 32)
-      if (slot_needed(a, slot, rp) && rows[slot].bad) nonfinite = kFlagNonfinite;
+      if (slot_needed(a, b, slot, rp) && rows[slot].bad) nonfinite = kFlagNonfinite;
     err |= __reduce_or_sync(0xFFFFFFFFu, nonfinite);
   }
 

@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 2) shard_tail_kernel(VerifyArgs a, c
   // local segment s % nseg
   const int nseg = a.nseg, Dm = a.D_max;
   for (int slot = warp; slot < a.slots; slot += kWarps) {
-    if (!slot_needed(a, slot, rp)) continue;
+    if (!slot_needed(a, b, slot, rp)) continue;
     const bool is_t = slot <= Dm;
     const int d = is_t ? slot : slot - Dm - 1;
     const bool top = !is_t && rp.mode == kSaguaro;

@@ -322,11 +322,8 @@ __device__ __noinline__ void stats_segment_top(const VerifyArgs& a, const char* 
 }
 
 // Whether row `slot` of a request with parameters rp is read by the rule.
-__device__ __forceinline__ bool row_needed(const VerifyArgs& a, int slot, const ReqParams& rp) {
-  if (rp.err) return false;
-  const bool is_target = slot <= a.D_max;
-  const int d = is_target ? slot : slot - a.D_max - 1;
-  return is_target ? d <= rp.Db : (d < rp.Db && rp.mode != kGreedy);
+__device__ __forceinline__ bool row_needed(const VerifyArgs& a, int b, int slot, const ReqParams& rp) {
+  return row_read(a, b, slot, rp);
 }
 
 // Statistics of segment `seg` of row `slot` of request b (one full warp).
@@ -404,7 +401,7 @@ __device__ __forceinline__ void stats_pass(const VerifyArgs& a, unsigned w0, uns
   it.init(a, w0, W);
   for (unsigned i = w0; i < total; i += W, it.advance(a)) {
     const ReqParams rp = load_req(a, it.b);
-    if (!row_needed(a, it.slot, rp)) continue;
+    if (!row_needed(a, it.b, it.slot, rp)) continue;
     stats_item<DT, WITH_TOP>(a, it.b, it.slot, it.seg, rp);
   }
 }

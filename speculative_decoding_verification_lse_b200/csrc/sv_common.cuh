@@ -164,6 +164,8 @@ struct VerifyArgs {
   int saguaro_k;
   float saguaro_c;
   uint32_t request_offset;
+  const int32_t* parents;  // tree verification: [B, D_max] parent position of each node; NULL: linear
+  int32_t* out_nodes;      // tree verification: [B, D_max] accepted nodes (optional)
 };
 
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
@@ -333,6 +335,26 @@ __device__ __forceinline__ ReqParams load_req(const VerifyArgs& a, int b) {
   return r;
 }
 
+// Whether draft row d (position d) of request b is read: for a tree, only a
+// position with a child (a node i < D_b hanging under it) has candidates to
+// test; a linear batch tests every d < D_b.
+__device__ __forceinline__ bool draft_row_read(const VerifyArgs& a, int b, int d, int Db) {
+  if (d >= Db) return false;
+  if (!a.parents) return true;
+  const int32_t* par = a.parents + (size_t)b * a.D_max;
+  for (int i = d; i < Db; ++i)
+    if (__ldg(&par[i]) == d) return true;
+  return false;
+}
+
+// Whether row `slot` of request b with parameters rp is read by the rule
+// (target slots 0..D_max, draft slots D_max+1 ..).
+__device__ __forceinline__ bool row_read(const VerifyArgs& a, int b, int slot, const ReqParams& rp) {
+  if (rp.err) return false;
+  if (slot <= a.D_max) return slot <= rp.Db;
+  return rp.mode != kGreedy && draft_row_read(a, b, slot - a.D_max - 1, rp.Db);
+}
+
 // k2 = fl(log2(e) / T): the one scale every kernel applies to logits.
 __device__ __forceinline__ float log2e_over_T(float T) { return __fdiv_rn(1.44269504088896341f, T); }
 
@@ -363,6 +385,7 @@ cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);
 cudaError_t launch_cluster(const VerifyArgs& a, cudaStream_t s);
+cudaError_t launch_tree(const VerifyArgs& a, cudaStream_t s);
 ShardLayout shard_layout(int B, int D_max, int V_local, int dtype);
 cudaError_t launch_shard_z(const VerifyArgs& a, void* zx, cudaStream_t s);
 cudaError_t launch_shard_tail(const VerifyArgs& a, const void* gathered1, int n_shards,

@@ -68,7 +68,7 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
   // the scan's inputs by the last warp (the fewest rows to merge), during the merges
   if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
   for (int slot = warp; slot < a.slots; slot += kWarps)
-    if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
+    if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
   __syncthreads();
   if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();
@@ -122,7 +122,7 @@ __device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared&
   // the scan's inputs by the last warp (the fewest rows to merge), during the merges
   if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
   for (int slot = warp; slot < a.slots; slot += kWarps)
-    if (slot_needed(a, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
+    if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
   __syncthreads();
   if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();

@@ -226,3 +226,119 @@ def make(name: str = "tiny", device="cpu", *, B=None, D=None, V=None, seed=None,
         saguaro_k=int(cfg.get("saguaro_k", 5)), saguaro_c=float(cfg.get("saguaro_c", 0.5)),
         seed=int(verify_seed), meta=dict(cfg),
     )
+
+
+# ---- draft trees
+
+TREE_CONFIGS = {
+    # B requests, a draft tree with `branching[k]` candidates under every node of
+    # depth k (breadth-first node order), V, bf16; target N(0, 3^2) at every
+    # position, draft = target + N(0, 1^2); candidates are independent draws
+    # from the draft at their parent position (Gumbel-max at T)
+    "tree": dict(B=64, branching=(3, 2, 2), V=128256, dtype=BF16, target_sd=3.0, draft_sd=1.0,
+                 T=1.0, seed=1005),
+}
+
+
+@dataclass
+class TreeWorkload:
+    name: str
+    target: torch.Tensor     # [B, N+1, V]
+    draft: torch.Tensor      # [B, N, V]
+    tokens: torch.Tensor     # [B, N] int32
+    parents: torch.Tensor    # [B, N] int32, parent position in [0, i]
+    temperature: float
+    mode: int
+    dtype: int
+    seed: int = 0
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def B(self):
+        return self.target.shape[0]
+
+    @property
+    def N(self):
+        return self.target.shape[1] - 1
+
+    @property
+    def D_max(self):
+        return self.N
+
+    @property
+    def V(self):
+        return self.target.shape[2]
+
+    def parent_list(self):
+        return [int(v) for v in self.parents[0].cpu().tolist()]
+
+    def verified_rows(self):
+        """Candidates tested per call: every node of every request, plus the row
+        the final token is drawn from."""
+        return self.B * (self.N + 1)
+
+    def algorithmic_bytes(self):
+        """Every target row and every draft row with candidates read once, plus
+        one row pair per request for the residual sums and the race."""
+        s = 4 if self.dtype == F32 else 2
+        with_child = len(set(self.parent_list()))
+        rows = (self.N + 1) + (0 if self.mode == GREEDY else with_child)
+        extra = 0 if self.mode == GREEDY else 2
+        return self.B * (rows + extra) * self.V * s
+
+
+def tree_parents(branching):
+    """Parent positions of a breadth-first tree: branching[k] children under
+    every node of depth k (the root has depth 0)."""
+    parents, level = [], [0]
+    for k in branching:
+        nxt = []
+        for pos in level:
+            for _ in range(k):
+                parents.append(pos)
+                nxt.append(len(parents))  # the new node's position
+        level = nxt
+    return parents
+
+
+def make_tree(name="tree", device="cpu", *, B=None, V=None, branching=None, seed=None,
+              mode=STOCHASTIC, dtype=None, T=None, chunk_rows=16) -> TreeWorkload:
+    cfg = dict(TREE_CONFIGS[name])
+    for k, v in (("B", B), ("V", V), ("branching", branching), ("seed", seed), ("dtype", dtype),
+                 ("T", T)):
+        if v is not None:
+            cfg[k] = v
+    parents = tree_parents(cfg["branching"])
+    Bn, N, Vn = cfg["B"], len(parents), cfg["V"]
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(cfg["seed"])
+    store = torch.float32 if cfg["dtype"] == F32 else torch.bfloat16
+    target = torch.empty((Bn, N + 1, Vn), dtype=store, device=device)
+    draft = torch.empty((Bn, N, Vn), dtype=store, device=device)
+    tokens = torch.empty((Bn, N), dtype=torch.int32, device=device)
+    par = torch.tensor(parents, dtype=torch.long, device=device)
+    for b0 in range(0, Bn, chunk_rows):
+        b1 = min(Bn, b0 + chunk_rows)
+        zt = torch.randn((b1 - b0, N + 1, Vn), generator=gen, device=device) * cfg["target_sd"]
+        zq = zt[:, :N] + torch.randn((b1 - b0, N, Vn), generator=gen, device=device) * cfg["draft_sd"]
+        target[b0:b1] = zt.to(store)
+        draft[b0:b1] = zq.to(store)
+        # node i's token: an independent draw from the draft at its parent position
+        zp = draft[b0:b1].float()[:, par, :]
+        tokens[b0:b1] = _gumbel_argmax(zp, cfg["T"], gen).to(torch.int32)
+        del zt, zq, zp
+    if mode == GREEDY:
+        # greedy drafting: each node's candidates are the draft's top tokens at its parent
+        # position, distinct, best first (the i-th child of a position takes the i-th best)
+        rank = {}
+        for i, p in enumerate(parents):
+            rank[i] = sum(1 for j in range(i) if parents[j] == p)
+        kmax = max(rank.values()) + 1
+        top = torch.topk(draft.float(), kmax, dim=-1).indices  # [B, N, kmax]
+        for i, p in enumerate(parents):
+            tokens[:, i] = top[:, p, rank[i]].to(torch.int32)
+    parents_t = torch.tensor(parents, dtype=torch.int32, device=device).repeat(Bn, 1).contiguous()
+    return TreeWorkload(name=name, target=target, draft=draft, tokens=tokens, parents=parents_t,
+                        temperature=float(cfg["T"]), mode=int(mode), dtype=int(cfg["dtype"]),
+                        seed=0, meta=dict(cfg, N=N))
