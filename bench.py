@@ -256,12 +256,23 @@ def acceptance_stats(sv, w, variant, nseeds, stream):
     import torch
     stoch = torch.tensor([m != sv.SV_GREEDY for m in w.modes()], device=w.target.device)
     hist = torch.zeros(w.D_max + 2, dtype=torch.int64, device=w.target.device)
-    in_top = rejected = 0
+    in_top = rejected = hits = 0
     k = min(w.saguaro_k, w.V)
     Db = torch.tensor(w.row_D_list(), device=w.target.device)
+    # the speculation cache of speculative speculative decoding: keys (d + 1, each of the
+    # draft's top-k at position d) for d < D, looked up with the verified outcome
+    dev = w.target.device
+    keys_tok = torch.topk(w.draft.float(), k, dim=-1).indices.to(torch.int32).reshape(w.B, -1)
+    keys_al = (torch.arange(w.D_max, device=dev, dtype=torch.int32) + 1).repeat_interleave(k)
+    keys_al = keys_al[None].repeat(w.B, 1).contiguous()
+    keys_tok = keys_tok.contiguous()
+    hit = torch.empty(w.B, dtype=torch.int32, device=dev)
     out = None
     for seed in range(nseeds):
         out = sv.verify_workload(w, seed=7000 + seed, variant=variant, stream=stream, out=out)
+        sv._check(sv.sv_ssd_lookup(out["tokens"], out["accept_len"], w.B, w.D_max, keys_al, keys_tok,
+                                   keys_al.shape[1], None, 0, hit, stream=stream))
+        hits += int(((hit >= 0) & stoch).sum())
         al = out["accept_len"].long()
         hist += torch.bincount(al[stoch], minlength=w.D_max + 2)
         n = al - 1
@@ -278,7 +289,8 @@ def acceptance_stats(sv, w, variant, nseeds, stream):
     return {"mean_al": sum(i * c for i, c in enumerate(hist)) / max(1, total),
             "al_hist": hist[1:], "requests": total,
             "rejections": rejected,
-            f"correction_in_draft_top{k}": in_top / max(1, rejected)}
+            f"correction_in_draft_top{k}": in_top / max(1, rejected),
+            f"speculation_cache_hit_rate_top{k}": hits / max(1, total)}
 
 
 def run_reference(args):
