@@ -36,7 +36,10 @@ def test_tiny_workload(sv, mode, variant):
 
 @VARIANTS
 @pytest.mark.parametrize("name", sorted(wl.CONFIGS))
-@pytest.mark.parametrize("V", [40000 + 13, 16384 * 2 + 7])
+# rows whose length in bytes is a multiple of 16 stream through the per-request
+# tail's bulk-copy ring, the others through registers; 32776 bf16 ends in a
+# segment of one 16-byte vector
+@pytest.mark.parametrize("V", [40000 + 13, 16384 * 2 + 7, 40000 + 8, 16384 * 2 + 8])
 def test_reduced_workloads(sv, name, V, variant):
     B = {"tiny": 3, "b32": 32, "b256": 24, "ragged": 24, "saguaro": 24}[name]
     w = wl.make(name, "cuda", B=B, V=V)
