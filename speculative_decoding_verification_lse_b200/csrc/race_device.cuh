@@ -60,6 +60,26 @@ __device__ __forceinline__ void offer(Best& B, double key, int x) {
   }
 }
 
+// The fields of the argument block that the race's out-of-line helpers read,
+// passed by value: a reference to the argument block (kernel parameter space)
+// would make every thread copy the block to its stack at each call.
+struct RowCtx {
+  uint64_t seed;
+  int dtype, V, nvec, vocab_offset;
+};
+
+__device__ __forceinline__ RowCtx row_ctx(const VerifyArgs& a) {
+  RowCtx c;
+  c.seed = a.seed;
+  c.dtype = a.dtype;
+  c.V = a.V;
+  c.nvec = a.nvec;
+  c.vocab_offset = a.vocab_offset;
+  return c;
+}
+
+__device__ __forceinline__ RowCtx row_ctx(const RowCtx& c) { return c; }
+
 __device__ __forceinline__ Best combine(const Best& A, const Best& C) {
   const bool c_wins =
       C.idx >= 0 && (A.idx < 0 || C.best > A.best || (C.best == A.best && C.idx < A.idx));
@@ -129,7 +149,9 @@ __device__ __forceinline__ uint32_t race_word(uint64_t seed, uint32_t g, int x) 
   return l == 0 ? w.x : l == 1 ? w.y : l == 2 ? w.z : w.w;
 }
 
-__device__ __forceinline__ double exact_key_of(const VerifyArgs& a, const RaceDesc& rd,
+// (A: the argument block or a RowCtx)
+template <class A>
+__device__ __forceinline__ double exact_key_of(const A& a, const RaceDesc& rd,
                                                const char* trow, const char* qrow,
                                                bool residual, int x) {
   const float zt = (a.dtype == kF32) ? logit_at<kF32>(trow, x) : logit_at<kBF16>(trow, x);
@@ -256,8 +278,8 @@ __device__ __forceinline__ uint32_t word_filter_compact(const uint4 (&raw)[32 / 
 
 // Vectors j0 .. j0 + NJ - 1 of one lane's part of segment `seg` (-inf past the
 // end of the row).
-template <int DT, int NJ>
-__device__ __forceinline__ void load_part(const VerifyArgs& a, const char* row, int seg, int j0,
+template <int DT, int NJ, class A>
+__device__ __forceinline__ void load_part(const A& a, const char* row, int seg, int j0,
                                           uint4 (&raw)[NJ]) {
   constexpr int VEC = Lanes<DT>::VEC;
   const int nfull = a.V / VEC;
@@ -282,7 +304,7 @@ __device__ __forceinline__ void load_part(const VerifyArgs& a, const char* row, 
 // each term bounded with slack for its rounding: log2 p from one FMA on k2
 // (within 2^-23 of log2(e)/T), log2f and expm1f (1 ulp each), the conversions,
 // and the sums (all below the 2^-21 relative slack added to each term).
-static __device__ __noinline__ float key2_upper(const VerifyArgs& a, const RaceDesc& rd,
+static __device__ __noinline__ float key2_upper(const RowCtx a, const RaceDesc& rd,
                                                 const char* trow, const char* qrow,
                                                 bool residual, int x) {
   const bool f32 = a.dtype == kF32;
@@ -325,7 +347,7 @@ static __device__ __noinline__ float key2_upper(const VerifyArgs& a, const RaceD
 // The best exact key among the lanes' largest target logits of a segment (one
 // token per lane, the lowest index on ties), over the warp; -inf if none.
 template <int DT>
-__device__ __noinline__ double lane_max_key(const VerifyArgs& a, const RaceDesc& rd,
+__device__ __noinline__ double lane_max_key(const RowCtx a, const RaceDesc& rd,
                                             const char* trow, const char* qrow, bool residual,
                                             int seg) {
   constexpr int VEC = Lanes<DT>::VEC;
@@ -364,8 +386,8 @@ __device__ __noinline__ double lane_max_key(const VerifyArgs& a, const RaceDesc&
 // small enough for the instruction cache.  Only groups g0 .. g1 - 1 of the
 // lane's NG (g1 < 0: to the end) are raced, so that a segment can be split
 // into independent items.
-template <int DT>
-__device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceDesc& rd,
+template <int DT, class A>
+__device__ __forceinline__ Best race_segment_in(const A& a, const RaceDesc& rd,
                                                 const RaceStream& R, const char* trow,
                                                 const char* qrow, bool residual, int seg,
                                                 double K0, float cup, int g0 = 0, int g1 = -1) {
@@ -373,7 +395,7 @@ __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceD
   if (g1 < 0) g1 = NG;
   const int v0 = seg * kSegVecs + (threadIdx.x & 31);
   if (!(K0 > -INFINITY)) {
-    K0 = lane_max_key<DT>(a, rd, trow, qrow, residual, seg);
+    K0 = lane_max_key<DT>(row_ctx(a), rd, trow, qrow, residual, seg);
     cup = filter_offset(K0, rd.lse_t);
   }
   // survivors whose single-precision bound falls below K0 - delta need no exact key
@@ -393,7 +415,7 @@ __device__ __forceinline__ Best race_segment_in(const VerifyArgs& a, const RaceD
         const int t = __clz((int)keep);
         keep &= ~(0x80000000u >> t);
         const int x = (v0 + 32 * (gi * QV + t / VEC)) * VEC + t % VEC;
-        if (x < a.V && key2_upper(a, rd, trow, qrow, residual, x) >= thr2)
+        if (x < a.V && key2_upper(row_ctx(a), rd, trow, qrow, residual, x) >= thr2)
           offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
       }
     }
@@ -423,7 +445,7 @@ __device__ __forceinline__ Best race_span_in(const VerifyArgs& a, const RaceDesc
   if (seg0 >= a.nseg) return B;
   int seg = seg0;
   double K = fmax(K0, from_ordered_u64(*(volatile unsigned long long*)shared));
-  if (!(K > -INFINITY)) K = lane_max_key<DT>(a, rd, trow, qrow, residual, seg);
+  if (!(K > -INFINITY)) K = lane_max_key<DT>(row_ctx(a), rd, trow, qrow, residual, seg);
   float cup = filter_offset(K, rd.lse_t);
   float thr2 = K > -INFINITY ? __double2float_rd((K - kRaceBand) * 1.4426950408889634 - 1e-5)
                              : -INFINITY;
@@ -445,7 +467,7 @@ __device__ __forceinline__ Best race_span_in(const VerifyArgs& a, const RaceDesc
         const int t = __clz((int)keep);
         keep &= ~(0x80000000u >> t);
         const int x = (v0 + 32 * (gi * QV + t / VEC)) * VEC + t % VEC;
-        if (x < a.V && key2_upper(a, rd, trow, qrow, residual, x) >= thr2)
+        if (x < a.V && key2_upper(row_ctx(a), rd, trow, qrow, residual, x) >= thr2)
           offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
       }
     }
@@ -458,7 +480,7 @@ __device__ __forceinline__ Best race_span_in(const VerifyArgs& a, const RaceDesc
       if (lane == 0 && wb > -INFINITY) atomicMax(shared, ordered_u64(wb));
       __syncwarp();
       K = fmax(K, fmax(wb, from_ordered_u64(*(volatile unsigned long long*)shared)));
-      if (!(K > -INFINITY)) K = lane_max_key<DT>(a, rd, trow, qrow, residual, nseg_);
+      if (!(K > -INFINITY)) K = lane_max_key<DT>(row_ctx(a), rd, trow, qrow, residual, nseg_);
       cup = filter_offset(K, rd.lse_t);
       thr2 = K > -INFINITY ? __double2float_rd((K - kRaceBand) * 1.4426950408889634 - 1e-5)
                            : -INFINITY;
@@ -526,7 +548,7 @@ __device__ __forceinline__ Best race_part(const VerifyArgs& a, const RaceDesc& r
         const int t = __clz((int)keep);
         keep &= ~(0x80000000u >> t);
         const int x = (v0 + 32 * (gi * QV + t / VEC)) * VEC + t % VEC;
-        if (x < a.V && key2_upper(a, rd, trow, qrow, residual, x) >= thr2)
+        if (x < a.V && key2_upper(row_ctx(a), rd, trow, qrow, residual, x) >= thr2)
           offer(B, exact_key_of(a, rd, trow, qrow, residual, x), x);
       }
     }
@@ -542,7 +564,7 @@ __device__ __forceinline__ Best race_part(const VerifyArgs& a, const RaceDesc& r
 }
 
 template <int DT>
-__device__ __noinline__ Best race_segment(const VerifyArgs& a, const RaceDesc& rd,
+__device__ __noinline__ Best race_segment(const RowCtx a, const RaceDesc& rd,
                                           const char* trow, const char* qrow, bool residual,
                                           int seg, double K0, float cup) {
   return race_segment_in<DT>(a, rd, race_stream(a.seed, rd.g, (uint32_t)a.vocab_offset >> 2), trow, qrow, residual, seg, K0, cup);

@@ -9,7 +9,7 @@ namespace sv {
 
 namespace {
 
-constexpr unsigned kBatch = 2;  // consecutive items per ticket
+constexpr unsigned kBatch = 1;  // consecutive items per ticket
 
 // TICKETS: warps take batches of kBatch consecutive items from ticket counters
 // (zero at launch; each warp fetches its next ticket while it works on the

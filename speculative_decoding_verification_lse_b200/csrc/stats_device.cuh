@@ -22,6 +22,8 @@
 #include <float.h>
 #include <limits.h>
 
+#include <type_traits>
+
 namespace sv {
 
 constexpr uint32_t kNegInfBf2 = 0xFF80FF80u;  // two bf16 -inf
@@ -74,13 +76,14 @@ __device__ __forceinline__ float elem(const uint4& v, int e) {
   return (e & 1) ? bf_hi(w) : bf_lo(w);
 }
 
-// Load the lane's kLaneVecs vectors of segment `seg`.
+// Load the lane's kLaneVecs vectors of segment `seg` of a row of V elements
+// (nvec vectors).
 template <int DT>
-__device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* row, int seg,
-                                             uint4 (&raw)[kLaneVecs]) {
+__device__ __forceinline__ void load_segment_v(const char* row, int V, int nvec, int seg,
+                                               uint4 (&raw)[kLaneVecs]) {
   constexpr int VEC = DT == kF32 ? 4 : 8;
   const int lane = threadIdx.x & 31;
-  const int nfull = a.V / VEC;
+  const int nfull = V / VEC;
   const int v0 = seg * kSegVecs + lane;
   const bool aligned = ((uintptr_t)row & 15u) == 0;
   if (aligned && (seg + 1) * kSegVecs <= nfull) {
@@ -90,8 +93,14 @@ __device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* ro
   } else {
 #pragma unroll
     for (int j = 0; j < kLaneVecs; ++j)
-      raw[j] = load_vec_checked<DT>(row, v0 + 32 * j, a.V, a.nvec, nfull, aligned);
+      raw[j] = load_vec_checked<DT>(row, v0 + 32 * j, V, nvec, nfull, aligned);
   }
+}
+
+template <int DT>
+__device__ __forceinline__ void load_segment(const VerifyArgs& a, const char* row, int seg,
+                                             uint4 (&raw)[kLaneVecs]) {
+  load_segment_v<DT>(row, a.V, a.nvec, seg, raw);
 }
 
 // "Largest value, then lowest index" keys in 32 bits for bf16 values and
@@ -111,7 +120,8 @@ __device__ __forceinline__ float key32_value(uint32_t k) {
 __device__ __forceinline__ int key32_index(uint32_t k) { return (int)(0xFFFFu - (k & 0xFFFFu)); }
 
 // Statistics of one segment whose lane vectors are raw[0..kLaneVecs-1] (the
-// vectors seg*kSegVecs + lane + 32 j of the row), by one full warp.
+// vectors seg*kSegVecs + lane + 32 j of the row, -inf past its end), by one
+// full warp; row (V elements) is read again only by the top list, rarely.
 template <int DT, bool LSE, bool ARGMAX, bool TOP>
 __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], const char* row,
                                              int V, int seg, float k2, int topk, PartStat* out,
@@ -190,13 +200,18 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
 
   // ---- the k largest logits (value desc, index asc), saguaro draft rows.
   // The k largest lane maxima are k distinct elements, so every element of the
-  // segment's top k is at least T, the k-th largest lane maximum.  A branch-free
-  // pass marks the lane's 16-byte vectors whose largest element reaches T (and
-  // is above -inf); a small rolled loop then re-reads the marked vectors (few,
-  // unless many values tie) and inserts their elements >= T into the lane's
-  // sorted list, in index order so that ties keep the lower index.  An element
-  // of the segment's top k is in its own lane's top k, which the list keeps.
+  // segment's top k is at least T, the k-th largest lane maximum.  Only the
+  // lanes holding the k largest maxima (barring ties) have vectors whose
+  // largest element reaches T, mostly just one: a branch-free pass marks them,
+  // and those lanes read their marked vectors again, all at once, one 16-byte
+  // load each (L2 hits: the segment has just been streamed), inserting their
+  // elements >= T into a list of the 8 largest "value, then lower index" keys
+  // (sorted by a branch-free max/min network; 32-bit keys for bf16: value bits
+  // and the index within the segment).  An element of the segment's top k is
+  // in its own lane's top k, which the list keeps; k rounds of a warp maximum
+  // then merge the lists.
   if (TOP) {
+    using Key = typename std::conditional<DT == kBF16, uint32_t, unsigned long long>::type;
     float T = -INFINITY;
     if constexpr (DT == kBF16) {
       uint32_t mine = value_index_key32(m_t, lane);
@@ -229,66 +244,61 @@ __device__ __forceinline__ void stats_reduce(const uint4 (&raw)[kLaneVecs], cons
       mark = __funnelshift_l(hit, mark, 1);
     }
     mark <<= (32 - kLaneVecs);
-    float tv[kMaxTopK];
-    int ti[kMaxTopK];
+    Key lk[kMaxTopK];
 #pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s) {
-      tv[s] = -INFINITY;
-      ti[s] = INT_MAX;
-    }
-    while (mark) {
-      const int j = __clz((int)mark);
-      mark &= ~(0x80000000u >> j);
+    for (int q = 0; q < kMaxTopK; ++q) lk[q] = 0;
+    // the marked vectors again, each with one 16-byte load (the segment has
+    // just been streamed through L2), two at a time
+    const int nvec = (V + VEC - 1) / VEC, nfull = V / VEC;
+    const bool aligned = ((uintptr_t)row & 15u) == 0;
 #pragma unroll 1
-      for (int e = 0; e < VEC; ++e) {
-        const int x = (v0 + 32 * j) * VEC + e;
-        if (x >= V) break;
-        const float z = DT == kF32 ? ((const float*)row)[x]
-                                   : __uint_as_float((uint32_t)((const uint16_t*)row)[x] << 16);
-        if (z >= T && z > tv[kMaxTopK - 1]) {
-          tv[kMaxTopK - 1] = z;
-          ti[kMaxTopK - 1] = x;
+    while (mark) {
+      const int ja = __clz((int)mark);
+      mark &= ~(0x80000000u >> ja);
+      const int jb = mark ? __clz((int)mark) : -1;
+      if (jb >= 0) mark &= ~(0x80000000u >> jb);
+      const uint4 wa = load_vec_checked<DT>(row, v0 + 32 * ja, V, nvec, nfull, aligned);
+      const uint4 wb = jb >= 0 ? load_vec_checked<DT>(row, v0 + 32 * jb, V, nvec, nfull, aligned)
+                               : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+      for (int t = 0; t < 2 * VEC; ++t) {
+        const int j = t < VEC ? ja : jb;
+        if (j < 0) break;
+        const int e = t < VEC ? t : t - VEC;
+        const float z = elem<DT>(t < VEC ? wa : wb, e);
+        if (z >= T && z > -INFINITY) {
+          Key k;
+          if constexpr (DT == kBF16) k = value_index_key32(z, (lane + 32 * j) * VEC + e);
+          else k = value_index_key(z, (lane + 32 * j) * VEC + e);
 #pragma unroll
-          for (int s = kMaxTopK - 1; s > 0; --s) {
-            if (tv[s] > tv[s - 1]) {
-              const float fv = tv[s];
-              tv[s] = tv[s - 1];
-              tv[s - 1] = fv;
-              const int fi = ti[s];
-              ti[s] = ti[s - 1];
-              ti[s - 1] = fi;
-            }
+          for (int q = 0; q < kMaxTopK; ++q) {
+            const Key hi = lk[q] > k ? lk[q] : k;
+            k = lk[q] > k ? k : lk[q];
+            lk[q] = hi;
           }
         }
       }
     }
+    const int base = seg * kSegVecs * VEC;  // indices in the keys are relative to it
     int h = 0;
     for (int r = 0; r < topk; ++r) {
-      float hv = -INFINITY;
-      int hi = INT_MAX;
+      Key mine = 0;
 #pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s)
-        if (s == h) {
-          hv = tv[s];
-          hi = ti[s];
-        }
+      for (int q = 0; q < kMaxTopK; ++q)
+        if (q == h) mine = lk[q];
       if constexpr (DT == kBF16) {
-        // indices relative to the segment's first token (below 4096)
-        const int base = seg * kSegVecs * VEC;
-        const uint32_t key = hi == INT_MAX ? 0u : value_index_key32(hv, hi - base);
-        const uint32_t win = __reduce_max_sync(0xFFFFFFFFu, key);
-        if (win != 0u && key == win) ++h;
+        const uint32_t win = __reduce_max_sync(0xFFFFFFFFu, mine);
+        if (win != 0u && mine == win) ++h;
         if (lane == 0) {
           tout->v[r] = win ? key32_value(win) : -INFINITY;
           tout->i[r] = win ? off + base + key32_index(win) : INT_MAX;
         }
       } else {
-        const unsigned long long key = hi == INT_MAX ? 0ull : value_index_key(hv, hi);
-        const unsigned long long win = warp_max_u64(key);
-        if (win != 0ull && key == win) ++h;
+        const unsigned long long win = warp_max_u64(mine);
+        if (win != 0ull && mine == win) ++h;
         if (lane == 0) {
           tout->v[r] = win ? key_value(win) : -INFINITY;
-          tout->i[r] = win ? off + key_index(win) : INT_MAX;
+          tout->i[r] = win ? off + base + key_index(win) : INT_MAX;
         }
       }
     }
@@ -315,10 +325,14 @@ __device__ __forceinline__ void stats_segment(const VerifyArgs& a, const char* r
 
 // The statistics of a saguaro draft-row segment (with its top list), compiled
 // on its own so that the common path keeps its registers.
+// It takes scalars, not the argument block: a reference to that would make
+// every thread copy it to its stack at each call.
 template <int DT>
-__device__ __noinline__ void stats_segment_top(const VerifyArgs& a, const char* row, int seg,
-                                               float k2, int topk, PartStat* out, TopPart* tout) {
-  stats_segment<DT, true, false, true>(a, row, seg, k2, topk, out, tout);
+__device__ __noinline__ void stats_segment_top(const char* row, int V, int nvec, int seg, float k2,
+                                               int topk, int off, PartStat* out, TopPart* tout) {
+  uint4 raw[kLaneVecs];
+  load_segment_v<DT>(row, V, nvec, seg, raw);
+  stats_reduce<DT, true, false, true>(raw, row, V, seg, k2, topk, out, tout, off);
 }
 
 // Whether row `slot` of a request with parameters rp is read by the rule.
@@ -347,7 +361,7 @@ __device__ __forceinline__ void stats_item(const VerifyArgs& a, int b, int slot,
   } else if (rp.mode == kSaguaro) {
     if (WITH_TOP) {
       TopPart* tout = a.tpart + ((size_t)b * a.D_max + (slot - a.D_max - 1)) * a.nseg + seg;
-      stats_segment_top<DT>(a, row, seg, k2, a.saguaro_k, out, tout);
+      stats_segment_top<DT>(row, a.V, a.nvec, seg, k2, a.saguaro_k, a.vocab_offset, out, tout);
     } else if ((threadIdx.x & 31) == 0) {
       atomicOr(a.status, kFlagBadParam);
     }

@@ -48,7 +48,7 @@ __device__ __forceinline__ void finish_race(const VerifyArgs& a, int b, const Ra
     const char* trow = row_base(a, b, rd.n);
     Best Bb{-INFINITY, -INFINITY, -1};
     for (int s = 0; s < a.nseg; ++s)
-      Bb = combine(Bb, race_segment<DT>(a, rd, trow, nullptr, false, s, -INFINITY, INFINITY));
+      Bb = combine(Bb, race_segment<DT>(row_ctx(a), rd, trow, nullptr, false, s, -INFINITY, INFINITY));
     r = Bb;
   }
   if (lane == 0) {

@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
         __syncwarp();
         Best Bb{-INFINITY, -INFINITY, -1};
         for (int s = 0; s < a.nseg; ++s)
-          Bb = combine(Bb, race_segment<DT>(a, S.rd, trow, keep ? qrow : nullptr, keep, s,
+          Bb = combine(Bb, race_segment<DT>(row_ctx(a), S.rd, trow, keep ? qrow : nullptr, keep, s,
                                             -INFINITY, INFINITY));
         r = Bb;
       }

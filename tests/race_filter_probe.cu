@@ -26,7 +26,7 @@ __device__ void probe_segment(const VerifyArgs& a, const RaceDesc& rd, const cha
       keep_out[x] = ((drop >> (31 - t)) & 1u) ? 0 : 1;
       words[x] = race_word(a.seed, rd.g, x);
       exact[x] = exact_key_of(a, rd, trow, qrow, residual, x);
-      upper[x] = key2_upper(a, rd, trow, qrow, residual, x);
+      upper[x] = key2_upper(row_ctx(a), rd, trow, qrow, residual, x);
     }
   }
 }
