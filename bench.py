@@ -124,7 +124,7 @@ def tail_items(w, sms):
     GPU (three split launches) rather than one CTA per request (two)."""
     seg_tokens = 4096 if w.dtype == 1 else 2048
     nseg = -(-w.V // seg_tokens)
-    return w.B < sms and w.B * nseg > sms
+    return 5 * w.B < 4 * sms and w.B * nseg > sms
 
 
 def input_copies(in_bytes):

@@ -93,9 +93,9 @@ enum { SV_OK = 0, SV_ERR_INVALID_ARG = -1, SV_ERR_UNSUPPORTED = -2, SV_ERR_CUDA 
 
 /* sv_params.variant: the launch structure, optionally OR-ed
  * with one layout of the work after the statistics pass (both layouts give the
- * same results; without one, the library takes ITEMS when B is below the device's
- * multiprocessor count and B times the row's 8 KiB segments is above it, and
- * PER_REQUEST otherwise):
+ * same results; without one, the library takes ITEMS when B is below four
+ * fifths of the device's multiprocessor count and B times the row's 8 KiB
+ * segments is above that count, and PER_REQUEST otherwise):
  *   SV_TAIL_PER_REQUEST: one CTA per request merges, scans and races it;
  *   SV_TAIL_ITEMS: one CTA per request merges and scans, then one warp per
  *     (request, segment of the sampled row) races -- per half segment while

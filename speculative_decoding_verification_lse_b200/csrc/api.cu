@@ -271,9 +271,11 @@ int prepare_call(const void* target_logits, const void* draft_logits,
   a.nseg = nseg;
   a.slots = (int)slots;
   a.mode = mode;
-  // one CTA per request once every multiprocessor gets one, or when there are too few race
-  // segments to spread; else the scan, then race items over the whole GPU
-  const bool spread = B < sms && (long long)B * nseg > sms;
+  // one CTA per request once the requests fill four fifths of the multiprocessors (each
+  // request's race then has a multiprocessor to itself, and one launch less beats spreading
+  // the races over the rest), or when there are too few race segments to spread; else the
+  // scan, then race items over the whole GPU
+  const bool spread = 5LL * B < 4LL * sms && (long long)B * nseg > sms;
   a.per_request = tail_bits == SV_TAIL_PER_REQUEST ? 1 : tail_bits == SV_TAIL_ITEMS ? 0 : (spread ? 0 : 1);
   // the fused kernel races half segments; the split path cuts them while one wave holds them
   a.rsplit = fused ? kMaxRaceSplit : a.per_request ? 1 : race_split(B, nseg, dtype, sms);
