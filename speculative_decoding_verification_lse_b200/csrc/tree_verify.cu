@@ -38,20 +38,41 @@ struct TreeShared {
 };
 
 // sum over the row of max(0, p(x) - c q(x)) for target row pos and draft row
-// pos of request b, by the whole CTA in a fixed order (each thread its strided
-// tokens, then the warps, then the CTA, in double).
+// pos of request b, by the whole CTA in a fixed order: thread t takes the
+// 16-byte vectors t, t + kThreads, ... of both rows, four of each in flight at
+// once, sums each vector's terms in single precision and adds that to its
+// double accumulator; then the warps, then the CTA, in double.
 template <int DT>
 __device__ double residual_mass(const VerifyArgs& a, int b, int pos, double lse_t, double lse_q,
                                 float k2, double c, TreeShared& T) {
+  constexpr int VEC = DT == kF32 ? 4 : 8;
+  constexpr int U = 4;
   const char* trow = row_base(a, b, pos);
   const char* qrow = row_base(a, b, a.D_max + 1 + pos);
   const float lt = (float)(lse_t * 1.4426950408889634), lq = (float)(lse_q * 1.4426950408889634);
   const float cf = (float)c;
+  const int nfull = a.V / VEC;
+  const bool aligned = ((uintptr_t)trow & 15u) == 0 && ((uintptr_t)qrow & 15u) == 0;
   double acc = 0.0;
-  for (int x = threadIdx.x; x < a.V; x += kThreads) {
-    const float p = ex2_approx(fmaf(logit_at<DT>(trow, x), k2, -lt));
-    const float q = ex2_approx(fmaf(logit_at<DT>(qrow, x), k2, -lq));
-    acc += (double)fmaxf(0.0f, fmaf(-cf, q, p));
+  for (int v0 = threadIdx.x; v0 < a.nvec; v0 += U * kThreads) {
+    uint4 wt[U], wq[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      // past the row's end: -inf, whose terms are 0
+      wt[u] = load_vec_checked<DT>(trow, v0 + u * kThreads, a.V, a.nvec, nfull, aligned);
+      wq[u] = load_vec_checked<DT>(qrow, v0 + u * kThreads, a.V, a.nvec, nfull, aligned);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float sv = 0.0f;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float p = ex2_approx(fmaf(elem<DT>(wt[u], e), k2, -lt));
+        const float q = ex2_approx(fmaf(elem<DT>(wq[u], e), k2, -lq));
+        sv += fmaxf(0.0f, fmaf(-cf, q, p));
+      }
+      acc += (double)sv;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
