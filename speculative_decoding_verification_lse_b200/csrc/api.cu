@@ -175,6 +175,7 @@ struct Call {
   unsigned int* status;
   int grid, base_variant;
   bool fused;
+  int sms = 0;  // the device's multiprocessors
 };
 
 // Everything sv_verify_ex does before its launches: the argument checks, the
@@ -290,6 +291,7 @@ int prepare_call(const void* target_logits, const void* draft_logits,
   call->grid = grid;
   call->base_variant = base_variant;
   call->fused = fused;
+  call->sms = sms;
   return SV_OK;
 }
 
@@ -526,7 +528,7 @@ int sv_verify_tree(const void* target_logits, const void* draft_logits,
   if ((e = launch_row_stats(a, s, call.grid, tickets)) != cudaSuccess)
     return cuda_fail(e, "row statistics launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  if ((e = launch_tree(a, s)) != cudaSuccess) return cuda_fail(e, "tree walk launch");
+  if ((e = launch_tree(a, s, call.sms)) != cudaSuccess) return cuda_fail(e, "tree walk launch");
   return SV_OK;
 }
 

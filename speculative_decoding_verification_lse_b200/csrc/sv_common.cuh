@@ -385,7 +385,9 @@ cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);
 cudaError_t launch_cluster(const VerifyArgs& a, cudaStream_t s);
-cudaError_t launch_tree(const VerifyArgs& a, cudaStream_t s);
+// One cluster of up to 4 CTAs per request (as many as fit one CTA per
+// multiprocessor: sms of them).
+cudaError_t launch_tree(const VerifyArgs& a, cudaStream_t s, int sms);
 ShardLayout shard_layout(int B, int D_max, int V_local, int dtype);
 cudaError_t launch_shard_z(const VerifyArgs& a, void* zx, cudaStream_t s);
 cudaError_t launch_shard_tail(const VerifyArgs& a, const void* gathered1, int n_shards,

@@ -1,5 +1,5 @@
 // tree_verify.cu -- tree (multi-candidate) verification after the statistics
-// pass: one CTA per request walks its draft tree from the root.
+// pass: one thread-block cluster per request walks its draft tree from the root.
 //
 // "Accélérer Sonar par la Spéculation", section "EAGLE": the draft proposes a
 // tree whose nodes hold several candidate tokens.  At position p (the root, or
@@ -15,14 +15,24 @@
 // the position's target and draft rows (the sum N, by the whole CTA, in a fixed
 // order), and the final draw is the residual race with q scaled by c_K -- the
 // linear path's race with the draft row's log-normaliser lowered by ln c_K.
+//
+// The C CTAs of a request's cluster (C = 1, 2 or 4) all merge the rows and take
+// the same decisions from the same numbers; each residual pass and the race
+// are split over all of them: a pass's partial sums are exchanged through
+// distributed shared memory and added in rank order (so every CTA holds the
+// same N), and rank 0 combines the race results and writes the outputs.
 // The accept uniform of candidate node i is word 0 of Philox at counter
 // (i, g, 0, 0), so a chain (one candidate per position) is the linear rule
 // exactly.  Greedy: the first candidate holding the target row's argmax is
 // accepted; otherwise that argmax is emitted.
+#include <cooperative_groups.h>
+
 #include <cstring>
 
 #include "specverify.h"
 #include "tail_device.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace sv {
 
@@ -35,16 +45,22 @@ struct TreeShared {
   uint32_t flags;
   double c, N, c_prev;
   double red[kWarps];
+  double part[2];  // this CTA's partial of the residual pass, by pass parity
+  Best rb;         // this CTA's race result
 };
 
 // sum over the row of max(0, p(x) - c q(x)) for target row pos and draft row
-// pos of request b, by the whole CTA in a fixed order: thread t takes the
-// 16-byte vectors t, t + kThreads, ... of both rows, four of each in flight at
-// once, sums each vector's terms in single precision and adds that to its
-// double accumulator; then the warps, then the CTA, in double.
+// pos of request b, by the whole cluster in a fixed order: thread t of rank r
+// takes the 16-byte vectors r kThreads + t + i C kThreads of both rows, four of
+// each in flight at once, sums each vector's terms in single precision and
+// adds that to its double accumulator; then the warps, the CTA (in double),
+// and the ranks in order through distributed shared memory.  Every thread of
+// the cluster returns the same value; `parity` alternates between calls.
 template <int DT>
 __device__ double residual_mass(const VerifyArgs& a, int b, int pos, double lse_t, double lse_q,
-                                float k2, double c, TreeShared& T) {
+                                float k2, double c, TreeShared& T, cg::cluster_group& cluster,
+                                int parity) {
+  const int C = (int)cluster.num_blocks(), r = (int)cluster.block_rank();
   constexpr int VEC = DT == kF32 ? 4 : 8;
   constexpr int U = 4;
   const char* trow = row_base(a, b, pos);
@@ -53,14 +69,15 @@ __device__ double residual_mass(const VerifyArgs& a, int b, int pos, double lse_
   const float cf = (float)c;
   const int nfull = a.V / VEC;
   const bool aligned = ((uintptr_t)trow & 15u) == 0 && ((uintptr_t)qrow & 15u) == 0;
+  const int stride = C * kThreads;
   double acc = 0.0;
-  for (int v0 = threadIdx.x; v0 < a.nvec; v0 += U * kThreads) {
+  for (int v0 = r * kThreads + threadIdx.x; v0 < a.nvec; v0 += U * stride) {
     uint4 wt[U], wq[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       // past the row's end: -inf, whose terms are 0
-      wt[u] = load_vec_checked<DT>(trow, v0 + u * kThreads, a.V, a.nvec, nfull, aligned);
-      wq[u] = load_vec_checked<DT>(qrow, v0 + u * kThreads, a.V, a.nvec, nfull, aligned);
+      wt[u] = load_vec_checked<DT>(trow, v0 + u * stride, a.V, a.nvec, nfull, aligned);
+      wq[u] = load_vec_checked<DT>(qrow, v0 + u * stride, a.V, a.nvec, nfull, aligned);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -78,18 +95,27 @@ __device__ double residual_mass(const VerifyArgs& a, int b, int pos, double lse_
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
   if ((threadIdx.x & 31) == 0) T.red[threadIdx.x >> 5] = acc;
   __syncthreads();
-  double s = 0.0;
-  for (int w = 0; w < kWarps; ++w) s += T.red[w];
-  __syncthreads();
-  return s;
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int w = 0; w < kWarps; ++w) s += T.red[w];
+    T.part[parity] = s;
+  }
+  // (a pass's slot is written again two passes later, after every rank has
+  // read it: each rank reads before it reaches the next pass's barrier)
+  cluster.sync();
+  double N = 0.0;
+  for (int k = 0; k < C; ++k) N += *cluster.map_shared_rank(&T.part[parity], k);
+  return N;
 }
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
   __shared__ TailShared S;
   __shared__ TreeShared T;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
   wait_for_previous_kernel();
-  const int b = blockIdx.x;
+  const int b = (int)(blockIdx.x / (unsigned)C);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Dm = a.D_max;
   const ReqParams rp = load_req(a, b);
@@ -127,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
     if (threadIdx.x == 0) T.flags |= bad;
     __syncthreads();
   }
-  if (a.out_row_lse) {
+  if (a.out_row_lse && rank == 0) {
     // natural-log LSE of every row the walk may read (stochastic requests), NaN elsewhere
     const bool ok = !(T.flags & kFlagErrors) && rp.mode != kGreedy;
     for (int s = threadIdx.x; s < a.slots; s += kThreads)
@@ -135,6 +161,8 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
           ok && slot_needed(a, b, s, rp) ? (float)S.rows[s].lse : NAN;
   }
   if (T.flags & kFlagErrors) {
+    // (every rank of the cluster returns here: the flags come from the same numbers)
+    if (rank != 0) return;
     for (int j = threadIdx.x; j <= Dm; j += kThreads) ot[j] = -1;
     if (a.out_nodes)
       for (int j = threadIdx.x; j < Dm; j += kThreads) a.out_nodes[(size_t)b * Dm + j] = -1;
@@ -149,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
   const bool greedy = rp.mode == kGreedy;
   const double Td = (double)rp.T;
   const float k2 = greedy ? 0.0f : log2e_over_T(rp.T);
+  int passes = 0;
   for (;;) {
     const int pos = T.pos;
     if (greedy) {
@@ -184,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
       if (any) {
         // the previous candidate was rejected: the residual for this one
         const double cn = T.c + T.N;
-        const double Nn = residual_mass<DT>(a, b, pos, lse_t, lse_q, k2, cn, T);
+        const double Nn = residual_mass<DT>(a, b, pos, lse_t, lse_q, k2, cn, T, cluster, passes & 1);
+        ++passes;
         if (threadIdx.x == 0) {
           if (Nn > 0.0) {
             T.c = cn;
@@ -281,7 +311,9 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
     for (int w = 1; w < kWarps; ++w) K0 = fmax(K0, S.key[w]);
     const char* trow = row_base(a, b, pos);
     const char* qrow = residual ? row_base(a, b, Dm + 1 + pos) : nullptr;
-    const Best Bw = race_span_in<DT>(a, S.rd, R, trow, qrow, residual, warp, kWarps, K0, &S.k0);
+    // the cluster's C * kWarps warps race the row's segments
+    const Best Bw = race_span_in<DT>(a, S.rd, R, trow, qrow, residual, rank * kWarps + warp,
+                                     C * kWarps, K0, &S.k0);
     if (lane == 0) {
       S.best[warp] = Bw.best;
       S.second[warp] = Bw.second;
@@ -295,6 +327,14 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
         r.second = S.second[lane];
         r.idx = S.idx[lane];
       }
+      r = warp_combine(r);
+      if (lane == 0) T.rb = r;
+    }
+    cluster.sync();
+    if (rank == 0 && warp == 0) {
+      // the ranks' results, in rank order
+      Best r{-INFINITY, -INFINITY, -1};
+      if (lane < C) r = *cluster.map_shared_rank(&T.rb, lane);
       r = warp_combine(r);
       uint32_t flags = T.flags;
       if (r.idx < 0 && residual) {
@@ -317,9 +357,11 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
         T.flags = flags;
       }
     }
-    __syncthreads();
+    // the other ranks' shared memory stays until rank 0 has read it
+    cluster.sync();
     emitted = T.emitted;
   }
+  if (rank != 0) return;
   // outputs: the accepted path's tokens, then the drawn or argmax token
   for (int j = threadIdx.x; j <= Dm; j += kThreads)
     ot[j] = j < len ? __ldg(&tok[T.path[j]]) : (j == len ? emitted : -1);
@@ -335,18 +377,24 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
 
 }  // namespace
 
-cudaError_t launch_tree(const VerifyArgs& a, cudaStream_t s) {
+cudaError_t launch_tree(const VerifyArgs& a, cudaStream_t s, int sms) {
   if (a.B == 0) return cudaSuccess;
+  int C = 4;
+  while (C > 1 && (long long)a.B * C > sms) C /= 2;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof cfg);
-  cfg.gridDim = dim3(a.B);
+  cfg.gridDim = dim3((unsigned)a.B * (unsigned)C);
   cfg.blockDim = dim3(kThreads);
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return a.dtype == kF32 ? cudaLaunchKernelEx(&cfg, tree_kernel<kF32>, a)
                          : cudaLaunchKernelEx(&cfg, tree_kernel<kBF16>, a);
 }

@@ -46,6 +46,16 @@ def test_tree_matches_the_oracle(sv, branching, mode):
         compare_tree(tree_gpu(w, seed), tree_oracle(w, seed), 22)
 
 
+@pytest.mark.parametrize("B", [30, 60, 160])
+def test_tree_every_cluster_size(sv, B):
+    # the walk spreads a request over a cluster of 4, 2 or 1 CTAs, as many as
+    # fit one CTA per multiprocessor (on 148 of them: 4 for B=30, 2 for B=60,
+    # 1 for B=160); the outputs are the oracle's whatever the size
+    w = wl.make_tree("tree", "cuda", B=B, V=5003, branching=(3, 2, 2))
+    for seed in range(2):
+        compare_tree(tree_gpu(w, seed), tree_oracle(w, seed), B - 2)
+
+
 def test_chain_tree_is_the_linear_path(sv):
     for name in ("b32", "b256", "tiny"):
         w = wl.make(name, "cuda", B=None if name == "tiny" else 16, V=None if name == "tiny" else 30011)
