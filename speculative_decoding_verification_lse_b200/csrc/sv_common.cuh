@@ -385,7 +385,7 @@ cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);
 cudaError_t launch_cluster(const VerifyArgs& a, cudaStream_t s);
-// One cluster of up to 4 CTAs per request (as many as fit one CTA per
+// One cluster of up to 4 CTAs per request (as many as fit two CTAs per
 // multiprocessor: sms of them).
 cudaError_t launch_tree(const VerifyArgs& a, cudaStream_t s, int sms);
 ShardLayout shard_layout(int B, int D_max, int V_local, int dtype);

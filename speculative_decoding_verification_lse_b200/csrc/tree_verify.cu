@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
 cudaError_t launch_tree(const VerifyArgs& a, cudaStream_t s, int sms) {
   if (a.B == 0) return cudaSuccess;
   int C = 4;
-  while (C > 1 && (long long)a.B * C > sms) C /= 2;
+  while (C > 1 && (long long)a.B * C > 2LL * sms) C /= 2;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = dim3((unsigned)a.B * (unsigned)C);

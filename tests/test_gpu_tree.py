@@ -46,10 +46,10 @@ def test_tree_matches_the_oracle(sv, branching, mode):
         compare_tree(tree_gpu(w, seed), tree_oracle(w, seed), 22)
 
 
-@pytest.mark.parametrize("B", [30, 60, 160])
+@pytest.mark.parametrize("B", [30, 100, 160])
 def test_tree_every_cluster_size(sv, B):
     # the walk spreads a request over a cluster of 4, 2 or 1 CTAs, as many as
-    # fit one CTA per multiprocessor (on 148 of them: 4 for B=30, 2 for B=60,
+    # fit two CTAs per multiprocessor (on 148 of them: 4 for B=30, 2 for B=100,
     # 1 for B=160); the outputs are the oracle's whatever the size
     w = wl.make_tree("tree", "cuda", B=B, V=5003, branching=(3, 2, 2))
     for seed in range(2):
