@@ -365,7 +365,7 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     return cuda_fail(e, "row statistics launch");
   if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if (a.per_request) {
-    if ((e = launch_requests(a, s)) != cudaSuccess) return cuda_fail(e, "scan and race launch");
+    if ((e = launch_requests(a, s, call.sms)) != cudaSuccess) return cuda_fail(e, "scan and race launch");
   } else {
     if ((e = launch_scan(a, s)) != cudaSuccess) return cuda_fail(e, "accept scan launch");
     if ((e = launch_race(a, s)) != cudaSuccess) return cuda_fail(e, "race launch");

@@ -380,7 +380,10 @@ int row_stats_blocks_per_sm(int dtype);
 cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
 int race_split(int B, int nseg, int dtype, int sms);
-cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s);
+// One CTA per request, or a cluster of 2 or 4 while B times that fits two CTAs
+// on each of the sms multiprocessors.
+cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s, int sms);
+int request_cluster_size(int B, int sms);
 cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);

@@ -112,6 +112,78 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
   __syncthreads();  // S is reused by the next request
 }
 
+// Request b by the C CTAs of a thread-block cluster (C > 1): rank 0 merges the
+// rows, runs the accept scan and finds the reference key, as tail_request
+// does; the other ranks copy its race description through distributed shared
+// memory, and the cluster's C * kWarps warps race the sampled row (warp w of
+// rank r taking segments 8r + w, 8r + w + 8C, ...); rank 0 combines the ranks'
+// results in rank order and writes the token.  rb: this CTA's slot for its
+// result.  Every thread of the cluster returns at the same point.
+template <int DT, class Cluster>
+__device__ __forceinline__ void tail_request_cluster(const VerifyArgs& a, int b, TailShared& S,
+                                                     Cluster& cluster, Best* rb) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+  const RaceStream R = race_stream(a.seed, a.request_offset + (uint32_t)b, (uint32_t)a.vocab_offset >> 2);
+  if (rank == 0) {
+    const ReqParams rp = load_req(a, b);
+    if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
+    for (int slot = warp; slot < a.slots; slot += kWarps)
+      if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
+    __syncthreads();
+    if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
+    __syncthreads();
+    if (S.rd.kind != kRaceNone) {
+      const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
+      if (lane == 0) S.key[warp] = kw;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        double K0 = S.key[0];
+        for (int w = 1; w < kWarps; ++w) K0 = fmax(K0, S.key[w]);
+        S.rd.K0 = K0;
+      }
+    }
+  }
+  cluster.sync();  // rank 0's race description is complete
+  constexpr int d16 = sizeof(RaceDesc) / 16;
+  static_assert(sizeof(RaceDesc) % 16 == 0, "RaceDesc is copied in 16-byte pieces");
+  if (rank != 0 && threadIdx.x < d16)
+    reinterpret_cast<uint4*>(&S.rd)[threadIdx.x] =
+        reinterpret_cast<const uint4*>(cluster.map_shared_rank(&S.rd, 0))[threadIdx.x];
+  if (threadIdx.x == 0) S.k0 = ordered_u64(-INFINITY);
+  cluster.sync();  // the copies are done before rank 0 goes on
+  const int kind = S.rd.kind;
+  if (kind == kRaceNone) return;
+  const bool residual = kind == kRaceResidual;
+  const char* trow = row_base(a, b, S.rd.n);
+  const char* qrow = residual ? row_base(a, b, a.D_max + 1 + S.rd.n) : nullptr;
+  const Best B = race_span_in<DT>(a, S.rd, R, trow, qrow, residual, rank * kWarps + warp,
+                                  C * kWarps, S.rd.K0, &S.k0);
+  if (lane == 0) {
+    S.best[warp] = B.best;
+    S.second[warp] = B.second;
+    S.idx[warp] = B.idx;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    Best r{-INFINITY, -INFINITY, -1};
+    if (lane < kWarps) {
+      r.best = S.best[lane];
+      r.second = S.second[lane];
+      r.idx = S.idx[lane];
+    }
+    r = warp_combine(r);
+    if (lane == 0) *rb = r;
+  }
+  cluster.sync();  // every rank's result is in place
+  if (rank == 0 && warp == 0) {
+    Best r{-INFINITY, -INFINITY, -1};
+    if (lane < C) r = *cluster.map_shared_rank(rb, lane);
+    finish_race<DT>(a, b, S.rd, warp_combine(r));
+  }
+  cluster.sync();  // the other ranks' shared memory stays until rank 0 has read it
+}
+
 // Request b, by the whole CTA (kThreads threads, S in shared memory); every
 // thread returns at the same point.  Writes the request's outputs (all of them
 // unless it races), and for a race a.rdesc[b] and the race counters.

@@ -2,10 +2,14 @@
 // (tail_device.cuh): either one CTA per request for everything, or the accept
 // scan (one CTA per request) followed by the race (one warp per request and
 // segment of the sampled row).
+#include <cooperative_groups.h>
+
 #include <atomic>
 #include <cstring>
 
 #include "tail_device.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace sv {
 
@@ -26,6 +30,16 @@ __global__ void __launch_bounds__(kThreads, 2) request_kernel(VerifyArgs a) {
   __shared__ TailShared S;
   wait_for_previous_kernel();
   tail_request<DT>(a, (int)blockIdx.x, S);
+}
+
+// One cluster of C CTAs per request (tail_request_cluster).
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 2) request_cluster_kernel(VerifyArgs a) {
+  __shared__ TailShared S;
+  __shared__ Best rb;
+  cg::cluster_group cluster = cg::this_cluster();
+  wait_for_previous_kernel();
+  tail_request_cluster<DT>(a, (int)(blockIdx.x / cluster.num_blocks()), S, cluster, &rb);
 }
 
 template <int DT>
@@ -63,10 +77,36 @@ cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s) {
                          : launch_dependent(scan_kernel<kBF16>, a.B, s, a);
 }
 
-cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s) {
+// A cluster of C = 4 or 2 CTAs per request while B C fits two CTAs per
+// multiprocessor (sms of them), else one CTA per request.
+int request_cluster_size(int B, int sms) {
+  int C = 4;
+  while (C > 1 && (long long)B * C > 2LL * sms) C /= 2;
+  return C;
+}
+
+cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s, int sms) {
   if (a.B == 0) return cudaSuccess;
-  return a.dtype == kF32 ? launch_dependent(request_kernel<kF32>, a.B, s, a)
-                         : launch_dependent(request_kernel<kBF16>, a.B, s, a);
+  const int C = request_cluster_size(a.B, sms);
+  if (C == 1)
+    return a.dtype == kF32 ? launch_dependent(request_kernel<kF32>, a.B, s, a)
+                           : launch_dependent(request_kernel<kBF16>, a.B, s, a);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3((unsigned)a.B * (unsigned)C);
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return a.dtype == kF32 ? cudaLaunchKernelEx(&cfg, request_cluster_kernel<kF32>, a)
+                         : cudaLaunchKernelEx(&cfg, request_cluster_kernel<kBF16>, a);
 }
 
 // Race items per segment: a race warp is bound by its own chain of Philox
