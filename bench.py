@@ -127,6 +127,28 @@ def tail_items(w, sms):
     return 5 * w.B < 4 * sms and w.B * nseg > sms
 
 
+def early_exit_bounds(D_max):
+    """The position rounds of SV_VARIANT_EARLY_EXIT (the library's rule, in
+    include/specverify.h): position 0, then 1-2, then 3 to D_max."""
+    return [0] + [p for p in (1, 3) if p < D_max + 1] + [D_max + 1]
+
+
+def early_exit_rows(accept_len, row_D, modes, D_max):
+    """Rows the early-exit rounds read for outcomes accept_len (n = AL - 1): a
+    request listed in a round reads every row of the round's positions up to
+    D_b (draft rows only for sampling requests), plus the race's row."""
+    bounds = early_exit_bounds(D_max)
+    rows = 0
+    for al, Db, m in zip(accept_len, row_D, modes):
+        n = al - 1
+        if n < 0:
+            continue  # a parameter error: nothing read
+        end = next(p1 for p0, p1 in zip(bounds, bounds[1:]) if p0 <= n < p1)
+        last = min(end - 1, Db)
+        rows += (last + 1) + (0 if m == 1 else min(end, Db) + 1)  # target, draft + race row
+    return rows
+
+
 def input_copies(in_bytes):
     """How many copies of a step's inputs the timed loop rotates over: enough
     that together they are at least twice the L2 (at most MAX_INPUT_COPIES),
@@ -371,7 +393,8 @@ def run_ours(args):
     variant = {"auto": sv.SV_VARIANT_AUTO, "split": sv.SV_VARIANT_SPLIT,
                "split-items": sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
                "split-per-request": sv.SV_VARIANT_SPLIT | sv.SV_TAIL_PER_REQUEST,
-               "fused": sv.SV_VARIANT_FUSED, "cluster": sv.SV_VARIANT_CLUSTER}[args.variant]
+               "fused": sv.SV_VARIANT_FUSED, "cluster": sv.SV_VARIANT_CLUSTER,
+               "early-exit": sv.SV_VARIANT_EARLY_EXIT}[args.variant]
 
     # every rank verifies its own batch (its own seed and request range)
     tree = args.workload in workloads.TREE_CONFIGS
@@ -468,6 +491,16 @@ def run_ours(args):
     k_med = statistics.median(k_list)
     ms_per_step = ms / args.steps
     rows_total = w.verified_rows() * args.steps * world
+    ee_rows = None
+    if args.variant == "early-exit" and not tree:
+        # the rows the timed steps read, from their outcomes (each step again,
+        # untimed: the same inputs and seeds give the same outcomes)
+        ee_rows = 0
+        for i in range(args.steps):
+            step(args.warmup + i)
+            ee_rows += early_exit_rows(out["accept_len"].cpu().tolist(), w.row_D_list(),
+                                       w.modes(), w.D_max)
+        ee_rows /= args.steps
     value = rows_total / (ms / 1e3)
 
     # acceptance: mean AL and its histogram (for saguaro next to the plain rule
@@ -541,7 +574,14 @@ def run_ours(args):
         peak, peak_kind = measured_peak()
         step_bytes = w.algorithmic_bytes()
         used_variant = args.variant if args.variant != "auto" else "split"
-        if used_variant in ("fused", "cluster"):
+        if ee_rows is not None:
+            # the bytes the rounds read (the rows up to each request's outcome)
+            # and the race's rows; the rounds are the timed kernels
+            step_bytes = int(ee_rows * w.V * (2 if w.dtype == 1 else 4))
+            kname = "early_exit_rounds"
+            kbytes = int((ee_rows - sum(m != 1 for m in w.modes())) * w.V * (2 if w.dtype == 1 else 4))
+            ksrc = ["speculative_decoding_verification_lse_b200/csrc/early_exit.cu"]
+        elif used_variant in ("fused", "cluster"):
             main = "fused_verify.cu" if used_variant == "fused" else "cluster_verify.cu"
             kname, kbytes = main[:-3], step_bytes
             ksrc = ["speculative_decoding_verification_lse_b200/csrc/" + f
@@ -608,7 +648,10 @@ def run_ours(args):
                 f"untimed steps after the timed region, every step the same call")),
             # fused: one launch; split: statistics, then one kernel per request or
             # the scan and the race items (the library's rule, in include/specverify.h)
-            "gpu_launches": (2 if tree else 1 if used_variant in ("fused", "cluster") else
+            "gpu_launches": (2 * (len(early_exit_bounds(w.D_max)) - 1) + (
+                                 2 if tail_items(w, torch.cuda.get_device_properties(dev).multi_processor_count)
+                                 else 1) if ee_rows is not None else
+                             2 if tree else 1 if used_variant in ("fused", "cluster") else
                              3 if (used_variant == "split-items" or (used_variant == "split" and tail_items(
                                  w, torch.cuda.get_device_properties(dev).multi_processor_count)))
                              else 2) * args.steps,
@@ -632,7 +675,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="b256")
     ap.add_argument("--variant", choices=["auto", "split", "split-items", "split-per-request",
-                                          "fused", "cluster"], default="auto")
+                                          "fused", "cluster", "early-exit"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -107,8 +107,24 @@ enum { SV_OK = 0, SV_ERR_INVALID_ARG = -1, SV_ERR_UNSUPPORTED = -2, SV_ERR_CUDA 
  *   SV_VARIANT_CLUSTER: one launch, one thread-block cluster (up to 8 CTAs) per
  *     request doing its statistics, merges, scan and race between cluster
  *     barriers;
- *   SV_VARIANT_AUTO: the library's choice for the shape. */
-enum { SV_VARIANT_AUTO = 0, SV_VARIANT_SPLIT = 1, SV_VARIANT_FUSED = 2, SV_VARIANT_CLUSTER = 3 };
+ *   SV_VARIANT_EARLY_EXIT: the rows read position by position, in rounds
+ *     (position 0, then 1-2, then 3 to D_max), each round only for the requests
+ *     that accepted every earlier draft, then the layout above; the rule's
+ *     rows after the first rejection are never read.  Same tokens, accepted
+ *     lengths and flags as SPLIT, except that the rows of the positions past
+ *     the outcome get no LSE (out_row_lse NaN), and those never read no
+ *     SV_FLAG_NONFINITE check.  Source: the rule
+ *     stops at the first rejection ("Speculative Speculative Decoding –
+ *     асинхронизируй это.", rule items 1-2);
+ *   SV_VARIANT_AUTO: the library's choice for the shape (never EARLY_EXIT,
+ *     whose outputs differ in out_row_lse). */
+enum {
+  SV_VARIANT_AUTO = 0,
+  SV_VARIANT_SPLIT = 1,
+  SV_VARIANT_FUSED = 2,
+  SV_VARIANT_CLUSTER = 3,
+  SV_VARIANT_EARLY_EXIT = 4
+};
 enum { SV_TAIL_PER_REQUEST = 1 << 4, SV_TAIL_ITEMS = 1 << 5 };
 
 /* per-request flag bits (sv_params.out_flags) */

@@ -15,6 +15,7 @@ SV_F32, SV_BF16 = 0, 1
 SV_STOCHASTIC, SV_GREEDY, SV_SAGUARO = 0, 1, 2
 SV_OK, SV_ERR_INVALID_ARG, SV_ERR_UNSUPPORTED, SV_ERR_CUDA = 0, -1, -2, -3
 SV_VARIANT_AUTO, SV_VARIANT_SPLIT, SV_VARIANT_FUSED, SV_VARIANT_CLUSTER = 0, 1, 2, 3
+SV_VARIANT_EARLY_EXIT = 4
 SV_TAIL_PER_REQUEST, SV_TAIL_ITEMS = 1 << 4, 1 << 5
 
 SV_FLAG_ACCEPT_NEAR_TIE = 1 << 0

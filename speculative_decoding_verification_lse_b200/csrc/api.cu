@@ -142,7 +142,7 @@ int check_args(const void* target_logits, const void* draft_logits, const int32_
     return fail(SV_ERR_INVALID_ARG, "saguaro_c must be in (0, 1] (got %g)", (double)c);
   const int tail_bits = prm.variant & (SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
   const int base_variant = prm.variant & ~(SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS);
-  if (base_variant < SV_VARIANT_AUTO || base_variant > SV_VARIANT_CLUSTER ||
+  if (base_variant < SV_VARIANT_AUTO || base_variant > SV_VARIANT_EARLY_EXIT ||
       tail_bits == (SV_TAIL_PER_REQUEST | SV_TAIL_ITEMS))
     return fail(SV_ERR_INVALID_ARG, "unknown variant %d", prm.variant);
   if (B == 0) return SV_OK;
@@ -357,13 +357,24 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     return run_epilogue(prm, out_tokens, out_accept_len, B, D_max, status, s);
   }
-  const bool tickets = row_stats_tickets(a, grid);
-  if (tickets && (e = cudaMemsetAsync(a.ticket, 0, 8 * 128, s)) != cudaSuccess)
-    return cuda_fail(e, "cudaMemsetAsync(ticket)");
-  if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  if ((e = launch_row_stats(a, s, grid, tickets)) != cudaSuccess)
-    return cuda_fail(e, "row statistics launch");
-  if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if (base_variant == SV_VARIANT_EARLY_EXIT) {
+    // the rows position by position, then the usual finish from the merged rows
+    a.ee_n = (int*)((char*)ws + L.ee);
+    a.ee_alive = a.ee_n + B;
+    a.ee_count = (unsigned int*)((char*)ws + align_up(L.ee + (size_t)3 * B * sizeof(int), 128));
+    if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = launch_early_exit_rounds(a, s, grid)) != cudaSuccess)
+      return cuda_fail(e, "early-exit rounds launch");
+    if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  } else {
+    const bool tickets = row_stats_tickets(a, grid);
+    if (tickets && (e = cudaMemsetAsync(a.ticket, 0, 8 * 128, s)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync(ticket)");
+    if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = launch_row_stats(a, s, grid, tickets)) != cudaSuccess)
+      return cuda_fail(e, "row statistics launch");
+    if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  }
   if (a.per_request) {
     if ((e = launch_requests(a, s, call.sms)) != cudaSuccess) return cuda_fail(e, "scan and race launch");
   } else {

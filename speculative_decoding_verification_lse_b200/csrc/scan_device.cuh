@@ -186,6 +186,37 @@ __device__ __forceinline__ ScanInputs scan_inputs(const VerifyArgs& a, int b, co
   return in;
 }
 
+// The accept test of draft position d of a request with parameters rp, from
+// its merged rows (rows[d] the target row, rows[D_max + 1 + d] the draft row)
+// and the scan inputs of lane d: greedy -- the draft token is the target
+// row's argmax; otherwise u_d < min(1, p(x_d) / q'(x_d)).  *near: |u - a| <
+// 1e-5 (sampling requests).
+__device__ inline bool accept_position(const VerifyArgs& a, const ReqParams& rp,
+                                       const RowRes* rows, const ScanInputs& in, int d,
+                                       bool* near) {
+  *near = false;
+  if (rp.mode == kGreedy) return in.x == rows[d].argmax;
+  const double Td = (double)rp.T;
+  const RowRes& rq = rows[a.D_max + 1 + d];
+  const double lp = (double)in.zt / Td - rows[d].lse;
+  double lq = (double)in.zq / Td - rq.lse;
+  if (rp.mode == kSaguaro && lq != -INFINITY) {
+    bool in_k = false;
+    for (int i = 0; i < rq.ntop; ++i) in_k |= (rq.top[i] == in.x);
+    lq += (in_k ? log((double)a.saguaro_c) : 0.0) - rq.lnZ;
+  }
+  double acc;
+  if (lp == -INFINITY)
+    acc = 0.0;  // p(x) = 0: the target never emits x
+  else if (lq == -INFINITY)
+    acc = 1.0;
+  else
+    acc = fmin(1.0, exp(lp - lq));
+  const double u = (double)(in.uw >> 8) * 0x1p-24;
+  *near = fabs(u - acc) < 1e-5;
+  return u < acc;
+}
+
 // The accept scan of request b by one full warp, once every row it reads has
 // been merged into rows (2*D_max+1 entries of shared memory); in: the warp's
 // scan_inputs.  Writes the
@@ -243,30 +274,7 @@ __device__ inline int scan_request(const VerifyArgs& a, int b, const RowRes* row
 
   // test every draft position in parallel
   bool accept = false, near = false;
-  if (lane < rp.Db) {
-    if (greedy) {
-      accept = (x == rows[lane].argmax);
-    } else {
-      const RowRes& rq = rows[Dm + 1 + lane];
-      const double lp = (double)in.zt / Td - rows[lane].lse;
-      double lq = (double)in.zq / Td - rq.lse;
-      if (saguaro && lq != -INFINITY) {
-        bool in_k = false;
-        for (int i = 0; i < rq.ntop; ++i) in_k |= (rq.top[i] == x);
-        lq += (in_k ? log(c) : 0.0) - rq.lnZ;
-      }
-      double acc;
-      if (lp == -INFINITY)
-        acc = 0.0;  // p(x) = 0: the target never emits x
-      else if (lq == -INFINITY)
-        acc = 1.0;
-      else
-        acc = fmin(1.0, exp(lp - lq));
-      const double u = (double)(in.uw >> 8) * 0x1p-24;
-      accept = u < acc;
-      near = fabs(u - acc) < 1e-5;
-    }
-  }
+  if (lane < rp.Db) accept = accept_position(a, rp, rows, in, lane, &near);
   const uint32_t rej = __ballot_sync(0xFFFFFFFFu, lane < rp.Db && !accept);
   const int n = rej ? __ffs(rej) - 1 : rp.Db;
   const uint32_t nearm = __ballot_sync(0xFFFFFFFFu, near);

@@ -166,13 +166,18 @@ struct VerifyArgs {
   uint32_t request_offset;
   const int32_t* parents;  // tree verification: [B, D_max] parent position of each node; NULL: linear
   int32_t* out_nodes;      // tree verification: [B, D_max] accepted nodes (optional)
+  // early exit (early_exit.cu): rows are read position by position, only for
+  // requests that accepted every earlier draft
+  int* ee_n;               // [B] the decided position n (-1: parameter error); NULL: not used
+  int* ee_alive;           // [2, B] the requests still accepting, by round parity
+  unsigned int* ee_count;  // two counters 32 words apart: the lists' lengths
 };
 
 // Workspace layout (offsets in bytes from the workspace base, 256-aligned).
 // [zero, total) must read zero when a fused launch starts.
 struct WsLayout {
-  size_t pstat, tpart, rdesc, rpart, rorder, rowres, zero, rcount, best_key, rowcnt, reqcnt, pubq,
-      ctl, ticket, total;
+  size_t pstat, tpart, rdesc, rpart, rorder, rowres, ee, zero, rcount, best_key, rowcnt, reqcnt,
+      pubq, ctl, ticket, total;
 };
 
 constexpr int kCtlWords = 8 * 32;  // the fused kernel's control words, 32 words (128 B) apart
@@ -207,6 +212,8 @@ inline WsLayout ws_layout(int B, int D_max, int V, int dtype, bool saguaro) {
   off = align_up(off + (size_t)B * nseg * sizeof(unsigned short), 256);
   L.rowres = off;
   off = align_up(off + (size_t)B * slots * sizeof(RowRes), 256);
+  L.ee = off;  // early exit: decided positions [B], two alive lists [2, B], two counters
+  off = align_up(off + (size_t)3 * B * sizeof(int) + 3 * 128, 256);  // counters on 128 B lines
   // everything from here on reads zero when a fused launch starts
   L.zero = off;
   L.rcount = off;
@@ -380,6 +387,10 @@ int row_stats_blocks_per_sm(int dtype);
 cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
 int race_split(int B, int nseg, int dtype, int sms);
+// The early-exit rounds (early_exit.cu), before the usual finish with a.ee_n set.
+cudaError_t launch_early_exit_rounds(const VerifyArgs& a, cudaStream_t s, int grid);
+int ee_rounds(int D_max, int* bounds);
+
 // One CTA per request, or a cluster of 2 or 4 while B times that fits two CTAs
 // on each of the sms multiprocessors.
 cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s, int sms);

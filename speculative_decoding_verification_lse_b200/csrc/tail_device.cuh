@@ -34,6 +34,35 @@ struct TailShared {
   unsigned long long k0;  // the best exact key so far (per-request layout), as ordered bits
 };
 
+// The merged rows of request b into rows[0 .. slots), by the whole CTA: from
+// the segment partials, or -- after the early-exit rounds (a.ee_n set) -- from
+// the rows those rounds merged, the rows past the decided position n left
+// without statistics (never read by the scan's decisions: the first rejection
+// is at n, or n = D_b).  Ends with the CTA synchronised.
+__device__ __forceinline__ void gather_rows(const VerifyArgs& a, int b, const ReqParams& rp,
+                                            RowRes* rows) {
+  const int warp = threadIdx.x >> 5;
+  if (a.ee_n == nullptr) {
+    for (int slot = warp; slot < a.slots; slot += kWarps)
+      if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &rows[slot]);
+  } else {
+    const int n = a.ee_n[b];
+    for (int slot = threadIdx.x; slot < a.slots; slot += kThreads) {
+      const int d = slot <= a.D_max ? slot : slot - a.D_max - 1;
+      RowRes r;
+      if (d <= n) {
+        r = a.rowres[(size_t)b * a.slots + slot];
+      } else {
+        memset(&r, 0, sizeof r);
+        r.lse = NAN;
+        r.argmax = -1;
+      }
+      rows[slot] = r;
+    }
+  }
+  __syncthreads();
+}
+
 // The end of request b's race, by one warp: r is the combination of every
 // segment's result.  An empty residual ({p > q} empty through rounding) is
 // drawn from p on the same row instead; then the token and the flags are
@@ -67,9 +96,7 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
   const ReqParams rp = load_req(a, b);
   // the scan's inputs by the last warp (the fewest rows to merge), during the merges
   if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
-  for (int slot = warp; slot < a.slots; slot += kWarps)
-    if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
-  __syncthreads();
+  gather_rows(a, b, rp, S.rows);
   if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();
   const int kind = S.rd.kind;
@@ -128,9 +155,7 @@ __device__ __forceinline__ void tail_request_cluster(const VerifyArgs& a, int b,
   if (rank == 0) {
     const ReqParams rp = load_req(a, b);
     if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
-    for (int slot = warp; slot < a.slots; slot += kWarps)
-      if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
-    __syncthreads();
+    gather_rows(a, b, rp, S.rows);
     if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
     __syncthreads();
     if (S.rd.kind != kRaceNone) {
@@ -193,9 +218,7 @@ __device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared&
   const ReqParams rp = load_req(a, b);
   // the scan's inputs by the last warp (the fewest rows to merge), during the merges
   if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
-  for (int slot = warp; slot < a.slots; slot += kWarps)
-    if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
-  __syncthreads();
+  gather_rows(a, b, rp, S.rows);
   if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();
   const int kind = S.rd.kind;

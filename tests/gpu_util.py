@@ -110,10 +110,12 @@ def check_valid(w, b, got, ref_lse, seed):
         assert lp > logq(n, x), (b, x)
 
 
-def compare(w, got, ref):
+def compare(w, got, ref, early_exit=False):
     """Assert parity; return a summary.  Requests the oracle flags as near-ties
     are exempt from bit-exactness; their outputs are checked for validity
-    (check_valid) instead.  Offsets are not used: request b is global index b."""
+    (check_valid) instead.  Offsets are not used: request b is global index b.
+    early_exit: rows past the request's outcome may be unread (no LSE); those
+    up to it must have one."""
     reqs = ref["reqs"]
     D_list = w.row_D_list()
     lse_tol = LSE_TOL[w.dtype]
@@ -134,7 +136,15 @@ def compare(w, got, ref):
         r = ref["row_lse"][i]
         g = got["row_lse"][b].astype(np.float64)
         used = ~np.isnan(r)
-        assert np.array_equal(used, ~np.isnan(g)), (b, r, g)
+        if early_exit:
+            n = int(ref["accept_len"][i]) - 1
+            pos = np.array([s if s <= w.D_max else s - w.D_max - 1 for s in range(len(r))])
+            needed = used & (pos <= n)
+            assert np.all(~np.isnan(g[needed])), (b, g)
+            assert np.all(np.isnan(g[~used])), (b, g)
+            used = used & ~np.isnan(g)
+        else:
+            assert np.array_equal(used, ~np.isnan(g)), (b, r, g)
         if used.any():
             # relative to |LSE|, or absolute where |LSE| < 1 (relative error is ill-posed near 0)
             rel = np.abs(g[used] - r[used]) / np.maximum(np.abs(r[used]), 1.0)
