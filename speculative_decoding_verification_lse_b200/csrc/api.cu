@@ -362,6 +362,8 @@ int sv_verify_ex(const void* target_logits, const void* draft_logits,
     a.ee_n = (int*)((char*)ws + L.ee);
     a.ee_alive = a.ee_n + B;
     a.ee_count = (unsigned int*)((char*)ws + align_up(L.ee + (size_t)3 * B * sizeof(int), 128));
+    if ((e = cudaMemsetAsync(a.ticket, 0, 8 * 128, s)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync(ticket)");
     if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_early_exit_rounds(a, s, grid)) != cudaSuccess)
       return cuda_fail(e, "early-exit rounds launch");

@@ -51,8 +51,16 @@ __global__ void __launch_bounds__(kThreads, 3) ee_stats_kernel(VerifyArgs a, int
   const int nsl = 2 * (p1 - p0);
   const unsigned per_entry = (unsigned)nsl * (unsigned)a.nseg;
   const unsigned total = (unsigned)listed * per_entry;
-  const unsigned W = gridDim.x * kWarps;
-  for (unsigned i = blockIdx.x * kWarps + (threadIdx.x >> 5); i < total; i += W) {
+  // items from eight ticket counters (zero at launch), counter c handing out
+  // c, c + 8, ..., so that the warps that run ahead take more
+  const unsigned lane = threadIdx.x & 31;
+  const unsigned c = (blockIdx.x * kWarps + (threadIdx.x >> 5)) & 7u;
+  unsigned* ctr = a.ticket + 32 * c;
+  for (;;) {
+    unsigned i = 0;
+    if (lane == 0) i = atomicAdd(ctr, 1u) * 8u + c;
+    i = __shfl_sync(0xFFFFFFFFu, i, 0);
+    if (i >= total) break;
     const int k = (int)(i / per_entry);
     const unsigned rem = i % per_entry;
     const int j = (int)(rem / (unsigned)a.nseg), seg = (int)(rem % (unsigned)a.nseg);
@@ -68,9 +76,11 @@ __global__ void __launch_bounds__(kThreads, 3) ee_stats_kernel(VerifyArgs a, int
   allow_next_kernel();
 }
 
-// Round r's decisions, positions [p0, p1): CTA k takes list entry k.
+// Round r's decisions, positions [p0, p1): CTA k takes list entry k.  CTA 0
+// also zeroes the statistics tickets for the next round.
 __global__ void __launch_bounds__(kThreads) ee_step_kernel(VerifyArgs a, int r, int p0, int p1) {
   wait_for_previous_kernel();
+  if (blockIdx.x == 0 && threadIdx.x < 8) a.ticket[32 * threadIdx.x] = 0u;
   const int k = blockIdx.x;
   if (k >= ee_listed(a, r)) {
     allow_next_kernel();
