@@ -491,6 +491,41 @@ def run_ours(args):
     k_med = statistics.median(k_list)
     ms_per_step = ms / args.steps
     rows_total = w.verified_rows() * args.steps * world
+    graph = None
+    if args.graph > 0 and not tree:
+        # the same steps captured in a CUDA graph (one per input copy and seed,
+        # args.graph of them) and replayed: the per-launch host and dependency
+        # costs a decode loop saves by capturing its calls
+        K = args.graph
+        ws = torch.empty(sv.sv_workspace_bytes(w.B, w.D_max, w.V, w.dtype), dtype=torch.uint8,
+                         device=dev)
+        gs = torch.cuda.Stream(dev)
+        with torch.cuda.stream(gs):
+            sv.verify_workload(copies[0], seed=999, out=out, workspace=ws, stream=gs,
+                               variant=variant)
+        torch.cuda.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=gs):
+            for i in range(K):
+                sv.verify_workload(copies[i % ncopies], seed=1000 + i, out=out, workspace=ws,
+                                   stream=gs, variant=variant)
+        reps = max(1, args.steps // K)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(gs):
+            for _ in range(3):
+                cg.replay()
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+            g0.record(gs)
+            for _ in range(reps):
+                cg.replay()
+            g1.record(gs)
+        torch.cuda.synchronize()
+        gms = max_over_ranks(g0.elapsed_time(g1), dev)
+        graph = {"ms_per_step": gms / (reps * K), "steps_per_graph": K, "replays": reps,
+                 "value": w.verified_rows() * reps * K * world / (gms / 1e3), "unit": "rows/s"}
+        del cg
     ee_rows = None
     if args.variant == "early-exit" and not tree:
         # the rows the timed steps read, from their outcomes (each step again,
@@ -658,6 +693,8 @@ def run_ours(args):
             "e2e": e2e,
             "acceptance": acceptance,
         }
+        if graph is not None:
+            line["graph"] = graph
         if args.cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -677,6 +714,8 @@ def main():
     ap.add_argument("--variant", choices=["auto", "split", "split-items", "split-per-request",
                                           "fused", "cluster", "early-exit"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--graph", type=int, default=0,
+                    help="also time the steps captured K at a time in a CUDA graph")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)

@@ -230,7 +230,15 @@ SV_API int sv_verify_greedy(const void* target_logits, const int32_t* draft_toke
                      const int32_t* row_D, int B, int D_max, int V, int dtype,
                      int32_t* out_tokens, int32_t* out_accept_len);
 
-/* sv_verify with optional parameters (p may be NULL). */
+/* sv_verify with optional parameters (p may be NULL).
+ * CUDA graphs: every call only enqueues work on sv_params.stream, so a decode
+ * loop can capture its calls (with their epilogues) by stream capture and
+ * replay them; the seed and the pointers are fixed at capture.  Make one call
+ * on the device before capturing (the first call does one-time device
+ * queries), and pass sv_params.workspace, or capture only after a call of at
+ * least the same sizes (the cached workspace grows with cudaMalloc, which a
+ * capture does not allow).  sv_get_device_status synchronises: call it
+ * outside the graph. */
 SV_API int sv_verify_ex(const void* target_logits, const void* draft_logits,
                  const int32_t* draft_tokens, const int32_t* row_D, int B, int D_max, int V,
                  int dtype, float temperature, int mode, uint64_t seed, int32_t* out_tokens,
