@@ -96,6 +96,10 @@ __global__ void __launch_bounds__(kThreads) ee_step_kernel(VerifyArgs a, int r, 
     return;
   }
   RowRes* rows = a.rowres + (size_t)b * a.slots;
+  // the scan's inputs (draft tokens, their logits, the accept words) by the
+  // last warp while the others merge
+  __shared__ ScanInputs s_in[32];
+  if (warp == kWarps - 1) s_in[lane] = scan_inputs(a, b, rp);
   // the round's rows (a request is listed only while p0 <= D_b)
   const int dend = min(p1 - 1, rp.Db);  // the last position whose target row is read
   for (int j = warp; j < 2 * (dend - p0 + 1); j += kWarps) {
@@ -107,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) ee_step_kernel(VerifyArgs a, int r, 
   }
   __syncthreads();
   if (warp == 0) {
-    const ScanInputs in = scan_inputs(a, b, rp);
+    const ScanInputs in = s_in[lane];
     // rows without statistics, or inputs out of range: decided here, the scan reports it
     uint32_t err = in.err;
     for (int j = lane; j < 2 * (dend - p0 + 1); j += 32) {
