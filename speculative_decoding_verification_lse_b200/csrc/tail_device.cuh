@@ -63,6 +63,14 @@ __device__ __forceinline__ void gather_rows(const VerifyArgs& a, int b, const Re
   __syncthreads();
 }
 
+// The scan's inputs of request b into S.in, by the CTA's last warp: the draft
+// tokens, their logits and the accept words -- kernel inputs only, so the
+// tail kernels load them before they wait for the statistics kernel (while it
+// drains); the first barrier of gather_rows makes them visible.
+__device__ __forceinline__ void load_scan_inputs(const VerifyArgs& a, int b, ScanInputs* in) {
+  if ((threadIdx.x >> 5) == kWarps - 1) in[threadIdx.x & 31] = scan_inputs(a, b, load_req(a, b));
+}
+
 // The end of request b's race, by one warp: r is the combination of every
 // segment's result.  An empty residual ({p > q} empty through rounding) is
 // drawn from p on the same row instead; then the token and the flags are
@@ -89,13 +97,13 @@ __device__ __forceinline__ void finish_race(const VerifyArgs& a, int b, const Ra
 }
 
 // Request b, everything after its statistics, by the whole CTA (kThreads
-// threads, S in shared memory); every thread returns at the same point.
+// threads, S in shared memory; S.in holds the scan's inputs, which the kernel
+// loads before it waits for the statistics: load_scan_inputs); every thread
+// returns at the same point.
 template <int DT>
 __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailShared& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const ReqParams rp = load_req(a, b);
-  // the scan's inputs by the last warp (the fewest rows to merge), during the merges
-  if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
   gather_rows(a, b, rp, S.rows);
   if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();
@@ -139,7 +147,8 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
   __syncthreads();  // S is reused by the next request
 }
 
-// Request b by the C CTAs of a thread-block cluster (C > 1): rank 0 merges the
+// Request b by the C CTAs of a thread-block cluster (C > 1; rank 0's S.in as
+// for tail_request): rank 0 merges the
 // rows, runs the accept scan and finds the reference key, as tail_request
 // does; the other ranks copy its race description through distributed shared
 // memory, and the cluster's C * kWarps warps race the sampled row (warp w of
@@ -154,7 +163,6 @@ __device__ __forceinline__ void tail_request_cluster(const VerifyArgs& a, int b,
   const RaceStream R = race_stream(a.seed, a.request_offset + (uint32_t)b, (uint32_t)a.vocab_offset >> 2);
   if (rank == 0) {
     const ReqParams rp = load_req(a, b);
-    if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
     gather_rows(a, b, rp, S.rows);
     if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
     __syncthreads();
@@ -209,15 +217,14 @@ __device__ __forceinline__ void tail_request_cluster(const VerifyArgs& a, int b,
   cluster.sync();  // the other ranks' shared memory stays until rank 0 has read it
 }
 
-// Request b, by the whole CTA (kThreads threads, S in shared memory); every
-// thread returns at the same point.  Writes the request's outputs (all of them
-// unless it races), and for a race a.rdesc[b] and the race counters.
+// Request b, by the whole CTA (kThreads threads, S in shared memory; S.in as
+// for tail_request); every thread returns at the same point.  Writes the
+// request's outputs (all of them unless it races), and for a race a.rdesc[b]
+// and the race counters.
 template <int DT>
 __device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared& S) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const ReqParams rp = load_req(a, b);
-  // the scan's inputs by the last warp (the fewest rows to merge), during the merges
-  if (warp == kWarps - 1) S.in[lane] = scan_inputs(a, b, rp);
   gather_rows(a, b, rp, S.rows);
   if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();

@@ -20,6 +20,7 @@ namespace {
 template <int DT>
 __global__ void __launch_bounds__(kThreads) scan_kernel(VerifyArgs a) {
   __shared__ TailShared S;
+  load_scan_inputs(a, (int)blockIdx.x, S.in);
   wait_for_previous_kernel();
   scan_cta<DT>(a, (int)blockIdx.x, S);
   allow_next_kernel();
@@ -28,6 +29,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(VerifyArgs a) {
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) request_kernel(VerifyArgs a) {
   __shared__ TailShared S;
+  load_scan_inputs(a, (int)blockIdx.x, S.in);
   wait_for_previous_kernel();
   tail_request<DT>(a, (int)blockIdx.x, S);
 }
@@ -38,8 +40,10 @@ __global__ void __launch_bounds__(kThreads, 2) request_cluster_kernel(VerifyArgs
   __shared__ TailShared S;
   __shared__ Best rb;
   cg::cluster_group cluster = cg::this_cluster();
+  const int b = (int)(blockIdx.x / cluster.num_blocks());
+  if (cluster.block_rank() == 0) load_scan_inputs(a, b, S.in);
   wait_for_previous_kernel();
-  tail_request_cluster<DT>(a, (int)(blockIdx.x / cluster.num_blocks()), S, cluster, &rb);
+  tail_request_cluster<DT>(a, b, S, cluster, &rb);
 }
 
 template <int DT>
