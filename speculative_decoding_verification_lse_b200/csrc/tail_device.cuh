@@ -148,13 +148,13 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
 }
 
 // Request b by the C CTAs of a thread-block cluster (C > 1; rank 0's S.in as
-// for tail_request): rank 0 merges the
-// rows, runs the accept scan and finds the reference key, as tail_request
-// does; the other ranks copy its race description through distributed shared
-// memory, and the cluster's C * kWarps warps race the sampled row (warp w of
-// rank r taking segments 8r + w, 8r + w + 8C, ...); rank 0 combines the ranks'
-// results in rank order and writes the token.  rb: this CTA's slot for its
-// result.  Every thread of the cluster returns at the same point.
+// for tail_request): rank 0 merges the rows, runs the accept scan and finds the
+// reference key, as tail_request does; the other ranks copy its race
+// description through distributed shared memory, and the cluster's C * kWarps
+// warps race the sampled row (warp w of rank r taking segments 8r + w,
+// 8r + w + 8C, ...); rank 0 combines the ranks' results in rank order and
+// writes the token.  rb: this CTA's slot for its result.  Every thread of the
+// cluster returns at the same point.
 template <int DT, class Cluster>
 __device__ __forceinline__ void tail_request_cluster(const VerifyArgs& a, int b, TailShared& S,
                                                      Cluster& cluster, Best* rb) {
