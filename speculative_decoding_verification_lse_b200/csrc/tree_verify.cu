@@ -47,6 +47,11 @@ struct TreeShared {
   double red[kWarps];
   double part[2];  // this CTA's partial of the residual pass, by pass parity
   Best rb;         // this CTA's race result
+  // node i's token logits in its parent position's target and draft rows, and
+  // its accept word (loaded before the walk, so that its decisions wait on no
+  // memory)
+  float zt[kMaxDraft], zq[kMaxDraft];
+  uint32_t uw[kMaxDraft];
 };
 
 // sum over the row of max(0, p(x) - c q(x)) for target row pos and draft row
@@ -124,16 +129,20 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
   const int32_t* par = a.parents + (size_t)b * Dm;
   int32_t* ot = a.out_tokens + (size_t)b * (Dm + 1);
 
-  for (int slot = warp; slot < a.slots; slot += kWarps)
-    if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
   if (warp == kWarps - 1) {
-    // errors: parameters, nodes (token range, parent order), unreadable rows
+    // errors: parameters, nodes (token range, parent order), unreadable rows;
+    // and the nodes' inputs, while the other warps merge the rows
     uint32_t err = rp.err | (rp.mode == kSaguaro ? kFlagBadParam : 0u);
     if (!rp.err)
       for (int i = lane; i < rp.Db; i += 32) {
         const int x = __ldg(&tok[i]), pi = __ldg(&par[i]);
         if (x < 0 || x >= a.V_global) err |= kFlagBadToken;
         if (pi < 0 || pi > i) err |= kFlagBadParam;
+        if (x >= 0 && x < a.V && pi >= 0 && pi <= i && rp.mode != kGreedy) {
+          T.zt[i] = logit_at<DT>(row_base(a, b, pi), x);
+          T.zq[i] = logit_at<DT>(row_base(a, b, Dm + 1 + pi), x);
+          T.uw[i] = accept_word(a.seed, g, (uint32_t)i);
+        }
       }
     err = __reduce_or_sync(0xFFFFFFFFu, err);
     if (lane == 0) {
@@ -143,6 +152,8 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
       T.done = 0;
     }
   }
+  for (int slot = warp; slot < a.slots; slot += kWarps)
+    if (slot_needed(a, b, slot, rp)) merge_row_into(a, b, slot, rp, &S.rows[slot]);
   __syncthreads();
   if (!T.flags) {
     // rows the walk may read that hold NaN, +inf or no finite entry
@@ -227,9 +238,8 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
       }
       any = 1;
       if (threadIdx.x == 0) {
-        const int x = __ldg(&tok[i]);
-        const double lp = (double)logit_at<DT>(row_base(a, b, pos), x) / Td - lse_t;
-        const double lq = (double)logit_at<DT>(row_base(a, b, Dm + 1 + pos), x) / Td - lse_q;
+        const double lp = (double)T.zt[i] / Td - lse_t;
+        const double lq = (double)T.zq[i] / Td - lse_q;
         double acc;
         if (T.c == 0.0) {
           // P = p: the linear rule's ratio
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
           else
             acc = fmin(1.0, r / (T.N * exp(lq)));
         }
-        const uint32_t uw = accept_word(a.seed, g, (uint32_t)i);
+        const uint32_t uw = T.uw[i];
         const double u = (double)(uw >> 8) * 0x1p-24;
         if (fabs(u - acc) < 1e-5) T.flags |= kFlagAcceptNearTie;
         T.emitted = u < acc ? i : -1;
