@@ -42,8 +42,9 @@ def _call(fn, w, seed, variant):
     return {k: v.cpu().numpy() for k, v in out.items()}
 
 
-@pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED, sv.SV_VARIANT_CLUSTER],
-                         ids=["split", "fused", "cluster"])
+@pytest.mark.parametrize("variant", [sv.SV_VARIANT_SPLIT, sv.SV_VARIANT_FUSED, sv.SV_VARIANT_CLUSTER,
+                                     sv.SV_VARIANT_EARLY_EXIT],
+                         ids=["split", "fused", "cluster", "early-exit"])
 @pytest.mark.parametrize("name", ["b256", "ragged", "saguaro", "tiny"])
 def test_static_entry_point_matches_the_ordinary_one(variant, name):
     sv.load()
