@@ -202,6 +202,10 @@ typedef struct sv_params {
                                         the step sv_epilogue describes, on this call's
                                         out_tokens / out_accept_len (and out_flags, which get
                                         SV_FLAG_SEQ_FULL); host struct, read during the call */
+  const uint64_t* seed_device;       /* optional device pointer: the seed is read from here when
+                                        the kernels run (the `seed` argument is then unused), so
+                                        that a captured graph draws new numbers on each replay
+                                        once the value is advanced (sv_advance_seed) */
 } sv_params;
 
 /*
@@ -233,7 +237,9 @@ SV_API int sv_verify_greedy(const void* target_logits, const int32_t* draft_toke
 /* sv_verify with optional parameters (p may be NULL).
  * CUDA graphs: every call only enqueues work on sv_params.stream, so a decode
  * loop can capture its calls (with their epilogues) by stream capture and
- * replay them; the seed and the pointers are fixed at capture.  Make one call
+ * replay them; the pointers are fixed at capture, and so is the seed unless
+ * it is read from sv_params.seed_device, which a captured sv_advance_seed can
+ * advance between the calls so that each replay draws new numbers.  Make one call
  * on the device before capturing (the first call does one-time device
  * queries), and pass sv_params.workspace, or capture only after a call of at
  * least the same sizes (the cached workspace grows with cudaMalloc, which a
@@ -396,6 +402,12 @@ SV_API int sv_shard_race(const void* target_local, const void* draft_local,
                          int32_t* out_tokens, int32_t* out_accept_len, void* exchange2);
 SV_API int sv_shard_finish(int B, int D_max, int n_shards, const void* gathered2,
                            int32_t* out_tokens, const sv_params* p);
+
+/* Enqueues *seed_device += by on `stream` (cudaStream_t, NULL = legacy
+ * default): between captured verification calls that read their seed from
+ * sv_params.seed_device, so that each replay of a graph draws new numbers.
+ * seed_device: device pointer, 8-byte aligned.  SV_ERR_INVALID_ARG for NULL. */
+SV_API int sv_advance_seed(uint64_t* seed_device, uint64_t by, void* stream);
 
 /* Bytes of scratch one call with these sizes needs (for sv_params.workspace). */
 SV_API size_t sv_workspace_bytes(int B, int D_max, int V, int dtype);

@@ -69,6 +69,7 @@ class SvParams(ctypes.Structure):
         ("timing_events", ctypes.c_void_p),
         ("out_draft_top", ctypes.c_void_p),
         ("epilogue", ctypes.POINTER(SvEpilogueArgs)),
+        ("seed_device", ctypes.c_void_p),
     ]
 
 
@@ -131,6 +132,8 @@ def load(build_if_needed=True):
         ctypes.c_float, ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_void_p, ctypes.POINTER(SvParams)]
     L.sv_verify_tree.restype = ctypes.c_int
+    L.sv_advance_seed.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p]
+    L.sv_advance_seed.restype = ctypes.c_int
     L.sv_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.sv_workspace_bytes.restype = ctypes.c_size_t
     L.sv_get_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]
@@ -247,7 +250,8 @@ def sv_verify_tree(target_logits, draft_logits, node_tokens, parents, n_nodes, B
 
 def verify_tree(target, draft, tokens, parents, n_nodes=None, *, temperature=1.0,
                 mode=SV_STOCHASTIC, seed=0, temperature_per_req=None, mode_per_req=None,
-                request_offset=0, stream=None, row_lse=False, timing_events=None):
+                request_offset=0, stream=None, row_lse=False, timing_events=None,
+                seed_device=None):
     """Tree verification of a batch held in CUDA tensors (sv_verify_tree):
     target [B, N+1, V], draft [B, N, V] (or None when greedy), tokens and parents
     [B, N] int32, n_nodes [B] int32 or None.  Returns dict(tokens, accept_len,
@@ -275,6 +279,7 @@ def verify_tree(target, draft, tokens, parents, n_nodes=None, *, temperature=1.0
     prm.request_offset = int(request_offset)
     prm.out_flags = _p(out["flags"])
     prm.out_row_lse = _p(out.get("row_lse"))
+    prm.seed_device = _seed_device_ptr(seed_device)
     if timing_events is not None:
         arr = (ctypes.c_void_p * 2)(timing_events[0].cuda_event, timing_events[1].cuda_event)
         prm.timing_events = ctypes.cast(arr, ctypes.c_void_p)
@@ -283,6 +288,13 @@ def verify_tree(target, draft, tokens, parents, n_nodes=None, *, temperature=1.0
                               float(temperature), int(mode), int(seed), out["tokens"],
                               out["accept_len"], out["nodes"], prm))
     return out
+
+
+def sv_advance_seed(seed_device, by=1, stream=None):
+    """Enqueue seed_device += by (a CUDA uint64/int64 tensor of one element, or
+    a device pointer) on `stream`: between the captured calls of a graph whose
+    calls read their seed from it (verify(..., seed_device=...))."""
+    _check(load().sv_advance_seed(_p(seed_device), int(by) & (2**64 - 1), _stream_ptr(stream)))
 
 
 def sv_workspace_bytes(B, D_max, V, dtype):
@@ -317,6 +329,15 @@ def _stream_ptr(stream):
     return stream.cuda_stream
 
 
+def _seed_device_ptr(t):
+    import torch
+    if t is None or isinstance(t, int):
+        return t
+    if not t.is_cuda or t.numel() != 1 or t.element_size() != 8 or t.dtype.is_floating_point:
+        raise ValueError("seed_device must be a one-element 64-bit integer CUDA tensor")
+    return t.data_ptr()
+
+
 def _dtype_code(t):
     import torch
     if t.dtype == torch.float32:
@@ -329,13 +350,17 @@ def _dtype_code(t):
 def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHASTIC, seed=0,
            temperature_per_req=None, mode_per_req=None, saguaro_k=5, saguaro_c=0.5,
            request_offset=0, variant=SV_VARIANT_AUTO, stream=None, row_lse=False,
-           out=None, workspace=None, timing_events=None, epilogue=None, draft_top=False):
+           out=None, workspace=None, timing_events=None, epilogue=None, draft_top=False,
+           seed_device=None):
     """Verify a batch held in CUDA tensors; returns dict(tokens, accept_len, flags
     [, row_lse]) as CUDA tensors, enqueued on `stream` (not synchronised).
     epilogue: optional dict(window, next_window, seq, seq_len) of int32 CUDA
     tensors (any may be None) for the on-device step after verification
     (sv_epilogue), run on the same stream.  draft_top: also return the k
-    largest logits of each saguaro draft row (sv_params.out_draft_top)."""
+    largest logits of each saguaro draft row (sv_params.out_draft_top).
+    seed_device: optional CUDA int64/uint64 tensor of one element whose value
+    the kernels read as the seed (sv_params.seed_device; `seed` is then
+    unused), for CUDA graphs that advance it between replays."""
     import torch
     if not target.is_cuda:
         raise ValueError("target logits must be a CUDA tensor (there is no CPU path)")
@@ -375,6 +400,7 @@ def verify(target, draft, tokens, row_D=None, *, temperature=1.0, mode=SV_STOCHA
     prm.out_row_lse = _p(out.get("row_lse"))
     prm.out_flags = _p(out.get("flags"))
     prm.out_draft_top = _p(out.get("draft_top"))
+    prm.seed_device = _seed_device_ptr(seed_device)
     if workspace is not None:
         prm.workspace = _p(workspace)
         prm.workspace_bytes = workspace.numel() * workspace.element_size()

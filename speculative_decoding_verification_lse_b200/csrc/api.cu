@@ -262,6 +262,7 @@ int prepare_call(const void* target_logits, const void* draft_logits,
   a.pubq = (unsigned int*)((char*)ws + L.pubq);
   a.ctl = (unsigned int*)((char*)ws + L.ctl);
   a.seed = seed;
+  a.seed_ptr = prm.seed_device;
   a.B = B;
   a.D_max = D_max;
   a.V = V;
@@ -304,6 +305,15 @@ extern "C" {
 int sv_version(void) { return 10000; }
 
 const char* sv_last_error(void) { return g_last_error.c_str(); }
+
+int sv_advance_seed(uint64_t* seed_device, uint64_t by, void* stream) {
+  g_last_error.clear();
+  if (seed_device == nullptr || (uintptr_t)seed_device % 8 != 0)
+    return fail(SV_ERR_INVALID_ARG, "sv_advance_seed: seed_device must be an 8-byte aligned device pointer");
+  cudaError_t e = launch_advance_seed(seed_device, by, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sv_advance_seed launch");
+  return SV_OK;
+}
 
 size_t sv_workspace_bytes(int B, int D_max, int V, int dtype) {
   if (B < 0 || D_max < 0 || V < 1 || (dtype != SV_F32 && dtype != SV_BF16)) return 0;

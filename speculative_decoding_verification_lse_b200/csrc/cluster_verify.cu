@@ -53,7 +53,7 @@ __device__ void cluster_scan(const VerifyArgs& a, int b, const ReqParams& rp, Ta
   if (warp == 0) scan_request(a, b, S.rows, &S.rd, S.in[lane]);
   __syncthreads();
   if (S.rd.kind != kRaceNone) {
-    const RaceStream R = race_stream(a.seed, S.rd.g, (uint32_t)a.vocab_offset >> 2);
+    const RaceStream R = race_stream(seed_of(a), S.rd.g, (uint32_t)a.vocab_offset >> 2);
     const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
     if (lane == 0) S.key[warp] = kw;
     __syncthreads();
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 2) cluster_kernel(VerifyArgs a) {
     const bool residual = kind == kRaceResidual;
     const char* trow = row_base(a, b, S.rd.n);
     const char* qrow = residual ? row_base(a, b, a.D_max + 1 + S.rd.n) : nullptr;
-    const RaceStream R = race_stream(a.seed, S.rd.g, (uint32_t)a.vocab_offset >> 2);
+    const RaceStream R = race_stream(seed_of(a), S.rd.g, (uint32_t)a.vocab_offset >> 2);
     const Best B = race_span_in<DT>(a, S.rd, R, trow, qrow, residual, gw, nw, S.rd.K0, &S.k0);
     if (lane == 0) {
       RacePart p;

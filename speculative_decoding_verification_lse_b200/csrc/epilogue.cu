@@ -132,4 +132,16 @@ cudaError_t launch_epilogue(const int32_t* window, const int32_t* out_tokens,
   return cudaLaunchKernelEx(&cfg, epilogue_kernel, e);
 }
 
+namespace {
+
+__global__ void advance_seed_kernel(uint64_t* seed, uint64_t by) { *seed += by; }
+
+}  // namespace
+
+// *seed += by on stream s (sv_advance_seed).
+cudaError_t launch_advance_seed(uint64_t* seed, uint64_t by, cudaStream_t s) {
+  advance_seed_kernel<<<1, 1, 0, s>>>(seed, by);
+  return cudaGetLastError();
+}
+
 }  // namespace sv

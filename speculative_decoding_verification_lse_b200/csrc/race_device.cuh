@@ -70,7 +70,7 @@ struct RowCtx {
 
 __device__ __forceinline__ RowCtx row_ctx(const VerifyArgs& a) {
   RowCtx c;
-  c.seed = a.seed;
+  c.seed = seed_of(a);
   c.dtype = a.dtype;
   c.V = a.V;
   c.nvec = a.nvec;
@@ -79,6 +79,8 @@ __device__ __forceinline__ RowCtx row_ctx(const VerifyArgs& a) {
 }
 
 __device__ __forceinline__ RowCtx row_ctx(const RowCtx& c) { return c; }
+
+__device__ __forceinline__ uint64_t seed_of(const RowCtx& c) { return c.seed; }
 
 __device__ __forceinline__ Best combine(const Best& A, const Best& C) {
   const bool c_wins =
@@ -158,7 +160,7 @@ __device__ __forceinline__ double exact_key_of(const A& a, const RaceDesc& rd,
   float zq = 0.0f;
   if (residual) zq = (a.dtype == kF32) ? logit_at<kF32>(qrow, x) : logit_at<kBF16>(qrow, x);
   const int gx = x + a.vocab_offset;  // the token's global index (Philox counter, saguaro K)
-  return exact_key(zt, zq, gx, race_word(a.seed, rd.g, gx), rd, residual);
+  return exact_key(zt, zq, gx, race_word(seed_of(a), rd.g, gx), rd, residual);
 }
 
 constexpr double kRaceBand = 1e-5;  // delta: the 1e-6 near-tie band plus every rounding error
@@ -337,7 +339,7 @@ static __device__ __noinline__ float key2_upper(const RowCtx a, const RaceDesc& 
       h = hl + fabsf(hl) * 0x1p-21f + 0x1p-40f;
     }
   }
-  const uint32_t o = race_word(a.seed, rd.g, x + a.vocab_offset);
+  const uint32_t o = race_word(seed_of(a), rd.g, x + a.vocab_offset);
   const float lw = log2f((float)o + 0.5f);
   const float nlw = 32.0f - lw + fabsf(lw) * 0x1p-21f + 0x1p-20f;
   const float sum = l2p + h + nlw;
@@ -540,7 +542,7 @@ __device__ __forceinline__ Best race_part(const VerifyArgs& a, const RaceDesc& r
     const float cup = filter_offset(K, rd.lse_t);
     const float thr2 = K > -INFINITY ? __double2float_rd((K - kRaceBand) * 1.4426950408889634 - 1e-5)
                                      : -INFINITY;
-    uint32_t keep = ~word_filter_compact<DT>(cur, gi * QV, a.seed, rd.g,
+    uint32_t keep = ~word_filter_compact<DT>(cur, gi * QV, seed_of(a), rd.g,
                                              (uint32_t)a.vocab_offset >> 2, v0, rd.k2, cup);
     // exact keys of the survivors, one token per lane at a time
     while (__any_sync(0xFFFFFFFFu, keep != 0u)) {
@@ -567,7 +569,7 @@ template <int DT>
 __device__ __noinline__ Best race_segment(const RowCtx a, const RaceDesc& rd,
                                           const char* trow, const char* qrow, bool residual,
                                           int seg, double K0, float cup) {
-  return race_segment_in<DT>(a, rd, race_stream(a.seed, rd.g, (uint32_t)a.vocab_offset >> 2), trow, qrow, residual, seg, K0, cup);
+  return race_segment_in<DT>(a, rd, race_stream(seed_of(a), rd.g, (uint32_t)a.vocab_offset >> 2), trow, qrow, residual, seg, K0, cup);
 }
 
 // A quick approximate key (natural-log units) with the hardware's approximate

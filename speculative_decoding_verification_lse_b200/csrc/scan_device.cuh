@@ -180,7 +180,7 @@ __device__ __forceinline__ ScanInputs scan_inputs(const VerifyArgs& a, int b, co
     } else if (rp.mode != kGreedy) {
       in.zt = load_logit(a, row_base(a, b, lane), in.x);
       in.zq = load_logit(a, row_base(a, b, a.D_max + 1 + lane), in.x);
-      in.uw = accept_word(a.seed, a.request_offset + (uint32_t)b, (uint32_t)lane);
+      in.uw = accept_word(seed_of(a), a.request_offset + (uint32_t)b, (uint32_t)lane);
     }
   }
   return in;

@@ -72,7 +72,7 @@ __device__ __forceinline__ ScanInputs shard_scan_inputs(const VerifyArgs& a, int
                               (size_t)b * a.D_max + lane);
       in.zt = z.x;
       in.zq = z.y;
-      in.uw = accept_word(a.seed, a.request_offset + (uint32_t)b, (uint32_t)lane);
+      in.uw = accept_word(seed_of(a), a.request_offset + (uint32_t)b, (uint32_t)lane);
     }
   }
   return in;
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 2) shard_tail_kernel(VerifyArgs a, c
     const bool residual = kind == kRaceResidual;
     const char* trowp = row_base(a, b, S.rd.n);
     const char* qrowp = residual ? row_base(a, b, Dm + 1 + S.rd.n) : nullptr;
-    const RaceStream R = race_stream(a.seed, S.rd.g, (uint32_t)a.vocab_offset >> 2);
+    const RaceStream R = race_stream(seed_of(a), S.rd.g, (uint32_t)a.vocab_offset >> 2);
     for (int pass = 0; pass < 2; ++pass) {
       // pass 0: the race of kind; pass 1: the bonus race, when no column here
       // is a residual candidate

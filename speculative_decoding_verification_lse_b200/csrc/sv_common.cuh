@@ -168,6 +168,7 @@ struct VerifyArgs {
   int32_t* out_nodes;      // tree verification: [B, D_max] accepted nodes (optional)
   // early exit (early_exit.cu): rows are read position by position, only for
   // requests that accepted every earlier draft
+  const uint64_t* seed_ptr;  // the seed in device memory, read by the kernels instead of `seed`; or NULL
   int* ee_n;               // [B] the decided position n (-1: parameter error); NULL: not used
   int* ee_alive;           // [2, B] the requests still accepting, by round parity
   unsigned int* ee_count;  // two counters 32 words apart: the lists' lengths
@@ -329,6 +330,12 @@ struct ReqParams {
   uint32_t err;  // kFlagBadRowD / kFlagBadParam found in the parameters
 };
 
+// The call's seed: from device memory when the caller keeps it there (so that
+// a captured graph draws new numbers each replay), else the argument.
+__device__ __forceinline__ uint64_t seed_of(const VerifyArgs& a) {
+  return a.seed_ptr != nullptr ? *a.seed_ptr : a.seed;
+}
+
 __device__ __forceinline__ ReqParams load_req(const VerifyArgs& a, int b) {
   ReqParams r;
   r.Db = a.row_D ? __ldg(&a.row_D[b]) : a.D_max;
@@ -387,6 +394,9 @@ int row_stats_blocks_per_sm(int dtype);
 cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s);
 cudaError_t launch_race(const VerifyArgs& a, cudaStream_t s);
 int race_split(int B, int nseg, int dtype, int sms);
+// *seed += by on stream s (epilogue.cu; sv_advance_seed).
+cudaError_t launch_advance_seed(uint64_t* seed, uint64_t by, cudaStream_t s);
+
 // The early-exit rounds (early_exit.cu), before the usual finish with a.ee_n set.
 cudaError_t launch_early_exit_rounds(const VerifyArgs& a, cudaStream_t s, int grid);
 int ee_rounds(int D_max, int* bounds);

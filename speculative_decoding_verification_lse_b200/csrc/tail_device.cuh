@@ -115,7 +115,7 @@ __device__ __forceinline__ void tail_request(const VerifyArgs& a, int b, TailSha
 
   // the reference key, from the segment holding the sampled row's largest logit
   // (the request's Philox stream from kernel arguments, the same on every thread)
-  const RaceStream R = race_stream(a.seed, a.request_offset + (uint32_t)b, (uint32_t)a.vocab_offset >> 2);
+  const RaceStream R = race_stream(seed_of(a), a.request_offset + (uint32_t)b, (uint32_t)a.vocab_offset >> 2);
   const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
   if (lane == 0) S.key[warp] = kw;
   if (threadIdx.x == 0) S.k0 = ordered_u64(-INFINITY);
@@ -160,7 +160,7 @@ __device__ __forceinline__ void tail_request_cluster(const VerifyArgs& a, int b,
                                                      Cluster& cluster, Best* rb) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
-  const RaceStream R = race_stream(a.seed, a.request_offset + (uint32_t)b, (uint32_t)a.vocab_offset >> 2);
+  const RaceStream R = race_stream(seed_of(a), a.request_offset + (uint32_t)b, (uint32_t)a.vocab_offset >> 2);
   if (rank == 0) {
     const ReqParams rp = load_req(a, b);
     gather_rows(a, b, rp, S.rows);
@@ -232,7 +232,7 @@ __device__ __forceinline__ void scan_cta(const VerifyArgs& a, int b, TailShared&
   if (kind != kRaceNone) {
     // the reference key: each warp ranks a share of the segment holding the
     // sampled row's largest logit and takes the exact key of its best token
-    const RaceStream R = race_stream(a.seed, S.rd.g, (uint32_t)a.vocab_offset >> 2);
+    const RaceStream R = race_stream(seed_of(a), S.rd.g, (uint32_t)a.vocab_offset >> 2);
     // the sampled row's segment maxima, for the race order, load while the
     // reference key is searched
     const bool ranked = a.nseg <= kThreads;
@@ -302,7 +302,7 @@ __device__ __forceinline__ void race_item(const VerifyArgs& a, long long item, R
   const char* qrow = residual ? row_base(a, b, a.D_max + 1 + rd->n) : nullptr;
   const unsigned long long bk = *(volatile unsigned long long*)&a.best_key[b];
   const double K = fmax(rd->K0, bk ? from_ordered_u64(bk) : -INFINITY);
-  const Best sb = race_segment_in<DT>(a, *rd, race_stream(a.seed, rd->g, (uint32_t)a.vocab_offset >> 2), trow, qrow, residual,
+  const Best sb = race_segment_in<DT>(a, *rd, race_stream(seed_of(a), rd->g, (uint32_t)a.vocab_offset >> 2), trow, qrow, residual,
                                       seg, K, filter_offset(K, rd->lse_t), h * NG / a.rsplit,
                                       (h + 1) * NG / a.rsplit);
   unsigned prev = 0;

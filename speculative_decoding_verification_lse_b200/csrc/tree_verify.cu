@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
         if (x >= 0 && x < a.V && pi >= 0 && pi <= i && rp.mode != kGreedy) {
           T.zt[i] = logit_at<DT>(row_base(a, b, pi), x);
           T.zq[i] = logit_at<DT>(row_base(a, b, Dm + 1 + pi), x);
-          T.uw[i] = accept_word(a.seed, g, (uint32_t)i);
+          T.uw[i] = accept_word(seed_of(a), g, (uint32_t)i);
         }
       }
     err = __reduce_or_sync(0xFFFFFFFFu, err);
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 2) tree_kernel(VerifyArgs a) {
       S.k0 = ordered_u64(-INFINITY);
     }
     __syncthreads();
-    const RaceStream R = race_stream(a.seed, g, (uint32_t)a.vocab_offset >> 2);
+    const RaceStream R = race_stream(seed_of(a), g, (uint32_t)a.vocab_offset >> 2);
     const double kw = race_ref_key_warp<DT>(a, S.rd, R, b, S.rd.ref_seg, warp, kWarps);
     if (lane == 0) S.key[warp] = kw;
     __syncthreads();

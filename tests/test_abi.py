@@ -132,6 +132,15 @@ def test_null_pointers_are_rejected_on_the_host(lib):
     assert rc == sv.SV_ERR_INVALID_ARG and "aligned" in sv.sv_last_error()
 
 
+def test_seed_advance_rejects_bad_pointers_on_the_host(lib):
+    L = sv.load()
+    assert L.sv_advance_seed(None, 1, None) == sv.SV_ERR_INVALID_ARG
+    assert "seed_device" in sv.sv_last_error()
+    assert L.sv_advance_seed((1 << 20) + 4, 1, None) == sv.SV_ERR_INVALID_ARG
+    with pytest.raises(sv.SvError):
+        sv.sv_advance_seed(None)
+
+
 def test_empty_batch_is_a_no_op(lib):
     assert sv.sv_verify(None, None, None, None, 0, 3, 100, sv.SV_BF16, 1.0, sv.SV_STOCHASTIC, 0,
                         None, None) == sv.SV_OK

@@ -98,3 +98,62 @@ def test_captured_decode_loop_with_the_epilogue(sv):
     # the sequences grew by the accepted lengths of the three steps
     grown = sum(al.to(torch.int64) for al in b[3])
     assert torch.equal(b[2].to(torch.int64), len0.cpu().to(torch.int64) + grown)
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", dict(mode=1)), ("tiny", dict(mode=2)),
+                                     ("b32", dict(B=16, V=30011)),
+                                     ("saguaro", dict(B=24, V=20008))])
+@pytest.mark.parametrize("variant", [sv.SV_VARIANT_AUTO, sv.SV_VARIANT_FUSED,
+                                     sv.SV_VARIANT_EARLY_EXIT])
+def test_seed_read_from_device_memory_equals_seed_argument(sv, name, kw, variant):
+    w = wl.make(name, "cuda", **kw)
+    for sd in (0, 7, 2**64 - 3):
+        sdev = torch.tensor([sd - 2**64 if sd >= 2**63 else sd], dtype=torch.int64, device="cuda")
+        got = sv.verify_workload(w, seed=12345, seed_device=sdev, variant=variant)
+        ref = sv.verify_workload(w, seed=sd, variant=variant)
+        torch.cuda.synchronize()
+        for k in ("tokens", "accept_len", "flags"):
+            assert torch.equal(got[k], ref[k]), (name, sd, k)
+
+
+def test_tree_seed_read_from_device_memory(sv):
+    w = wl.make_tree("tree", "cuda", B=20, V=12011, branching=(3, 2, 2))
+    sdev = torch.tensor([99], dtype=torch.int64, device="cuda")
+    args = (w.target, w.draft, w.tokens, w.parents)
+    got = sv.verify_tree(*args, temperature=w.temperature, mode=w.mode, seed=5, seed_device=sdev)
+    ref = sv.verify_tree(*args, temperature=w.temperature, mode=w.mode, seed=99)
+    torch.cuda.synchronize()
+    for k in ("tokens", "accept_len", "nodes", "flags"):
+        assert torch.equal(got[k], ref[k]), k
+
+
+def test_graph_replays_draw_new_numbers_with_an_advanced_seed(sv):
+    # three steps captured once, each followed by seed += 1 on the device: the
+    # first replay draws with seeds S, S+1, S+2, the second with S+3 .. S+5
+    w = wl.make("b32", "cuda", B=16, V=30011)
+    ws = torch.empty(sv.sv_workspace_bytes(w.B, w.D_max, w.V, w.dtype), dtype=torch.uint8,
+                     device="cuda")
+    S = 1000
+    sdev = torch.tensor([S], dtype=torch.int64, device="cuda")
+    s = torch.cuda.Stream()
+    outs = [_out(w) for _ in range(3)]
+    with torch.cuda.stream(s):
+        sv.verify_workload(w, seed=0, out=_out(w), workspace=ws, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for o in outs:
+            sv.verify_workload(w, out=o, workspace=ws, stream=s, seed_device=sdev)
+            sv.sv_advance_seed(sdev, 1, stream=s)
+    assert int(sdev.item()) == S  # nothing ran during the capture
+    for rep in range(2):
+        with torch.cuda.stream(s):
+            g.replay()
+        torch.cuda.synchronize()
+        assert int(sdev.item()) == S + 3 * (rep + 1)
+        for i, o in enumerate(outs):
+            ref = sv.verify_workload(w, seed=S + 3 * rep + i)
+            torch.cuda.synchronize()
+            for k in ("tokens", "accept_len", "flags"):
+                assert torch.equal(o[k], ref[k]), (rep, i, k)
+    assert sv.sv_get_device_status() == 0
