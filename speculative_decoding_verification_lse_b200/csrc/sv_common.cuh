@@ -402,9 +402,10 @@ cudaError_t launch_early_exit_rounds(const VerifyArgs& a, cudaStream_t s, int gr
 int ee_rounds(int D_max, int* bounds);
 
 // One CTA per request, or a cluster of 2 or 4 while B times that fits two CTAs
-// on each of the sms multiprocessors.
+// on each of the sms multiprocessors and the row has a segment for each of
+// the cluster's warps.
 cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s, int sms);
-int request_cluster_size(int B, int sms);
+int request_cluster_size(int B, int nseg, int sms);
 cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid);
 int fused_blocks_per_sm(int dtype, int slots);
 int fused_race_sm_every(const VerifyArgs& a, int grid);

@@ -82,16 +82,17 @@ cudaError_t launch_scan(const VerifyArgs& a, cudaStream_t s) {
 }
 
 // A cluster of C = 4 or 2 CTAs per request while B C fits two CTAs per
-// multiprocessor (sms of them), else one CTA per request.
-int request_cluster_size(int B, int sms) {
+// multiprocessor (sms of them) and the row has a segment for every warp of
+// the cluster (nseg of them), else one CTA per request.
+int request_cluster_size(int B, int nseg, int sms) {
   int C = 4;
-  while (C > 1 && (long long)B * C > 2LL * sms) C /= 2;
+  while (C > 1 && ((long long)B * C > 2LL * sms || C * kWarps > nseg)) C /= 2;
   return C;
 }
 
 cudaError_t launch_requests(const VerifyArgs& a, cudaStream_t s, int sms) {
   if (a.B == 0) return cudaSuccess;
-  const int C = request_cluster_size(a.B, sms);
+  const int C = request_cluster_size(a.B, a.nseg, sms);
   if (C == 1)
     return a.dtype == kF32 ? launch_dependent(request_kernel<kF32>, a.B, s, a)
                            : launch_dependent(request_kernel<kBF16>, a.B, s, a);
