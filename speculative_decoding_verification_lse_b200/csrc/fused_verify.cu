@@ -304,6 +304,10 @@ cudaError_t launch_fused(const VerifyArgs& a, cudaStream_t s, int grid) {
     fn = top ? (const void*)fused_kernel<kF32, true> : (const void*)fused_kernel<kF32, false>;
   else
     fn = top ? (const void*)fused_kernel<kBF16, true> : (const void*)fused_kernel<kBF16, false>;
+  // the kernel's dynamic shared memory limit is one attribute for every draft
+  // length, last set by whichever occupancy query ran last: set it for this one
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kThreads), params, smem, s);
 }
 

@@ -50,6 +50,16 @@ def test_draft_lengths(sv, D, variant):
 
 
 @VARIANTS
+def test_draft_lengths_long_short_long(sv, variant):
+    # each draft length gets its own launch shape (the fused kernel's shared
+    # memory grows with it): a long draft, a short one, then a new long one
+    # must each launch and match the oracle, whatever was launched before
+    for D, seed in ((12, 41), (1, 42), (11, 43), (12, 44)):
+        w = make_random(5, D, 2500, seed=seed)
+        compare(w, gpu_run(w, variant=variant), oracle_on(w))
+
+
+@VARIANTS
 def test_row_D_with_zero_and_nan_padding(sv, variant):
     w = make_random(8, 5, 5000, seed=3)
     row_D = torch.tensor([0, 5, 1, 0, 3, 5, 2, 4], dtype=torch.int32, device="cuda")
