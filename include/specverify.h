@@ -406,7 +406,12 @@ SV_API int sv_shard_finish(int B, int D_max, int n_shards, const void* gathered2
 /* Enqueues *seed_device += by on `stream` (cudaStream_t, NULL = legacy
  * default): between captured verification calls that read their seed from
  * sv_params.seed_device, so that each replay of a graph draws new numbers.
- * seed_device: device pointer, 8-byte aligned.  SV_ERR_INVALID_ARG for NULL. */
+ * seed_device: device pointer, 8-byte aligned, owned by the caller.
+ * SV_ERR_INVALID_ARG for NULL or a misaligned pointer; SV_ERR_CUDA if the
+ * launch fails.  No passage of the pages defines this call: it serves decode
+ * loops that replay the verification step of "Accélérer Sonar par la
+ * Spéculation" (section "Inférence avec décodage spéculatif": the step runs
+ * once per generated window) from a captured graph. */
 SV_API int sv_advance_seed(uint64_t* seed_device, uint64_t by, void* stream);
 
 /* Bytes of scratch one call with these sizes needs (for sv_params.workspace). */
