@@ -103,8 +103,12 @@ def test_captured_decode_loop_with_the_epilogue(sv):
 @pytest.mark.parametrize("name,kw", [("tiny", dict(mode=1)), ("tiny", dict(mode=2)),
                                      ("b32", dict(B=16, V=30011)),
                                      ("saguaro", dict(B=24, V=20008))])
-@pytest.mark.parametrize("variant", [sv.SV_VARIANT_AUTO, sv.SV_VARIANT_FUSED,
-                                     sv.SV_VARIANT_EARLY_EXIT])
+@pytest.mark.parametrize("variant", [sv.SV_VARIANT_AUTO,
+                                     sv.SV_VARIANT_SPLIT | sv.SV_TAIL_PER_REQUEST,
+                                     sv.SV_VARIANT_SPLIT | sv.SV_TAIL_ITEMS,
+                                     sv.SV_VARIANT_FUSED, sv.SV_VARIANT_CLUSTER,
+                                     sv.SV_VARIANT_EARLY_EXIT],
+                         ids=["auto", "per-request", "items", "fused", "cluster", "early-exit"])
 def test_seed_read_from_device_memory_equals_seed_argument(sv, name, kw, variant):
     w = wl.make(name, "cuda", **kw)
     for sd in (0, 7, 2**64 - 3):
