@@ -76,9 +76,10 @@ class VocabShardCall:
     def __init__(self, target_local, draft_local, tokens, row_D=None, *, n_shards, shard,
                  temperature=1.0, mode=0, seed=0, temperature_per_req=None, mode_per_req=None,
                  saguaro_k=5, saguaro_c=0.5, request_offset=0, stream=None, row_lse=False,
-                 draft_top=False):
+                 draft_top=False, seed_device=None):
         import torch
-        from . import SvParams, _dtype_code, _p, _stream_ptr, sv_shard_exchange_bytes
+        from . import (SvParams, _dtype_code, _p, _seed_device_ptr, _stream_ptr,
+                       sv_shard_exchange_bytes)
         B, Dp1, Vl = target_local.shape
         D = Dp1 - 1
         dt = _dtype_code(target_local)
@@ -90,6 +91,7 @@ class VocabShardCall:
         prm.saguaro_k = int(saguaro_k)
         prm.saguaro_c = float(saguaro_c)
         prm.request_offset = int(request_offset)
+        prm.seed_device = _seed_device_ptr(seed_device)
         out = dict(tokens=torch.empty((B, D + 1), dtype=torch.int32, device=dev),
                    accept_len=torch.empty((B,), dtype=torch.int32, device=dev),
                    flags=torch.empty((B,), dtype=torch.int32, device=dev))

@@ -78,3 +78,19 @@ def test_full_size_eight_shards(sv):
     same = np.mean(np.all(outs[0]["tokens"] == flat["tokens"], axis=1))
     assert same >= 0.99
     assert sv.sv_get_device_status() & sv.SV_FLAG_ERRORS == 0
+
+
+def test_sharded_seed_read_from_device_memory(sv):
+    # the seed in device memory (sv_params.seed_device) reaches every stage
+    w = wl.make("b32", "cuda", B=8, V=20011)
+    sdev = torch.tensor([77], dtype=torch.int64, device="cuda")
+    got = verify_vocab_parallel_in_one_process(
+        w.target, w.draft, w.tokens, w.row_D, n_shards=3, temperature=w.temperature,
+        mode=w.mode, seed=5, seed_device=sdev)
+    ref = verify_vocab_parallel_in_one_process(
+        w.target, w.draft, w.tokens, w.row_D, n_shards=3, temperature=w.temperature,
+        mode=w.mode, seed=77)
+    torch.cuda.synchronize()
+    for g, r in zip(got, ref):
+        for k in ("tokens", "accept_len", "flags"):
+            assert torch.equal(g[k], r[k]), k
