@@ -153,6 +153,18 @@ def test_no_cpu_path_in_the_binding():
         sv.verify(t, t[:, :1], torch.zeros((1, 1), dtype=torch.int32))
 
 
+def test_device_seed_must_be_a_64_bit_integer_cuda_tensor():
+    import torch
+    from speculative_decoding_verification_lse_b200 import _seed_device_ptr
+    assert _seed_device_ptr(None) is None
+    assert _seed_device_ptr(1 << 20) == 1 << 20  # a raw device address passes through
+    # host tensors (this test needs no GPU), of the right and of wrong shapes and types
+    for bad in (torch.zeros(1, dtype=torch.int64), torch.zeros(2, dtype=torch.int64),
+                torch.zeros(1, dtype=torch.float64), torch.zeros(1, dtype=torch.int32)):
+        with pytest.raises(ValueError, match="seed_device"):
+            _seed_device_ptr(bad)
+
+
 def test_product_never_imports_the_oracle():
     pkg = os.path.join(ROOT, "speculative_decoding_verification_lse_b200")
     for dirpath, _, files in os.walk(pkg):
